@@ -1,0 +1,211 @@
+/*
+ * bitlinear.h — C ABI of the B200 (sm_100a) BitNet b1.58 BitLinear forward.
+ *
+ * The operations follow the blog post "BitNet b1.58 — quantização ternária,
+ * BitLinear, Zero-GEMM" (BLOG below) and the API names of "Arquitetura
+ * Hibrida Multimodal para bitnet.cpp", section utils/ — bit_layers.py
+ * (quantise_weights_ternary, quantise_activations_8bit, BitLinear,
+ * ReLUSquared).
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ *  * Tensors are row-major and contiguous. Activations A are [M, K]
+ *    (tokens × in-features); weights W are [N, K] (out × in, the nn.Linear
+ *    layout); outputs Y are [M, N]. The layer computes Y = f(A · Wᵀ).
+ *  * Every pointer argument, unless stated otherwise, is a DEVICE pointer to
+ *    memory the caller owns. The library never allocates, frees or keeps
+ *    pointers after the call returns. Scratch memory ("workspace") is passed
+ *    in by the caller; its size comes from the matching *_workspace_bytes().
+ *  * Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and makes no host synchronisation. Scales
+ *    (γ, γ_A) are passed by device pointer for the same reason.
+ *  * Pointers must be 16-byte aligned. K must be a positive multiple of 64;
+ *    M, N ≥ 0 (M == 0 or N == 0 is a no-op returning BL_OK). eps must be
+ *    finite and > 0. NaN/Inf inputs are outside the contract (not checked).
+ *  * Errors are returned, never thrown or aborted: argument errors are found
+ *    on the host before any launch (nothing is launched then); launch errors
+ *    map to BL_ERR_CUDA. Device-side waits are bounded: a wait that gives up
+ *    raises a per-device error flag, read (and cleared) by
+ *    bl_check_device_error().
+ *  * The device must be sm_100 (B200); otherwise BL_ERR_UNSUPPORTED.
+ *
+ * Packed ternary weight format (this library's; the BLOG, section "Como o
+ * BitNet quebra o Memory Wall...", fixes only "2 bits per weight"):
+ *  * code c = w + 1 ∈ {0, 1, 2} for w ∈ {-1, 0, +1}; 3 is never written;
+ *  * a row of K weights is K/16 little-endian 32-bit words (K/4 bytes),
+ *    rows are contiguous: the packed matrix is [N, K/4] bytes;
+ *  * within word g of a row, weight k = 16·g + 4·j + i (i, j ∈ 0..3) sits in
+ *    bits 8·i + 2·j and 8·i + 2·j + 1.
+ *  So (word >> 2·j) & 0x03030303 holds the codes of weights 16g+4j .. 16g+4j+3
+ *  as four bytes in natural order.
+ */
+#ifndef BITLINEAR_H_
+#define BITLINEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BL_OK = 0,
+  BL_ERR_INVALID_ARG = 1, /* null pointer, bad eps, bad flag or dtype value */
+  BL_ERR_SHAPE = 2,       /* negative size, K not a positive multiple of 64,
+                             size too large for the kernels' index types */
+  BL_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+  BL_ERR_DTYPE = 4,       /* dtype not allowed for this argument */
+  BL_ERR_CUDA = 5,        /* a CUDA runtime/driver call or launch failed */
+  BL_ERR_TIMEOUT = 6,     /* a device-side bounded wait gave up */
+  BL_ERR_UNSUPPORTED = 7, /* current device is not sm_100 */
+  BL_ERR_WORKSPACE = 8    /* workspace missing or smaller than required */
+} bl_status;
+
+typedef enum { BL_F32 = 0, BL_BF16 = 1 } bl_dtype;
+
+/* cudaStream_t-compatible handle (cudaStream_t is struct CUstream_st*). */
+typedef struct CUstream_st* bl_stream_t;
+
+/* Flags for the *_ex entry points. */
+enum {
+  /* Launch with programmatic dependent launch: the kernel streams its packed
+   * weights into shared memory BEFORE waiting for the previous kernel on the
+   * stream, and lets the next kernel start early. Only valid when the weight
+   * buffer was NOT written by the kernel immediately preceding this call on
+   * `stream` (true for a decode chain over static weights). Activations and
+   * outputs are still ordered after the previous kernel. */
+  BL_FLAG_PDL = 1
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* bl_status_string(bl_status s);
+
+/* Library ABI version (major*100 + minor). */
+int bl_version(void);
+
+/* Number of decoded tokens up to which bl_linear uses the fused GEMV path. */
+int bl_gemv_max_tokens(void);
+
+/* ---------------------------------------------------------------------------
+ * bl_quant_weights — quantise_weights_ternary.
+ * BLOG, section "Por que 1,58 bits por peso e qual a matemática da
+ * ternarização?": γ = (1/(N·K)) Σ|W_ij| over the whole matrix;
+ * W_q = Round(Clip(W / (γ+ε), -1, 1)) ∈ {-1, 0, +1}, Round = half-to-even.
+ *   W         [N, K] fp32 or bf16 (w_dtype), device.
+ *   W_packed  [N, K/4] bytes, device, written in the packed format above.
+ *   gamma     1 fp32, device, written with γ (sum in double, rounded once).
+ *   workspace ≥ bl_quant_weights_workspace_bytes(N, K) bytes, device.
+ * The code decision equals the fp32 division W ÷ (γ+ε) followed by
+ * round-half-to-even, exactly.
+ */
+size_t bl_quant_weights_workspace_bytes(int64_t N, int64_t K);
+bl_status bl_quant_weights(const void* W, bl_dtype w_dtype, int64_t N, int64_t K,
+                           float eps, uint8_t* W_packed, float* gamma,
+                           void* workspace, size_t ws_bytes, bl_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * bl_quant_acts — quantise_activations_8bit.
+ * BLOG, same section, activation paragraph: per token m,
+ * γ_A[m] = max_k |A[m,k]|; A_q = Clip(Round(A · (127 / (γ_A+ε))), -128, 127),
+ * taken in fp32 (127/(γ_A+ε) by IEEE division, then one fp32 product).
+ *   A       [M, K] fp32 or bf16, device.
+ *   A_q     [M, K] int8, device.
+ *   gamma_A [M] fp32, device.
+ *   rowsum  [M] int32, device, optional (NULL to skip): Σ_k A_q[m,k], the
+ *           term the contraction kernels subtract to undo the +1 code
+ *           offset; pass it on to bl_linear_q to save one pass.
+ */
+bl_status bl_quant_acts(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
+                        float eps, int8_t* A_q, float* gamma_A, int32_t* rowsum,
+                        bl_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * bl_zero_gemm — the INT32 contraction alone.
+ * BLOG, section "Como funciona a camada BitLinear e a eliminação de
+ * multiplicações (Zero-GEMM)?": acc[m,n] = Σ_k W_q[n,k]·A_q[m,k] (add on +1,
+ * subtract on -1, skip on 0), INT32 accumulation.
+ *   A_q [M, K] int8; W_packed [N, K/4]; acc [M, N] int32 (all device).
+ *   workspace ≥ bl_zero_gemm_workspace_bytes(M, K, N).
+ */
+size_t bl_zero_gemm_workspace_bytes(int64_t M, int64_t K, int64_t N);
+bl_status bl_zero_gemm(const int8_t* A_q, int64_t M, int64_t K,
+                       const uint8_t* W_packed, int64_t N, int32_t* acc,
+                       void* workspace, size_t ws_bytes, bl_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * bl_linear_q — contraction + dequantisation from already-quantised tokens.
+ * BLOG, Zero-GEMM section, last paragraph: Y = (A_q·W_qᵀ) · (γ_A·γ)/127, one
+ * scalar per (token, matrix); with relu2 != 0, Y = max(Y, 0)² (ReLUSquared).
+ * The scale is taken in fp32 as (γ_A[m]·γ)/127 (no ε, as the page writes it).
+ *   A_q [M, K] int8; gamma_A [M] fp32; rowsum [M] int32 or NULL (then it is
+ *   recomputed into the workspace); W_packed [N, K/4]; gamma 1 fp32;
+ *   Y [M, N] fp32 or bf16 (y_dtype; bf16 rounds to nearest even).
+ *   workspace ≥ bl_linear_q_workspace_bytes(M, K, N).
+ */
+size_t bl_linear_q_workspace_bytes(int64_t M, int64_t K, int64_t N);
+bl_status bl_linear_q(const int8_t* A_q, const float* gamma_A,
+                      const int32_t* rowsum, int64_t M, int64_t K,
+                      const uint8_t* W_packed, const float* gamma, int64_t N,
+                      int relu2, void* Y, bl_dtype y_dtype, void* workspace,
+                      size_t ws_bytes, bl_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * bl_linear — BitLinear forward from float activations:
+ * bl_quant_acts, bl_zero_gemm and the dequantisation of bl_linear_q in one
+ * call. For M ≤ bl_gemv_max_tokens() it is a single fused GEMV launch (the
+ * activation quantiser runs in the kernel prologue; no workspace needed);
+ * above that, an activation-quantiser launch and a tensor-core launch.
+ *   A [M, K] fp32/bf16; W_packed [N, K/4]; gamma 1 fp32; Y [M, N] fp32/bf16.
+ *   workspace ≥ bl_linear_workspace_bytes(M, K, N) (may be 0 → NULL ok).
+ * bl_linear_ex adds `flags` (BL_FLAG_PDL; only honoured on the GEMV path).
+ */
+size_t bl_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
+bl_status bl_linear(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
+                    const uint8_t* W_packed, const float* gamma, int64_t N,
+                    float eps, int relu2, void* Y, bl_dtype y_dtype,
+                    void* workspace, size_t ws_bytes, bl_stream_t stream);
+bl_status bl_linear_ex(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
+                       const uint8_t* W_packed, const float* gamma, int64_t N,
+                       float eps, int relu2, void* Y, bl_dtype y_dtype,
+                       void* workspace, size_t ws_bytes, unsigned flags,
+                       bl_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * bl_ffn_relu2 — ternary FFN block (BitLinear up → ReLU² → BitLinear down).
+ * Composition of the BLOG formulas with ReLUSquared (bit_layers.py): per
+ * token, h = dequantised up-projection (fp32), r = max(h,0)² (fp32), AbsMax
+ * requantisation of r with the activation rule above (γ_r = max_n r), then
+ * the down-projection dequantised with (γ_r·γ_down)/127.
+ *   X [M, K] fp32/bf16; W_up [H, K/4]; gamma_up 1 fp32;
+ *   W_down [K_out=K, H/4]; gamma_down 1 fp32; Y [M, K] fp32/bf16.
+ *   H must be a positive multiple of 64.
+ *   workspace ≥ bl_ffn_workspace_bytes(M, K, H).
+ */
+size_t bl_ffn_workspace_bytes(int64_t M, int64_t K, int64_t H);
+bl_status bl_ffn_relu2(const void* X, bl_dtype x_dtype, int64_t M, int64_t K,
+                       int64_t H, const uint8_t* W_up, const float* gamma_up,
+                       const uint8_t* W_down, const float* gamma_down,
+                       float eps, void* Y, bl_dtype y_dtype, void* workspace,
+                       size_t ws_bytes, bl_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Device error flag. Synchronises `stream`, then returns BL_ERR_TIMEOUT if
+ * any kernel of this library on the current device gave up a bounded wait
+ * since the last check (and clears the flag), BL_ERR_CUDA if the stream
+ * reports an error, else BL_OK.
+ */
+bl_status bl_check_device_error(bl_stream_t stream);
+
+/* Self-test of the bounded-wait machinery: launches one tiny kernel that
+ * waits on a shared-memory barrier nothing will ever complete, giving up
+ * after `limit_ns` nanoseconds (1e3 .. 1e9), which raises the device error
+ * flag. Used by the test-suite to exercise the timeout path without hanging
+ * or faulting a GPU. */
+bl_status bl_selftest_wait_timeout(int64_t limit_ns, bl_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H_ */

@@ -1,0 +1,191 @@
+"""BitNet b1.58 BitLinear forward on B200 (sm_100a): Python binding.
+
+Thin marshalling layer over the C ABI of ``libbitlinear.so``
+(``include/bitlinear.h``): each function has the name of the C entry point,
+takes CUDA ``torch.Tensor`` arguments, allocates outputs and workspace with
+torch, and passes raw device pointers plus the current CUDA stream. Every
+computation happens in the library's CUDA kernels; there is no fallback.
+
+Method: "BitNet b1.58 — quantização ternária, BitLinear, Zero-GEMM" (AbsMean
+ternary weights, AbsMax per-token INT8 activations, INT32 add/subtract/skip
+contraction, dequantisation by γ·γ_A/127) with the API names of the
+utils/bit_layers.py library of "Arquitetura Hibrida Multimodal para
+bitnet.cpp" (quantise_weights_ternary, quantise_activations_8bit, BitLinear,
+ReLUSquared).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+from ._lib import BL_BF16, BL_F32, BL_FLAG_PDL, BitLinearError, check, load
+
+__all__ = [
+    "bl_quant_weights", "bl_quant_acts", "bl_zero_gemm", "bl_linear_q", "bl_linear",
+    "bl_ffn_relu2", "bl_check_device_error", "bl_selftest_wait_timeout",
+    "bl_gemv_max_tokens", "workspace_bytes", "BitLinearError", "load", "BL_FLAG_PDL",
+]
+
+_DT = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _dt(t: torch.Tensor, what: str) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"{what}: dtype {t.dtype} not supported (float32 or bfloat16)")
+    return _DT[t.dtype]
+
+
+def _cuda(t: torch.Tensor, what: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{what} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    return t
+
+
+def _ws(nbytes: int, device) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def bl_gemv_max_tokens() -> int:
+    return int(load().bl_gemv_max_tokens())
+
+
+def workspace_bytes(op: str, M: int, K: int, N: int) -> int:
+    """Workspace size for 'quant_weights', 'zero_gemm', 'linear_q', 'linear'
+    or 'ffn' (for 'ffn', N is the hidden size H)."""
+    L = load()
+    if op == "quant_weights":
+        return int(L.bl_quant_weights_workspace_bytes(N, K))
+    return int(getattr(L, f"bl_{op}_workspace_bytes" if op != "ffn" else "bl_ffn_workspace_bytes")(M, K, N))
+
+
+def bl_quant_weights(W: torch.Tensor, eps: float = 1e-5, *, out=None, gamma=None,
+                     workspace=None, stream=None):
+    """quantise_weights_ternary: W [N, K] fp32/bf16 → (packed uint8 [N, K/4], γ fp32 [1])."""
+    _cuda(W, "W")
+    N, K = W.shape
+    if out is None:
+        out = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    if gamma is None:
+        gamma = torch.empty((1,), dtype=torch.float32, device=W.device)
+    L = load()
+    if workspace is None:
+        workspace = _ws(int(L.bl_quant_weights_workspace_bytes(N, K)), W.device)
+    check(L.bl_quant_weights(W.data_ptr(), _dt(W, "W"), N, K, float(eps), out.data_ptr(),
+                             gamma.data_ptr(), _ptr(workspace), _nbytes(workspace),
+                             _stream(stream)), "bl_quant_weights")
+    return out, gamma
+
+
+def bl_quant_acts(A: torch.Tensor, eps: float = 1e-5, *, rowsum: bool = True, stream=None):
+    """quantise_activations_8bit: A [M, K] → (A_q int8 [M,K], γ_A fp32 [M], Σ A_q int32 [M] or None)."""
+    _cuda(A, "A")
+    M, K = A.shape
+    Aq = torch.empty((M, K), dtype=torch.int8, device=A.device)
+    gA = torch.empty((M,), dtype=torch.float32, device=A.device)
+    rs = torch.empty((M,), dtype=torch.int32, device=A.device) if rowsum else None
+    check(load().bl_quant_acts(A.data_ptr(), _dt(A, "A"), M, K, float(eps), Aq.data_ptr(),
+                               gA.data_ptr(), _ptr(rs), _stream(stream)), "bl_quant_acts")
+    return Aq, gA, rs
+
+
+def bl_zero_gemm(A_q: torch.Tensor, W_packed: torch.Tensor, *, stream=None):
+    """INT32 contraction acc[M, N] = A_q · W_qᵀ."""
+    _cuda(A_q, "A_q")
+    _cuda(W_packed, "W_packed")
+    M, K = A_q.shape
+    N = W_packed.shape[0]
+    if W_packed.shape[1] * 4 != K:
+        raise ValueError("W_packed must be [N, K/4]")
+    acc = torch.empty((M, N), dtype=torch.int32, device=A_q.device)
+    L = load()
+    ws = _ws(int(L.bl_zero_gemm_workspace_bytes(M, K, N)), A_q.device)
+    check(L.bl_zero_gemm(A_q.data_ptr(), M, K, W_packed.data_ptr(), N, acc.data_ptr(), _ptr(ws),
+                         _nbytes(ws), _stream(stream)), "bl_zero_gemm")
+    return acc
+
+
+def bl_linear_q(A_q, gamma_A, W_packed, gamma, *, rowsum=None, relu2=False,
+                out_dtype=torch.bfloat16, out=None, stream=None):
+    """Y = (A_q·W_qᵀ)·(γ_A·γ)/127 (ReLU² optional) from int8 tokens."""
+    for t, n in ((A_q, "A_q"), (gamma_A, "gamma_A"), (W_packed, "W_packed"), (gamma, "gamma")):
+        _cuda(t, n)
+    M, K = A_q.shape
+    N = W_packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=A_q.device)
+    L = load()
+    ws = None if rowsum is not None else _ws(int(L.bl_linear_q_workspace_bytes(M, K, N)), A_q.device)
+    check(L.bl_linear_q(A_q.data_ptr(), gamma_A.data_ptr(), _ptr(rowsum), M, K,
+                        W_packed.data_ptr(), gamma.data_ptr(), N, int(bool(relu2)),
+                        out.data_ptr(), _dt(out, "out"), _ptr(ws), _nbytes(ws),
+                        _stream(stream)), "bl_linear_q")
+    return out
+
+
+def bl_linear(A, W_packed, gamma, eps: float = 1e-5, *, relu2=False, out_dtype=torch.bfloat16,
+              out=None, workspace=None, pdl=False, stream=None):
+    """BitLinear forward: Y [M, N] = dequant(quant(A) · W_qᵀ), ReLU² optional."""
+    _cuda(A, "A")
+    _cuda(W_packed, "W_packed")
+    _cuda(gamma, "gamma")
+    M, K = A.shape
+    N = W_packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    L = load()
+    if workspace is None:
+        workspace = _ws(int(L.bl_linear_workspace_bytes(M, K, N)), A.device)
+    check(L.bl_linear_ex(A.data_ptr(), _dt(A, "A"), M, K, W_packed.data_ptr(), gamma.data_ptr(),
+                         N, float(eps), int(bool(relu2)), out.data_ptr(), _dt(out, "out"),
+                         _ptr(workspace), _nbytes(workspace), BL_FLAG_PDL if pdl else 0,
+                         _stream(stream)), "bl_linear")
+    return out
+
+
+def bl_ffn_relu2(X, W_up, gamma_up, W_down, gamma_down, eps: float = 1e-5, *,
+                 out_dtype=torch.bfloat16, out=None, workspace=None, stream=None):
+    """Ternary FFN block: BitLinear up (K→H), ReLU², per-token requant, BitLinear down (H→K)."""
+    for t, n in ((X, "X"), (W_up, "W_up"), (gamma_up, "gamma_up"), (W_down, "W_down"),
+                 (gamma_down, "gamma_down")):
+        _cuda(t, n)
+    M, K = X.shape
+    H = W_up.shape[0]
+    if W_up.shape[1] * 4 != K or W_down.shape[0] != K or W_down.shape[1] * 4 != H:
+        raise ValueError("W_up must be [H, K/4] and W_down [K, H/4]")
+    if out is None:
+        out = torch.empty((M, K), dtype=out_dtype, device=X.device)
+    L = load()
+    if workspace is None:
+        workspace = _ws(int(L.bl_ffn_workspace_bytes(M, K, H)), X.device)
+    check(L.bl_ffn_relu2(X.data_ptr(), _dt(X, "X"), M, K, H, W_up.data_ptr(), gamma_up.data_ptr(),
+                         W_down.data_ptr(), gamma_down.data_ptr(), float(eps), out.data_ptr(),
+                         _dt(out, "out"), _ptr(workspace), _nbytes(workspace), _stream(stream)),
+          "bl_ffn_relu2")
+    return out
+
+
+def bl_check_device_error(stream=None) -> int:
+    """Synchronise the stream; return the library status (0 = BL_OK)."""
+    return int(load().bl_check_device_error(_stream(stream)))
+
+
+def bl_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    check(load().bl_selftest_wait_timeout(int(limit_ns), _stream(stream)),
+          "bl_selftest_wait_timeout")

@@ -1,0 +1,720 @@
+// C-ABI entry points of libbitlinear: argument checks, workspace layout,
+// kernel selection and launches. See include/bitlinear.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "bitlinear.h"
+#include "bl_device.cuh"
+#include "gemv_kernel.cuh"
+#include "quant_kernels.cuh"
+#include "tc_gemm_kernel.cuh"
+
+namespace bl {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kAbsmeanMaxBlocks = 1024;
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define BL_TRY(expr)                 \
+  do {                               \
+    bl_status _s = (expr);           \
+    if (_s != BL_OK) return _s;      \
+  } while (0)
+
+#define BL_CUDA(expr)                          \
+  do {                                         \
+    cudaError_t _e = (expr);                   \
+    if (_e != cudaSuccess) return BL_ERR_CUDA; \
+  } while (0)
+
+// --------------------------------------------------------------------------
+// Per-device state: architecture check and the number of SMs.
+struct DeviceInfo {
+  int checked = 0;
+  int ok = 0;
+  int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+bl_status current_device(int* dev_out, int* sms_out) {
+  int dev = 0;
+  BL_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return BL_ERR_UNSUPPORTED;
+  DeviceInfo& d = g_dev[dev];
+  if (!d.checked) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!d.checked) {
+      int major = 0, minor = 0, sms = 0;
+      BL_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+      BL_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+      BL_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+      d.ok = (major == 10 && minor == 0);
+      d.sms = sms;
+      d.checked = 1;
+    }
+  }
+  if (!d.ok) return BL_ERR_UNSUPPORTED;
+  *dev_out = dev;
+  if (sms_out) *sms_out = d.sms;
+  return BL_OK;
+}
+
+// Opt a kernel into large dynamic shared memory, once per (kernel, device).
+template <typename F>
+bl_status ensure_smem(F* kernel, int dev, size_t bytes) {
+  struct Entry {
+    const void* fn;
+    int dev;
+    size_t bytes;
+  };
+  static Entry cache[512];
+  static int n = 0;
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (int i = 0; i < n; ++i)
+    if (cache[i].fn == (const void*)kernel && cache[i].dev == dev && cache[i].bytes >= bytes)
+      return BL_OK;
+  BL_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
+  if (n < 512) cache[n++] = Entry{(const void*)kernel, dev, bytes};
+  return BL_OK;
+}
+
+// --------------------------------------------------------------------------
+// Tensor maps (TMA descriptors) through the driver entry point, so the
+// library does not link libcuda directly.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static int tried = 0;
+  if (!tried) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!tried) {
+      void* p = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+              cudaSuccess &&
+          q == cudaDriverEntryPointSuccess)
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+      tried = 1;
+    }
+  }
+  return fn;
+}
+
+// 2-D uint8 tensor [rows, cols] (cols contiguous), box {box_cols, box_rows}.
+bl_status make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                      uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return BL_ERR_CUDA;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? BL_OK : BL_ERR_CUDA;
+}
+
+// --------------------------------------------------------------------------
+// Argument checks.
+bl_status check_k(int64_t K) {
+  if (K <= 0 || K % 64 != 0) return BL_ERR_SHAPE;
+  if (K > ((int64_t)1 << 30)) return BL_ERR_SHAPE;
+  return BL_OK;
+}
+bl_status check_rows(int64_t R) {
+  if (R < 0 || R > ((int64_t)1 << 31) - 1) return BL_ERR_SHAPE;
+  return BL_OK;
+}
+bl_status check_eps(float eps) {
+  if (!(eps > 0.0f) || !std::isfinite(eps)) return BL_ERR_INVALID_ARG;
+  return BL_OK;
+}
+bl_status check_ptr(const void* p) {
+  if (p == nullptr) return BL_ERR_INVALID_ARG;
+  if (!aligned16(p)) return BL_ERR_ALIGN;
+  return BL_OK;
+}
+bl_status check_dtype(int d) {
+  if (d != BL_F32 && d != BL_BF16) return BL_ERR_DTYPE;
+  return BL_OK;
+}
+
+// --------------------------------------------------------------------------
+// Workspace layouts (offsets are multiples of 256 bytes).
+struct ActWs {
+  size_t aq, gamma, rowsum, total;
+};
+ActWs act_ws(int64_t M, int64_t K) {
+  ActWs w;
+  w.aq = 0;
+  w.gamma = align_up((size_t)M * K);
+  w.rowsum = w.gamma + align_up((size_t)M * 4);
+  w.total = w.rowsum + align_up((size_t)M * 4);
+  return w;
+}
+
+struct FfnWs {
+  ActWs x;        // quantised X (M > GEMV limit)
+  size_t acc_up;  // int32 [M, H]
+  size_t gamma_x; // [M] (GEMV path)
+  size_t rq;      // int8 [M, H]
+  size_t gamma_r, rs_r, total;
+};
+FfnWs ffn_ws(int64_t M, int64_t K, int64_t H) {
+  FfnWs w{};
+  if (M <= kGemvMaxTokens) {
+    w.acc_up = 0;
+    w.gamma_x = align_up((size_t)M * H * 4);
+    w.total = w.gamma_x + align_up((size_t)M * 4);
+    return w;
+  }
+  w.x = act_ws(M, K);
+  w.acc_up = w.x.total;
+  w.rq = w.acc_up + align_up((size_t)M * H * 4);
+  w.gamma_r = w.rq + align_up((size_t)M * H);
+  w.rs_r = w.gamma_r + align_up((size_t)M * 4);
+  w.total = w.rs_r + align_up((size_t)M * 4);
+  return w;
+}
+
+// --------------------------------------------------------------------------
+// GEMV launches.
+template <int MT, int RPL, typename TA, int SRC, int OUT>
+bl_status launch_gemv_t(const GemvParams& p, int grid, size_t smem, bool pdl, int dev,
+                        cudaStream_t st) {
+  auto* k = gemv_ternary_kernel<MT, RPL, TA, SRC, OUT>;
+  BL_TRY(ensure_smem(k, dev, smem));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  BL_CUDA(cudaLaunchKernelEx(&cfg, k, p));
+  return BL_OK;
+}
+
+template <int MT, typename TA, int SRC, int OUT>
+bl_status launch_gemv_rpl(const GemvParams& p, int rpl, int grid, size_t smem, bool pdl, int dev,
+                          cudaStream_t st) {
+  switch (rpl) {
+    case 1: return launch_gemv_t<MT, 1, TA, SRC, OUT>(p, grid, smem, pdl, dev, st);
+    case 2: return launch_gemv_t<MT, 2, TA, SRC, OUT>(p, grid, smem, pdl, dev, st);
+    case 3: return launch_gemv_t<MT, 3, TA, SRC, OUT>(p, grid, smem, pdl, dev, st);
+    default: return launch_gemv_t<MT, 4, TA, SRC, OUT>(p, grid, smem, pdl, dev, st);
+  }
+}
+
+template <typename TA, int SRC, int OUT>
+bl_status launch_gemv_mt(const GemvParams& p, int rpl, int grid, size_t smem, bool pdl, int dev,
+                         cudaStream_t st) {
+  // Token counts 1 and 2 get their own instantiations (fewer registers);
+  // 3 and 4 share MT = 4 with runtime guards.
+  if (p.M == 1) return launch_gemv_rpl<1, TA, SRC, OUT>(p, rpl, grid, smem, pdl, dev, st);
+  if (p.M == 2) return launch_gemv_rpl<2, TA, SRC, OUT>(p, rpl, grid, smem, pdl, dev, st);
+  return launch_gemv_rpl<4, TA, SRC, OUT>(p, rpl, grid, smem, pdl, dev, st);
+}
+
+constexpr size_t kGemvSmemCap = 200 * 1024;
+
+// Choose rows per CTA: one wave over the SMs when shared memory allows,
+// at most 128 rows (4 per lane).
+bl_status gemv_plan(int64_t N, int64_t K, int M, int sms, int* rows, int* rpl, int* grid,
+                    size_t* smem) {
+  int64_t r = (N + sms - 1) / sms;
+  if (r < 1) r = 1;
+  if (r > 128) r = 128;
+  while (r > 1 && gemv_smem_bytes(K, (int)r, M) > kGemvSmemCap) r = (r + 1) / 2;
+  if (gemv_smem_bytes(K, (int)r, M) > kGemvSmemCap) return BL_ERR_SHAPE;
+  *rows = (int)r;
+  *rpl = (int)((r + 31) / 32);
+  *grid = (int)((N + r - 1) / r);
+  *smem = gemv_smem_bytes(K, (int)r, M);
+  return BL_OK;
+}
+
+// src: kSrcFloat (a_dtype says f32/bf16), kSrcFfnRequant, kSrcInt8.
+bl_status run_gemv(int src, int out, bl_dtype a_dtype, GemvParams p, bool pdl, int dev, int sms,
+                   cudaStream_t st) {
+  int rows, rpl, grid;
+  size_t smem;
+  BL_TRY(gemv_plan(p.N, p.K, p.M, sms, &rows, &rpl, &grid, &smem));
+  p.rows_per_cta = rows;
+  p.pitch = gemv_pitch(p.K);
+  if (src == kSrcFloat) {
+    if (a_dtype == BL_BF16) {
+      return out == kOutDequant
+                 ? launch_gemv_mt<__nv_bfloat16, kSrcFloat, kOutDequant>(p, rpl, grid, smem, pdl, dev, st)
+                 : launch_gemv_mt<__nv_bfloat16, kSrcFloat, kOutRawI32>(p, rpl, grid, smem, pdl, dev, st);
+    }
+    return out == kOutDequant
+               ? launch_gemv_mt<float, kSrcFloat, kOutDequant>(p, rpl, grid, smem, pdl, dev, st)
+               : launch_gemv_mt<float, kSrcFloat, kOutRawI32>(p, rpl, grid, smem, pdl, dev, st);
+  }
+  if (src == kSrcFfnRequant)
+    return launch_gemv_mt<float, kSrcFfnRequant, kOutDequant>(p, rpl, grid, smem, pdl, dev, st);
+  return out == kOutDequant
+             ? launch_gemv_mt<float, kSrcInt8, kOutDequant>(p, rpl, grid, smem, pdl, dev, st)
+             : launch_gemv_mt<float, kSrcInt8, kOutRawI32>(p, rpl, grid, smem, pdl, dev, st);
+}
+
+// --------------------------------------------------------------------------
+// Tensor-core launches.
+template <int BN, int OUT>
+bl_status launch_tc_t(const CUtensorMap& ta, const CUtensorMap& tw, const TcParams& p, int dev,
+                      cudaStream_t st) {
+  auto* k = tc_ternary_gemm_kernel<BN, OUT>;
+  constexpr size_t smem = TcConfig<BN>::kSmemBytes;
+  BL_TRY(ensure_smem(k, dev, smem));
+  dim3 grid((unsigned)((p.N + 127) / 128), (unsigned)((p.M + BN - 1) / BN));
+  k<<<grid, kTcThreads, smem, st>>>(ta, tw, p);
+  BL_CUDA(cudaGetLastError());
+  return BL_OK;
+}
+
+template <int OUT>
+bl_status launch_tc_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tw, const TcParams& p,
+                       int dev, cudaStream_t st) {
+  switch (bn) {
+    case 16: return launch_tc_t<16, OUT>(ta, tw, p, dev, st);
+    case 32: return launch_tc_t<32, OUT>(ta, tw, p, dev, st);
+    case 64: return launch_tc_t<64, OUT>(ta, tw, p, dev, st);
+    case 128: return launch_tc_t<128, OUT>(ta, tw, p, dev, st);
+    default: return launch_tc_t<256, OUT>(ta, tw, p, dev, st);
+  }
+}
+
+int tc_pick_bn(int64_t M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  if (M <= 128) return 128;
+  return 256;
+}
+
+// acc/Y[M,N] = epilogue(A_q[M,K] · W_q[N,K]ᵀ − rowsum).
+bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,
+                 const float* gamma, const float* gammaA, const int32_t* rowsum, void* Y,
+                 int out, int relu2, int y_bf16, int dev, cudaStream_t st) {
+  if (M > 0x7FFFFFFF || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
+  const int bn = tc_pick_bn(M);
+  CUtensorMap ta, tw;
+  BL_TRY(make_map_u8(&ta, Aq, (uint64_t)M, (uint64_t)K, kTcBK, (uint32_t)bn,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+  BL_TRY(make_map_u8(&tw, Wp, (uint64_t)N, (uint64_t)(K / 4), kTcBK / 4, 128,
+                     CU_TENSOR_MAP_SWIZZLE_NONE));
+  TcParams p;
+  p.gamma = gamma;
+  p.gammaA = gammaA;
+  p.rowsum = rowsum;
+  p.Y = Y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.relu2 = relu2;
+  p.y_bf16 = y_bf16;
+  return out == kTcDequant ? launch_tc_bn<kTcDequant>(bn, ta, tw, p, dev, st)
+                           : launch_tc_bn<kTcRawI32>(bn, ta, tw, p, dev, st);
+}
+
+bl_status run_quant_acts(const void* A, bl_dtype dt, int64_t M, int64_t K, float eps, int8_t* Aq,
+                         float* gA, int32_t* rs, cudaStream_t st) {
+  if (M == 0) return BL_OK;
+  if (dt == BL_BF16)
+    quant_acts_kernel<__nv_bfloat16><<<(unsigned)M, kQuantThreads, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(A), K, eps, Aq, gA, rs);
+  else
+    quant_acts_kernel<float><<<(unsigned)M, kQuantThreads, 0, st>>>(
+        reinterpret_cast<const float*>(A), K, eps, Aq, gA, rs);
+  BL_CUDA(cudaGetLastError());
+  return BL_OK;
+}
+
+}  // namespace
+}  // namespace bl
+
+using namespace bl;
+
+// ==========================================================================
+// Public C ABI
+// ==========================================================================
+extern "C" {
+
+const char* bl_status_string(bl_status s) {
+  switch (s) {
+    case BL_OK: return "BL_OK";
+    case BL_ERR_INVALID_ARG: return "BL_ERR_INVALID_ARG: null pointer, bad eps, flag or value";
+    case BL_ERR_SHAPE: return "BL_ERR_SHAPE: size negative, too large, or K/H not a positive multiple of 64";
+    case BL_ERR_ALIGN: return "BL_ERR_ALIGN: pointer not 16-byte aligned";
+    case BL_ERR_DTYPE: return "BL_ERR_DTYPE: dtype not supported for this argument";
+    case BL_ERR_CUDA: return "BL_ERR_CUDA: CUDA call or kernel launch failed";
+    case BL_ERR_TIMEOUT: return "BL_ERR_TIMEOUT: a device-side bounded wait gave up";
+    case BL_ERR_UNSUPPORTED: return "BL_ERR_UNSUPPORTED: device is not sm_100 (B200)";
+    case BL_ERR_WORKSPACE: return "BL_ERR_WORKSPACE: workspace missing or too small";
+  }
+  return "BL_ERR_UNKNOWN";
+}
+
+int bl_version(void) { return 100; }
+
+int bl_gemv_max_tokens(void) { return kGemvMaxTokens; }
+
+size_t bl_quant_weights_workspace_bytes(int64_t N, int64_t K) {
+  (void)N;
+  (void)K;
+  return (size_t)kAbsmeanMaxBlocks * sizeof(double);
+}
+
+bl_status bl_quant_weights(const void* W, bl_dtype w_dtype, int64_t N, int64_t K, float eps,
+                           uint8_t* W_packed, float* gamma, void* workspace, size_t ws_bytes,
+                           bl_stream_t stream) {
+  BL_TRY(check_dtype(w_dtype));
+  BL_TRY(check_k(K));
+  BL_TRY(check_rows(N));
+  BL_TRY(check_eps(eps));
+  if (N == 0) return BL_OK;
+  BL_TRY(check_ptr(W));
+  BL_TRY(check_ptr(W_packed));
+  if (gamma == nullptr) return BL_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(gamma) & 3u) != 0) return BL_ERR_ALIGN;
+  if (workspace == nullptr || ws_bytes < bl_quant_weights_workspace_bytes(N, K))
+    return BL_ERR_WORKSPACE;
+  BL_TRY(check_ptr(workspace));
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t count = N * K;
+  const int vec = w_dtype == BL_BF16 ? 8 : 4;
+  const int64_t nvec = count / vec;
+  int64_t blocks = (nvec + kQuantThreads - 1) / kQuantThreads;
+  if (blocks > kAbsmeanMaxBlocks) blocks = kAbsmeanMaxBlocks;
+  if (blocks > 8 * (int64_t)sms) blocks = 8 * (int64_t)sms;
+  double* partials = reinterpret_cast<double*>(workspace);
+  const int64_t nwords = count / 16;
+  int64_t pblocks = (nwords + kQuantThreads - 1) / kQuantThreads;
+  if (pblocks > 16 * (int64_t)sms) pblocks = 16 * (int64_t)sms;
+  if (w_dtype == BL_BF16) {
+    auto* Wt = reinterpret_cast<const __nv_bfloat16*>(W);
+    absmean_partial_kernel<__nv_bfloat16><<<(unsigned)blocks, kQuantThreads, 0, st>>>(Wt, count, partials);
+    BL_CUDA(cudaGetLastError());
+    ternary_pack_kernel<__nv_bfloat16><<<(unsigned)pblocks, kQuantThreads, 0, st>>>(
+        Wt, nwords, (double)count, eps, partials, (int)blocks,
+        reinterpret_cast<uint32_t*>(W_packed), gamma);
+  } else {
+    auto* Wt = reinterpret_cast<const float*>(W);
+    absmean_partial_kernel<float><<<(unsigned)blocks, kQuantThreads, 0, st>>>(Wt, count, partials);
+    BL_CUDA(cudaGetLastError());
+    ternary_pack_kernel<float><<<(unsigned)pblocks, kQuantThreads, 0, st>>>(
+        Wt, nwords, (double)count, eps, partials, (int)blocks,
+        reinterpret_cast<uint32_t*>(W_packed), gamma);
+  }
+  BL_CUDA(cudaGetLastError());
+  return BL_OK;
+}
+
+bl_status bl_quant_acts(const void* A, bl_dtype a_dtype, int64_t M, int64_t K, float eps,
+                        int8_t* A_q, float* gamma_A, int32_t* rowsum, bl_stream_t stream) {
+  BL_TRY(check_dtype(a_dtype));
+  BL_TRY(check_k(K));
+  BL_TRY(check_rows(M));
+  BL_TRY(check_eps(eps));
+  if (M == 0) return BL_OK;
+  BL_TRY(check_ptr(A));
+  BL_TRY(check_ptr(A_q));
+  BL_TRY(check_ptr(gamma_A));
+  if (rowsum != nullptr) BL_TRY(check_ptr(rowsum));
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  return run_quant_acts(A, a_dtype, M, K, eps, A_q, gamma_A, rowsum,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t bl_zero_gemm_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+  (void)K;
+  (void)N;
+  if (M <= kGemvMaxTokens) return 0;
+  return align_up((size_t)M * 4);
+}
+
+bl_status bl_zero_gemm(const int8_t* A_q, int64_t M, int64_t K, const uint8_t* W_packed,
+                       int64_t N, int32_t* acc, void* workspace, size_t ws_bytes,
+                       bl_stream_t stream) {
+  BL_TRY(check_k(K));
+  BL_TRY(check_rows(M));
+  BL_TRY(check_rows(N));
+  if (M == 0 || N == 0) return BL_OK;
+  BL_TRY(check_ptr(A_q));
+  BL_TRY(check_ptr(W_packed));
+  BL_TRY(check_ptr(acc));
+  const size_t need = bl_zero_gemm_workspace_bytes(M, K, N);
+  if (need > 0) {
+    if (workspace == nullptr || ws_bytes < need) return BL_ERR_WORKSPACE;
+    BL_TRY(check_ptr(workspace));
+  }
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (M <= kGemvMaxTokens) {
+    GemvParams p = {};
+    p.A = A_q;
+    p.W = W_packed;
+    p.Y = acc;
+    p.N = N;
+    p.K = K;
+    p.M = (int)M;
+    p.eps = 1.0f;
+    return run_gemv(kSrcInt8, kOutRawI32, BL_F32, p, false, dev, sms, st);
+  }
+  int32_t* rs = reinterpret_cast<int32_t*>(workspace);
+  rowsum_i8_kernel<<<(unsigned)M, kQuantThreads, 0, st>>>(A_q, K, rs);
+  BL_CUDA(cudaGetLastError());
+  return run_tc(A_q, W_packed, M, K, N, nullptr, nullptr, rs, acc, kTcRawI32, 0, 0, dev, st);
+}
+
+size_t bl_linear_q_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+  (void)K;
+  (void)N;
+  if (M <= kGemvMaxTokens) return 0;
+  return align_up((size_t)M * 4);
+}
+
+bl_status bl_linear_q(const int8_t* A_q, const float* gamma_A, const int32_t* rowsum, int64_t M,
+                      int64_t K, const uint8_t* W_packed, const float* gamma, int64_t N, int relu2,
+                      void* Y, bl_dtype y_dtype, void* workspace, size_t ws_bytes,
+                      bl_stream_t stream) {
+  BL_TRY(check_dtype(y_dtype));
+  BL_TRY(check_k(K));
+  BL_TRY(check_rows(M));
+  BL_TRY(check_rows(N));
+  if (M == 0 || N == 0) return BL_OK;
+  BL_TRY(check_ptr(A_q));
+  BL_TRY(check_ptr(gamma_A));
+  if (rowsum != nullptr) BL_TRY(check_ptr(rowsum));
+  BL_TRY(check_ptr(W_packed));
+  if (gamma == nullptr) return BL_ERR_INVALID_ARG;
+  BL_TRY(check_ptr(Y));
+  const size_t need = rowsum ? 0 : bl_linear_q_workspace_bytes(M, K, N);
+  if (need > 0) {
+    if (workspace == nullptr || ws_bytes < need) return BL_ERR_WORKSPACE;
+    BL_TRY(check_ptr(workspace));
+  }
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (M <= kGemvMaxTokens) {
+    GemvParams p = {};
+    p.A = A_q;
+    p.a_scale = gamma_A;
+    p.a_rowsum = rowsum;
+    p.W = W_packed;
+    p.gamma = gamma;
+    p.Y = Y;
+    p.N = N;
+    p.K = K;
+    p.M = (int)M;
+    p.eps = 1.0f;
+    p.relu2 = relu2 ? 1 : 0;
+    p.y_bf16 = y_dtype == BL_BF16;
+    return run_gemv(kSrcInt8, kOutDequant, BL_F32, p, false, dev, sms, st);
+  }
+  const int32_t* rs = rowsum;
+  if (rs == nullptr) {
+    int32_t* w = reinterpret_cast<int32_t*>(workspace);
+    rowsum_i8_kernel<<<(unsigned)M, kQuantThreads, 0, st>>>(A_q, K, w);
+    BL_CUDA(cudaGetLastError());
+    rs = w;
+  }
+  return run_tc(A_q, W_packed, M, K, N, gamma, gamma_A, rs, Y, kTcDequant, relu2 ? 1 : 0,
+                y_dtype == BL_BF16, dev, st);
+}
+
+size_t bl_linear_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+  (void)N;
+  if (M <= kGemvMaxTokens) return 0;
+  return act_ws(M, K).total;
+}
+
+bl_status bl_linear_ex(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
+                       const uint8_t* W_packed, const float* gamma, int64_t N, float eps,
+                       int relu2, void* Y, bl_dtype y_dtype, void* workspace, size_t ws_bytes,
+                       unsigned flags, bl_stream_t stream) {
+  BL_TRY(check_dtype(a_dtype));
+  BL_TRY(check_dtype(y_dtype));
+  BL_TRY(check_k(K));
+  BL_TRY(check_rows(M));
+  BL_TRY(check_rows(N));
+  BL_TRY(check_eps(eps));
+  if ((flags & ~(unsigned)BL_FLAG_PDL) != 0) return BL_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return BL_OK;
+  BL_TRY(check_ptr(A));
+  BL_TRY(check_ptr(W_packed));
+  if (gamma == nullptr) return BL_ERR_INVALID_ARG;
+  BL_TRY(check_ptr(Y));
+  const size_t need = bl_linear_workspace_bytes(M, K, N);
+  if (need > 0) {
+    if (workspace == nullptr || ws_bytes < need) return BL_ERR_WORKSPACE;
+    BL_TRY(check_ptr(workspace));
+  }
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (M <= kGemvMaxTokens) {
+    GemvParams p = {};
+    p.A = A;
+    p.W = W_packed;
+    p.gamma = gamma;
+    p.Y = Y;
+    p.N = N;
+    p.K = K;
+    p.M = (int)M;
+    p.eps = eps;
+    p.relu2 = relu2 ? 1 : 0;
+    p.y_bf16 = y_dtype == BL_BF16;
+    return run_gemv(kSrcFloat, kOutDequant, a_dtype, p, (flags & BL_FLAG_PDL) != 0, dev, sms, st);
+  }
+  const ActWs w = act_ws(M, K);
+  uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
+  int8_t* Aq = reinterpret_cast<int8_t*>(base + w.aq);
+  float* gA = reinterpret_cast<float*>(base + w.gamma);
+  int32_t* rs = reinterpret_cast<int32_t*>(base + w.rowsum);
+  BL_TRY(run_quant_acts(A, a_dtype, M, K, eps, Aq, gA, rs, st));
+  return run_tc(Aq, W_packed, M, K, N, gamma, gA, rs, Y, kTcDequant, relu2 ? 1 : 0,
+                y_dtype == BL_BF16, dev, st);
+}
+
+bl_status bl_linear(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
+                    const uint8_t* W_packed, const float* gamma, int64_t N, float eps, int relu2,
+                    void* Y, bl_dtype y_dtype, void* workspace, size_t ws_bytes,
+                    bl_stream_t stream) {
+  return bl_linear_ex(A, a_dtype, M, K, W_packed, gamma, N, eps, relu2, Y, y_dtype, workspace,
+                      ws_bytes, 0u, stream);
+}
+
+size_t bl_ffn_workspace_bytes(int64_t M, int64_t K, int64_t H) { return ffn_ws(M, K, H).total; }
+
+bl_status bl_ffn_relu2(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, int64_t H,
+                       const uint8_t* W_up, const float* gamma_up, const uint8_t* W_down,
+                       const float* gamma_down, float eps, void* Y, bl_dtype y_dtype,
+                       void* workspace, size_t ws_bytes, bl_stream_t stream) {
+  BL_TRY(check_dtype(x_dtype));
+  BL_TRY(check_dtype(y_dtype));
+  BL_TRY(check_k(K));
+  BL_TRY(check_k(H));
+  BL_TRY(check_rows(M));
+  BL_TRY(check_eps(eps));
+  if (M == 0) return BL_OK;
+  BL_TRY(check_ptr(X));
+  BL_TRY(check_ptr(W_up));
+  BL_TRY(check_ptr(W_down));
+  if (gamma_up == nullptr || gamma_down == nullptr) return BL_ERR_INVALID_ARG;
+  BL_TRY(check_ptr(Y));
+  const FfnWs w = ffn_ws(M, K, H);
+  if (workspace == nullptr || ws_bytes < w.total) return BL_ERR_WORKSPACE;
+  BL_TRY(check_ptr(workspace));
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
+  int32_t* acc_up = reinterpret_cast<int32_t*>(base + w.acc_up);
+  if (M <= kGemvMaxTokens) {
+    float* gX = reinterpret_cast<float*>(base + w.gamma_x);
+    GemvParams up = {};
+    up.A = X;
+    up.W = W_up;
+    up.gamma = gamma_up;
+    up.Y = acc_up;
+    up.gamma_out = gX;
+    up.N = H;
+    up.K = K;
+    up.M = (int)M;
+    up.eps = eps;
+    BL_TRY(run_gemv(kSrcFloat, kOutRawI32, x_dtype, up, false, dev, sms, st));
+    GemvParams dn = {};
+    dn.A = acc_up;
+    dn.a_scale = gX;
+    dn.a_gamma_up = gamma_up;
+    dn.W = W_down;
+    dn.gamma = gamma_down;
+    dn.Y = Y;
+    dn.N = K;
+    dn.K = H;
+    dn.M = (int)M;
+    dn.eps = eps;
+    dn.y_bf16 = y_dtype == BL_BF16;
+    return run_gemv(kSrcFfnRequant, kOutDequant, BL_F32, dn, false, dev, sms, st);
+  }
+  int8_t* Xq = reinterpret_cast<int8_t*>(base + w.x.aq);
+  float* gX = reinterpret_cast<float*>(base + w.x.gamma);
+  int32_t* rsX = reinterpret_cast<int32_t*>(base + w.x.rowsum);
+  int8_t* Rq = reinterpret_cast<int8_t*>(base + w.rq);
+  float* gR = reinterpret_cast<float*>(base + w.gamma_r);
+  int32_t* rsR = reinterpret_cast<int32_t*>(base + w.rs_r);
+  BL_TRY(run_quant_acts(X, x_dtype, M, K, eps, Xq, gX, rsX, st));
+  BL_TRY(run_tc(Xq, W_up, M, K, H, gamma_up, gX, rsX, acc_up, kTcRawI32, 0, 0, dev, st));
+  relu2_requant_kernel<<<(unsigned)M, kQuantThreads, 0, st>>>(acc_up, H, gX, gamma_up, eps, Rq, gR,
+                                                              rsR);
+  BL_CUDA(cudaGetLastError());
+  return run_tc(Rq, W_down, M, H, K, gamma_down, gR, rsR, Y, kTcDequant, 0, y_dtype == BL_BF16,
+                dev, st);
+}
+
+bl_status bl_check_device_error(bl_stream_t stream) {
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return BL_ERR_CUDA;
+  unsigned flags = 0;
+  BL_CUDA(cudaMemcpyFromSymbol(&flags, g_error_flags, sizeof(flags)));
+  if (flags != 0) {
+    const unsigned zero = 0;
+    BL_CUDA(cudaMemcpyToSymbol(g_error_flags, &zero, sizeof(zero)));
+    return BL_ERR_TIMEOUT;
+  }
+  return BL_OK;
+}
+
+}  // extern "C"
+
+namespace bl {
+namespace {
+__global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    // Nothing ever arrives on `bar`: the bounded wait must give up.
+    if (!mbar_wait_for(&bar, 0, limit_ns)) raise_error(kErrTimeout);
+  }
+}
+}  // namespace
+}  // namespace bl
+
+extern "C" bl_status bl_selftest_wait_timeout(int64_t limit_ns, bl_stream_t stream) {
+  if (limit_ns < 1000 || limit_ns > 1000000000) return BL_ERR_INVALID_ARG;
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  bl::wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      (unsigned long long)limit_ns);
+  BL_CUDA(cudaGetLastError());
+  return BL_OK;
+}

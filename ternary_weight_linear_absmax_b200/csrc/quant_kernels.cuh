@@ -1,0 +1,260 @@
+// Quantiser kernels: AbsMean ternary weight quantisation + 2-bit packing,
+// AbsMax per-token INT8 activation quantisation, and the FFN ReLU²
+// requantisation. All are single-pass, HBM-bound streaming kernels.
+//
+// Formulas: "BitNet b1.58 — quantização ternária, BitLinear, Zero-GEMM",
+// section "Por que 1,58 bits por peso e qual a matemática da ternarização?"
+// (γ = mean|W|, W_q = Round(Clip(W/(γ+ε), -1, 1)); γ_A = max|A| per token,
+// A_q = Clip(Round(A·127/(γ_A+ε)), -128, 127)); ReLU² from the BitLinear
+// utilities (ReLUSquared) of "Arquitetura Hibrida Multimodal para bitnet.cpp".
+#pragma once
+
+#include "bl_device.cuh"
+
+namespace bl {
+
+constexpr int kQuantThreads = 256;
+
+// ---------------------------------------------------------------------------
+// AbsMean, pass 1: per-block partial sums of |W| in double. Each thread
+// reads 16-byte vectors (8 bf16 or 4 fp32) in a grid-stride loop.
+template <typename T>
+__global__ void __launch_bounds__(kQuantThreads)
+absmean_partial_kernel(const T* __restrict__ W, int64_t count, double* __restrict__ partials) {
+  constexpr int VEC = 16 / sizeof(T);
+  const int64_t nvec = count / VEC;
+  const uint4* W4 = reinterpret_cast<const uint4*>(W);
+  double s = 0.0;
+  for (int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; v < nvec;
+       v += (int64_t)gridDim.x * blockDim.x) {
+    uint4 u = __ldg(W4 + v);
+    const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) s += fabs((double)to_f32<T>(e[i]));
+  }
+  // tail (count not a multiple of VEC cannot happen: K % 64 == 0)
+  s = warp_sum_d(s);
+  __shared__ double red[kQuantThreads / 32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    double t = threadIdx.x < kQuantThreads / 32 ? red[threadIdx.x] : 0.0;
+    t = warp_sum_d(t);
+    if (threadIdx.x == 0) partials[blockIdx.x] = t;
+  }
+}
+
+// Deterministic block-wide sum of the partials (fixed order for a given
+// partial count), result broadcast through shared memory.
+__device__ __forceinline__ double sum_partials(const double* __restrict__ partials, int n) {
+  __shared__ double red[kQuantThreads / 32];
+  __shared__ double total;
+  double s = 0.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) s += partials[i];
+  s = warp_sum_d(s);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    double t = threadIdx.x < (int)(blockDim.x / 32) ? red[threadIdx.x] : 0.0;
+    t = warp_sum_d(t);
+    if (threadIdx.x == 0) total = t;
+  }
+  __syncthreads();
+  return total;
+}
+
+// AbsMean, pass 2: γ from the partials, then ternary codes and packing.
+// One thread produces one 32-bit packed word (16 consecutive weights).
+//
+// Code decision. The pages' rule is Round(Clip(x)) with x = fl32(W/g),
+// g = fl32(γ+ε). Since fl32 is monotone and the quotients in
+// (1/2, 1/2 + 2^-25] round to 1/2 (a tie that round-half-even sends to 0),
+//   Round(Clip(fl32(W/g))) = +1  iff  W >  g·(1/2 + 2^-25),
+//                            -1  iff  W < -g·(1/2 + 2^-25),   else 0,
+// where the threshold g·(1/2 + 2^-25) is exact in double (24 + 25 bits).
+// This reproduces the fp32 division bit for bit without dividing per weight.
+template <typename T>
+__global__ void __launch_bounds__(kQuantThreads)
+ternary_pack_kernel(const T* __restrict__ W, int64_t nwords, double count, float eps,
+                    const double* __restrict__ partials, int npartials,
+                    uint32_t* __restrict__ packed, float* __restrict__ gamma_out) {
+  const double total = sum_partials(partials, npartials);
+  const float gamma = (float)(total / count);  // mean in double, rounded once
+  if (blockIdx.x == 0 && threadIdx.x == 0) *gamma_out = gamma;
+  const float g = __fadd_rn(gamma, eps);
+  const double thr = (double)g * (0.5 + 0x1p-25);
+  constexpr int VEC = 16 / sizeof(T);
+  constexpr int NV = 16 / VEC;  // 16-byte vectors per 16 weights
+  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < nwords;
+       w += (int64_t)gridDim.x * blockDim.x) {
+    const uint4* src = reinterpret_cast<const uint4*>(W + w * 16);
+    T e[16];
+#pragma unroll
+    for (int v = 0; v < NV; ++v) *reinterpret_cast<uint4*>(&e[v * VEC]) = __ldg(src + v);
+    uint32_t word = 0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const double x = (double)to_f32<T>(e[k]);
+      const uint32_t c = x > thr ? 2u : (x < -thr ? 0u : 1u);
+      const int j = k >> 2, i = k & 3;
+      word |= c << (8 * i + 2 * j);
+    }
+    packed[w] = word;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// AbsMax activation quantisation: one block per token row.
+// Writes int8 A_q, γ_A and (optionally) the row sum of A_q.
+template <typename T>
+__global__ void __launch_bounds__(kQuantThreads)
+quant_acts_kernel(const T* __restrict__ A, int64_t K, float eps, int8_t* __restrict__ Aq,
+                  float* __restrict__ gammaA, int32_t* __restrict__ rowsum) {
+  const int64_t m = blockIdx.x;
+  const T* row = A + m * K;
+  constexpr int VEC = 16 / sizeof(T);
+  const int64_t nvec = K / VEC;
+  const uint4* r4 = reinterpret_cast<const uint4*>(row);
+  __shared__ float redf[kQuantThreads / 32];
+  __shared__ int redi[kQuantThreads / 32];
+  __shared__ float s_scale;
+
+  float mx = 0.0f;
+  for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
+    uint4 u = __ldg(r4 + v);
+    const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) mx = fmaxf(mx, fabsf(to_f32<T>(e[i])));
+  }
+  mx = warp_max(mx);
+  if ((threadIdx.x & 31) == 0) redf[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float t = threadIdx.x < kQuantThreads / 32 ? redf[threadIdx.x] : 0.0f;
+    t = warp_max(t);
+    if (threadIdx.x == 0) {
+      gammaA[m] = t;
+      s_scale = __fdiv_rn(127.0f, __fadd_rn(t, eps));
+    }
+  }
+  __syncthreads();
+  const float s = s_scale;
+  int sum = 0;
+  for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
+    uint4 u = __ldg(r4 + v);
+    const T* e = reinterpret_cast<const T*>(&u);
+    int8_t q[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+      q[i] = quant_i8(to_f32<T>(e[i]), s);
+      sum += q[i];
+    }
+    if constexpr (VEC == 8) {
+      *reinterpret_cast<uint2*>(Aq + m * K + v * VEC) = *reinterpret_cast<uint2*>(q);
+    } else {
+      *reinterpret_cast<uint32_t*>(Aq + m * K + v * VEC) = *reinterpret_cast<uint32_t*>(q);
+    }
+  }
+  if (rowsum != nullptr) {
+    sum = warp_sum_i(sum);
+    if ((threadIdx.x & 31) == 0) redi[threadIdx.x >> 5] = sum;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      int t = threadIdx.x < kQuantThreads / 32 ? redi[threadIdx.x] : 0;
+      t = warp_sum_i(t);
+      if (threadIdx.x == 0) rowsum[m] = t;
+    }
+  }
+}
+
+// Row sums of an int8 matrix (one block per row), for callers that pass
+// quantised activations without their sums.
+__global__ void __launch_bounds__(kQuantThreads)
+rowsum_i8_kernel(const int8_t* __restrict__ Aq, int64_t K, int32_t* __restrict__ rowsum) {
+  const int64_t m = blockIdx.x;
+  const uint4* r4 = reinterpret_cast<const uint4*>(Aq + m * K);
+  int sum = 0;
+  for (int64_t v = threadIdx.x; v < K / 16; v += blockDim.x) {
+    uint4 u = __ldg(r4 + v);
+    sum = dp4a(u.x, 0x01010101u, sum);
+    sum = dp4a(u.y, 0x01010101u, sum);
+    sum = dp4a(u.z, 0x01010101u, sum);
+    sum = dp4a(u.w, 0x01010101u, sum);
+  }
+  __shared__ int redi[kQuantThreads / 32];
+  sum = warp_sum_i(sum);
+  if ((threadIdx.x & 31) == 0) redi[threadIdx.x >> 5] = sum;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    int t = threadIdx.x < kQuantThreads / 32 ? redi[threadIdx.x] : 0;
+    t = warp_sum_i(t);
+    if (threadIdx.x == 0) rowsum[m] = t;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// FFN requantisation of the up-projection, one block per token:
+//   h = fp32(acc · fp32((γ_X·γ_up)/127)),  r = max(h,0)²  (fp32),
+//   γ_r = max_n r,  q = Clip(Round(r · 127/(γ_r+ε)), -128, 127),  Σq.
+// ReLU² is monotone in acc and fp32 rounding is monotone, so γ_r is also
+// the image of the largest accumulator; computing it from r keeps the
+// kernel a literal restatement.
+__global__ void __launch_bounds__(kQuantThreads)
+relu2_requant_kernel(const int32_t* __restrict__ acc, int64_t H, const float* __restrict__ gammaX,
+                     const float* __restrict__ g_up, float eps, int8_t* __restrict__ Rq,
+                     float* __restrict__ gammaR, int32_t* __restrict__ rowsum) {
+  const int64_t m = blockIdx.x;
+  const int4* a4 = reinterpret_cast<const int4*>(acc + m * H);
+  const float sc = __fdiv_rn(__fmul_rn(gammaX[m], *g_up), 127.0f);
+  __shared__ float redf[kQuantThreads / 32];
+  __shared__ int redi[kQuantThreads / 32];
+  __shared__ float s_scale;
+  float mx = 0.0f;
+  for (int64_t v = threadIdx.x; v < H / 4; v += blockDim.x) {
+    int4 u = __ldg(a4 + v);
+    const int e[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float h = __fmul_rn((float)e[i], sc);
+      float p = fmaxf(h, 0.0f);
+      mx = fmaxf(mx, __fmul_rn(p, p));
+    }
+  }
+  mx = warp_max(mx);
+  if ((threadIdx.x & 31) == 0) redf[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float t = threadIdx.x < kQuantThreads / 32 ? redf[threadIdx.x] : 0.0f;
+    t = warp_max(t);
+    if (threadIdx.x == 0) {
+      gammaR[m] = t;
+      s_scale = __fdiv_rn(127.0f, __fadd_rn(t, eps));
+    }
+  }
+  __syncthreads();
+  const float s = s_scale;
+  int sum = 0;
+  for (int64_t v = threadIdx.x; v < H / 4; v += blockDim.x) {
+    int4 u = __ldg(a4 + v);
+    const int e[4] = {u.x, u.y, u.z, u.w};
+    int8_t q[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float h = __fmul_rn((float)e[i], sc);
+      float p = fmaxf(h, 0.0f);
+      q[i] = quant_i8(__fmul_rn(p, p), s);
+      sum += q[i];
+    }
+    *reinterpret_cast<uint32_t*>(Rq + m * H + v * 4) = *reinterpret_cast<uint32_t*>(q);
+  }
+  sum = warp_sum_i(sum);
+  if ((threadIdx.x & 31) == 0) redi[threadIdx.x >> 5] = sum;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    int t = threadIdx.x < kQuantThreads / 32 ? redi[threadIdx.x] : 0;
+    t = warp_sum_i(t);
+    if (threadIdx.x == 0) rowsum[m] = t;
+  }
+}
+
+}  // namespace bl

@@ -1,0 +1,93 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol include/bitlinear.h declares, and rejects bad arguments on the
+host with the documented status codes before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from ternary_weight_linear_absmax_b200 import _lib
+    from ternary_weight_linear_absmax_b200 import build as b
+    b.build()
+    return _lib.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bl_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_symbols_exported(lib):
+    from ternary_weight_linear_absmax_b200 import _lib
+    syms = declared_symbols()
+    assert len(syms) >= 15
+    for s in syms:
+        assert hasattr(lib, s), f"{s} declared in bitlinear.h but not exported"
+    # the binding declares a signature for every exported entry point
+    assert set(syms) == set(_lib.SIGNATURES)
+
+
+def test_status_strings(lib):
+    for code in range(9):
+        s = lib.bl_status_string(code).decode()
+        assert s.startswith("BL_")
+    assert lib.bl_status_string(99).decode() == "BL_ERR_UNKNOWN"
+    assert lib.bl_version() >= 100
+    assert lib.bl_gemv_max_tokens() == 4
+
+
+def test_workspace_sizes(lib):
+    assert lib.bl_quant_weights_workspace_bytes(4096, 4096) >= 1024 * 8
+    assert lib.bl_linear_workspace_bytes(1, 2560, 6912) == 0
+    ws = lib.bl_linear_workspace_bytes(2048, 4096, 4096)
+    assert ws >= 2048 * 4096 + 2 * 2048 * 4
+    assert lib.bl_ffn_workspace_bytes(1, 4096, 11008) >= 11008 * 4 + 4
+    assert lib.bl_ffn_workspace_bytes(512, 4096, 11008) >= 512 * 11008 * 5 + 512 * 4096
+    assert lib.bl_zero_gemm_workspace_bytes(4, 512, 256) == 0
+
+
+def _aligned_buf(n=4096):
+    buf = ctypes.create_string_buffer(n + 64)
+    addr = (ctypes.addressof(buf) + 15) & ~15
+    return buf, addr
+
+
+def test_argument_errors_on_host(lib):
+    """Shape, eps, pointer, alignment, dtype and workspace errors are caught
+    before any CUDA call (these run without a GPU)."""
+    keep, p = _aligned_buf()
+    BL_ERR_INVALID_ARG, BL_ERR_SHAPE, BL_ERR_ALIGN, BL_ERR_DTYPE, BL_ERR_WORKSPACE = 1, 2, 3, 4, 8
+    # K not a multiple of 64
+    assert lib.bl_quant_weights(p, 0, 16, 100, 1e-5, p, p, p, 8192, None) == BL_ERR_SHAPE
+    assert lib.bl_quant_weights(p, 0, 16, 0, 1e-5, p, p, p, 8192, None) == BL_ERR_SHAPE
+    assert lib.bl_quant_weights(p, 0, -1, 64, 1e-5, p, p, p, 8192, None) == BL_ERR_SHAPE
+    # eps must be > 0 and finite
+    assert lib.bl_quant_weights(p, 0, 16, 64, 0.0, p, p, p, 8192, None) == BL_ERR_INVALID_ARG
+    assert lib.bl_quant_weights(p, 0, 16, 64, float("nan"), p, p, p, 8192, None) == BL_ERR_INVALID_ARG
+    # dtype
+    assert lib.bl_quant_weights(p, 7, 16, 64, 1e-5, p, p, p, 8192, None) == BL_ERR_DTYPE
+    # null and misaligned pointers
+    assert lib.bl_quant_weights(None, 0, 16, 64, 1e-5, p, p, p, 8192, None) == BL_ERR_INVALID_ARG
+    assert lib.bl_quant_weights(p + 4, 0, 16, 64, 1e-5, p, p, p, 8192, None) == BL_ERR_ALIGN
+    # workspace
+    assert lib.bl_quant_weights(p, 0, 16, 64, 1e-5, p, p, None, 0, None) == BL_ERR_WORKSPACE
+    assert lib.bl_quant_weights(p, 0, 16, 64, 1e-5, p, p, p, 16, None) == BL_ERR_WORKSPACE
+    # linear: workspace required above the GEMV token limit
+    assert lib.bl_linear(p, 1, 64, 512, p, p, 256, 1e-5, 0, p, 1, None, 0, None) == BL_ERR_WORKSPACE
+    assert lib.bl_linear(p, 1, 4, 500, p, p, 256, 1e-5, 0, p, 1, None, 0, None) == BL_ERR_SHAPE
+    assert lib.bl_linear_ex(p, 1, 4, 512, p, p, 256, 1e-5, 0, p, 1, None, 0, 8, None) == BL_ERR_INVALID_ARG
+    # FFN hidden size must be a multiple of 64
+    assert lib.bl_ffn_relu2(p, 1, 1, 512, 100, p, p, p, p, 1e-5, p, 1, p, 1 << 20, None) == BL_ERR_SHAPE
+    # empty problems are no-ops
+    assert lib.bl_linear(p, 1, 0, 512, p, p, 256, 1e-5, 0, p, 1, None, 0, None) == 0
+    assert lib.bl_quant_acts(p, 1, 0, 512, 1e-5, p, p, None, None) == 0
+    assert lib.bl_selftest_wait_timeout(10, None) == BL_ERR_INVALID_ARG
