@@ -1,0 +1,566 @@
+#!/usr/bin/env python
+"""Benchmark of the BitLinear forward on B200.
+
+Headline workload (one JSON line on rank 0): decode GEMV — 1 token, K = 2560,
+N = 6912, bf16 activations with 1 % ×20 outlier channels, 2-bit packed
+ternary weights (pre-quantised), bf16 output. One step = 1000 BitLinear calls
+(1 token each) chained on one stream with programmatic dependent launch,
+replayed as a CUDA graph, each call against the next matrix of a rotating
+pool of distinct packed weight matrices whose total size is ≥ 3× the L2
+cache (so weights stream from HBM, no L2 flush needed). Metric: tokens/s.
+
+Secondary workloads (key "extra"): small-batch decode (16 tokens, 4096 →
+11008), prefill (2048 tokens, 4096 → 4096; INT8 tensor-core contraction timed
+apart from the activation quantiser), the ternary FFN block (4096 → 11008 →
+4096, M ∈ {1, 64, 512}) and the weight quantiser.
+
+--impl reference times the CPU oracle (test infrastructure, the reference
+arm) on the host cores on the decode workload.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own decode
+stream (weak scaling, no data-path collective); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth_inputs as si  # noqa: E402
+
+METRIC = "BitLinear tokens/s; decode % of HBM roofline, prefill % of INT8 TC peak"
+UNIT = "tokens/s"
+EPS = 1e-5
+DECODE = dict(M=1, K=2560, N=6912)
+CALLS_PER_STEP = 1000
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense ratio (B200: 4.5 PFLOP/s fp8/int8, 2.25 bf16)
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "gemv_decode_k2560_n6912.md")
+GEMV_SOURCE = os.path.join(ROOT, "ternary_weight_linear_absmax_b200", "csrc", "gemv_kernel.cuh")
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (also exercised on CPU with gloo by the tests)
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(per_rank_units: float, elapsed_max_s: float, world: int) -> float:
+    """Whole-job throughput: units processed by all ranks ÷ the slowest rank's time."""
+    return per_rank_units * world / elapsed_max_s
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# measured peaks and profile-derived traffic
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def sha256_file(path):
+    h = hashlib.sha256()
+    with open(path, "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the decode GEMV from the committed ncu
+    summary, or None when missing or taken on a different kernel source."""
+    try:
+        kv = {}
+        with open(PROFILE_TRAFFIC) as f:
+            for line in f:
+                if ":" in line and line.startswith("- "):
+                    k, v = line[2:].split(":", 1)
+                    kv[k.strip()] = v.strip().strip("`")
+        if kv.get("kernel_source_sha256") != sha256_file(GEMV_SOURCE):
+            return None
+        return float(kv["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# clocks sampler (nvidia-smi during the timed region)
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CUDA helpers
+
+def l2_bytes(device_index: int) -> int:
+    import torch
+    try:
+        return int(torch.cuda.get_device_properties(device_index).L2_cache_size)
+    except Exception:
+        return 126 * 1024 * 1024
+
+
+def time_graph(graph, stream, reps: int):
+    """Replay a captured graph `reps` times; device time in seconds."""
+    import torch
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / 1e3
+
+
+def capture(fn, stream):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        fn()  # one eager call first (binds workspaces, sets kernel attributes)
+        stream.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def weight_pool(bl, N, K, seed, device, min_bytes, max_count=512):
+    """Distinct packed matrices: one seeded bf16 matrix quantised by the
+    library, then row-rotated copies (different contents, same statistics)."""
+    import torch
+    W = si.weights(N, K, seed=seed, dtype="bf16").torch(device)
+    packed, gamma = bl.bl_quant_weights(W, EPS)
+    del W
+    count = max(1, min(max_count, math.ceil(min_bytes / packed.numel())))
+    pool = [packed] + [torch.roll(packed, shifts=37 * i, dims=0).contiguous() for i in range(1, count)]
+    return pool, gamma
+
+
+# ---------------------------------------------------------------------------
+# decode (headline)
+
+def run_decode(bl, device, steps, warmup, peaks, world):
+    import torch
+    M, K, N = DECODE["M"], DECODE["K"], DECODE["N"]
+    stream = torch.cuda.Stream(device)
+    l2 = l2_bytes(device.index)
+    pool, gamma = weight_pool(bl, N, K, 0, device, 3 * l2)
+    tok = si.activations(CALLS_PER_STEP, K, seed=0, dtype="bf16").torch(device)
+    Y = torch.empty((CALLS_PER_STEP, N), dtype=torch.bfloat16, device=device)
+
+    def chain():
+        for i in range(CALLS_PER_STEP):
+            bl.bl_linear(tok[i:i + 1], pool[i % len(pool)], gamma, EPS, out=Y[i:i + 1],
+                         pdl=True, stream=stream)
+
+    graph = capture(chain, stream)
+    for _ in range(max(3, warmup)):
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier(device)
+    torch.cuda.synchronize()
+    with ClockSampler(device.index) as clk:
+        t = time_graph(graph, stream, steps)
+    torch.cuda.synchronize()
+    barrier(device)
+    t_max = reduce_max(t, device)
+    status = bl.bl_check_device_error(stream)
+    if status != 0:
+        raise RuntimeError(f"device error flag {status} after decode timing")
+
+    launch_s = t / (steps * CALLS_PER_STEP)
+    alg_bytes = N * K // 4 + M * K * 2 + M * N * 2
+    achieved = alg_bytes / launch_s / 1e9
+    res = {
+        "value": aggregate(steps * CALLS_PER_STEP * M, t_max, world),
+        "ms_per_step": t_max / steps * 1e3,
+        "launch_us": launch_s * 1e6,
+        "alg_bytes": alg_bytes,
+        "achieved_gbs": achieved,
+        "pool": {"matrices": len(pool), "bytes": len(pool) * pool[0].numel(), "l2_bytes": l2},
+        "clocks": clk.summary(),
+        "launches": steps * CALLS_PER_STEP,
+    }
+
+    # End to end through the public API: per step, copy the step's 1000
+    # tokens from pinned host memory, run the chain, copy the 1000 outputs back.
+    h_tok = tok.cpu().pin_memory()
+    h_out = torch.empty(Y.shape, dtype=Y.dtype, pin_memory=True)
+    e2e_steps = max(10, min(steps, 200))
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            tok.copy_(h_tok, non_blocking=True)
+            graph.replay()
+            h_out.copy_(Y, non_blocking=True)
+        stream.synchronize()
+        barrier(device)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(e2e_steps):
+            tok.copy_(h_tok, non_blocking=True)
+            graph.replay()
+            h_out.copy_(Y, non_blocking=True)
+        e.record(stream)
+        e.synchronize()
+    te = reduce_max(s.elapsed_time(e) / 1e3, device)
+    res["e2e"] = {"value": aggregate(e2e_steps * CALLS_PER_STEP * M, te, world), "unit": UNIT,
+                  "h2d_bytes_per_step": h_tok.numel() * h_tok.element_size(),
+                  "d2h_bytes_per_step": h_out.numel() * h_out.element_size()}
+
+    # Single isolated call (no PDL overlap, weights cold in L2).
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=device)
+    lat = []
+    with torch.cuda.stream(stream):
+        for i in range(20):
+            flush.fill_(i & 0xFF)
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            bl.bl_linear(tok[0:1], pool[i % len(pool)], gamma, EPS, out=Y[0:1], stream=stream)
+            e.record(stream)
+            e.synchronize()
+            lat.append(s.elapsed_time(e) * 1e3)
+    res["single_call_us_median"] = statistics.median(lat[3:])
+    del graph
+    return res
+
+
+# ---------------------------------------------------------------------------
+# secondary workloads
+
+def run_small_batch(bl, device, peaks, reps=200):
+    import torch
+    M, K, N = 16, 4096, 11008
+    stream = torch.cuda.Stream(device)
+    pool, gamma = weight_pool(bl, N, K, 0, device, 3 * l2_bytes(device.index))
+    A = si.activations(M, K, seed=0, dtype="bf16").torch(device)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    ws = torch.empty(bl.workspace_bytes("linear", M, K, N), dtype=torch.uint8, device=device)
+    calls = len(pool)
+
+    def chain():
+        for i in range(calls):
+            bl.bl_linear(A, pool[i], gamma, EPS, out=Y, workspace=ws, stream=stream)
+
+    g = capture(chain, stream)
+    for _ in range(3):
+        g.replay()
+    t = time_graph(g, stream, max(1, reps // calls)) / max(1, reps // calls) / calls
+    alg = N * K // 4 + M * K * 2 + M * N * 2
+    del g
+    return {"workload": "16 tokens, K=4096 -> N=11008, bf16, rotating weight pool > L2",
+            "tokens_per_s": M / t, "us_per_call": t * 1e6,
+            "gbs": alg / t / 1e9, "hbm_frac": alg / t / 1e9 / peaks["hbm_gbs"],
+            "tops": 2.0 * M * N * K / t / 1e12}
+
+
+def per_launch_times(fn, stream, reps, flush):
+    """Per-launch device time (s) of fn() with an L2 flush between launches."""
+    import torch
+    ts = []
+    with torch.cuda.stream(stream):
+        for i in range(reps):
+            flush.fill_(i & 0xFF)
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            fn()
+            e.record(stream)
+            e.synchronize()
+            ts.append(s.elapsed_time(e) / 1e3)
+    return ts
+
+
+def run_prefill(bl, device, peaks, reps=30):
+    import torch
+    M, K, N = 2048, 4096, 4096
+    stream = torch.cuda.Stream(device)
+    W = si.weights(N, K, seed=0, dtype="bf16").torch(device)
+    packed, gamma = bl.bl_quant_weights(W, EPS)
+    del W
+    A = si.activations(M, K, seed=0, dtype="bf16").torch(device)
+    flush = torch.empty(2 * l2_bytes(device.index), dtype=torch.uint8, device=device)
+    with torch.cuda.stream(stream):
+        Aq, gA, rs = bl.bl_quant_acts(A, EPS, stream=stream)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        for _ in range(3):
+            bl.bl_linear_q(Aq, gA, packed, gamma, rowsum=rs, out=Y, stream=stream)
+    tq = per_launch_times(lambda: bl.bl_quant_acts(A, EPS, stream=stream), stream, reps, flush)
+    tg = per_launch_times(lambda: bl.bl_linear_q(Aq, gA, packed, gamma, rowsum=rs, out=Y,
+                                                 stream=stream), stream, reps, flush)
+    tq, tg = statistics.median(tq[2:]), statistics.median(tg[2:])
+    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    ops = 2.0 * M * N * K
+    return {"workload": "2048 tokens, K=4096 -> N=4096, int8 x ternary on tcgen05 kind::i8, bf16 out",
+            "gemm_us": tg * 1e6, "quant_acts_us": tq * 1e6,
+            "tokens_per_s": M / (tg + tq), "gemm_tops": ops / tg / 1e12,
+            "roofline": {"bound": "tensor", "achieved": ops / tg / 1e12, "peak": int8_peak,
+                         "unit": "TOPS", "frac": ops / tg / 1e12 / int8_peak,
+                         "peak_source": f"{peaks['source']} bf16 burst x {INT8_OVER_BF16:g} (nominal int8/bf16)"},
+            "quant_acts_gbs": (M * K * 2 + M * K + 8 * M) / tq / 1e9}
+
+
+def run_ffn(bl, device, peaks, Ms=(1, 64, 512), reps=30):
+    import torch
+    K, H = 4096, 11008
+    stream = torch.cuda.Stream(device)
+    Wu = si.weights(H, K, seed=1, dtype="bf16").torch(device)
+    pu, gu = bl.bl_quant_weights(Wu, EPS)
+    del Wu
+    Wd = si.weights(K, H, seed=2, dtype="bf16").torch(device)
+    pd, gd = bl.bl_quant_weights(Wd, EPS)
+    del Wd
+    flush = torch.empty(2 * l2_bytes(device.index), dtype=torch.uint8, device=device)
+    out = {}
+    for M in Ms:
+        X = si.activations(M, K, seed=0, dtype="bf16").torch(device)
+        Y = torch.empty((M, K), dtype=torch.bfloat16, device=device)
+        ws = torch.empty(max(1, bl.workspace_bytes("ffn", M, K, H)), dtype=torch.uint8, device=device)
+        fn = lambda: bl.bl_ffn_relu2(X, pu, gu, pd, gd, EPS, out=Y, workspace=ws, stream=stream)
+        with torch.cuda.stream(stream):
+            fn()
+        t = statistics.median(per_launch_times(fn, stream, reps, flush)[2:])
+        wbytes = 2 * H * K // 4
+        out[f"M{M}"] = {"us": t * 1e6, "tokens_per_s": M / t, "weight_gbs": wbytes / t / 1e9,
+                        "tops": 4.0 * M * K * H / t / 1e12}
+    return out
+
+
+def run_quant_weights(bl, device, reps=10):
+    import torch
+    N, K = 11008, 4096
+    stream = torch.cuda.Stream(device)
+    W = si.weights(N, K, seed=0, dtype="bf16").torch(device)
+    out = torch.empty((N, K // 4), dtype=torch.uint8, device=device)
+    gamma = torch.empty((1,), dtype=torch.float32, device=device)
+    ws = torch.empty(bl.workspace_bytes("quant_weights", 0, K, N), dtype=torch.uint8, device=device)
+    flush = torch.empty(2 * l2_bytes(device.index), dtype=torch.uint8, device=device)
+    fn = lambda: bl.bl_quant_weights(W, EPS, out=out, gamma=gamma, workspace=ws, stream=stream)
+    with torch.cuda.stream(stream):
+        fn()
+    t = statistics.median(per_launch_times(fn, stream, reps, flush)[2:])
+    alg = N * K * 2 * 2 + N * K // 4  # W read twice (γ pass, pack pass) + packed write
+    return {"workload": "11008x4096 bf16 -> 2-bit packed", "us": t * 1e6,
+            "gbs": alg / t / 1e9, "weights_per_s": N * K / t}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and --impl reference)
+
+def oracle_decode_rate(seconds: float = 12.0, max_calls: int | None = None):
+    """Oracle BitLinear forward on the decode workload, one token per call,
+    for about `seconds` (or `max_calls`). Returns (tokens/s, calls, threads)."""
+    import oracle
+    M, K, N = DECODE["M"], DECODE["K"], DECODE["N"]
+    W = si.weights(N, K, seed=0, dtype="bf16").f32
+    codes, g = oracle.quant_weights(W, EPS)
+    tok = si.activations(64, K, seed=0, dtype="bf16").f32
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.bitlinear(tok[n % 64:n % 64 + 1], codes, g, EPS)
+        n += 1
+        el = time.perf_counter() - t0
+        if (max_calls is not None and n >= max_calls) or (max_calls is None and el >= seconds):
+            break
+    return n * M / el, n, oracle.max_threads()
+
+
+def run_reference(args):
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    import synth_inputs  # noqa: F401
+    # warm-up calls, then the timed steps: one step = one decode call (1 token).
+    oracle_decode_rate(max_calls=max(1, args.warmup))
+    rate, n, cores = oracle_decode_rate(max_calls=max(1, args.steps))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 / rate, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8xternary->int32, fp32 scales", "data": "synthetic",
+        "config": {"workload": "decode GEMV: 1 token, K=2560, N=6912, bf16 in/out",
+                   "step": "one BitLinear call (1 token) of the CPU oracle"},
+        "cpu_baseline": {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{n} decode calls (1 token each) after {args.warmup} warm-up calls"},
+        "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    args.warmup = max(3, args.warmup)
+
+    import torch
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import ternary_weight_linear_absmax_b200 as bl
+    bl.load()
+    peaks = load_peaks()
+
+    dec = run_decode(bl, device, args.steps, args.warmup, peaks, ws)
+    extra = {}
+    if not args.no_extra and rank == 0:
+        extra["decode_single_call_us"] = dec["single_call_us_median"]
+        extra["decode_pool"] = dec["pool"]
+        extra["small_batch"] = run_small_batch(bl, device, peaks)
+        extra["prefill"] = run_prefill(bl, device, peaks)
+        extra["ffn"] = run_ffn(bl, device, peaks)
+        extra["quant_weights"] = run_quant_weights(bl, device)
+    cpu = None
+    if rank == 0 and ws == 1:
+        rate, n, cores = oracle_decode_rate(seconds=args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{n} decode calls (1 token, K=2560, N=6912) in ~{args.cpu_seconds:g} s"}
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    traffic = profiled_traffic()
+    line = {
+        "metric": METRIC, "value": dec["value"], "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dec["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8 x ternary -> int32 (bf16 in/out, fp32 scales)", "data": "synthetic",
+        "config": {"workload": "decode GEMV: 1 token, K=2560, N=6912, bf16 in/out, 1% x20 outlier channels",
+                   "calls_per_step": CALLS_PER_STEP, "launch": "CUDA graph, programmatic dependent launch",
+                   "l2": f"no flush: rotating pool of {dec['pool']['matrices']} packed matrices "
+                         f"({dec['pool']['bytes'] / 1e6:.0f} MB) > 3x L2",
+                   "parallelism": f"replicas x{ws}"},
+        "roofline": {"bound": "hbm", "achieved": dec["achieved_gbs"], "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": dec["achieved_gbs"] / peaks["hbm_gbs"],
+                     "traffic": traffic, "kernel": "gemv_ternary_kernel",
+                     "alg_bytes_per_launch": dec["alg_bytes"], "launch_us": dec["launch_us"],
+                     "peak_source": f"{peaks['source']} hbm_gbs"},
+        "cpu_baseline": cpu,
+        "e2e": dec["e2e"],
+        "gpu_launches": dec["launches"],
+        "clocks": dec["clocks"],
+        "extra": extra,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

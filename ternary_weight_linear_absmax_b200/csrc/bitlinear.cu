@@ -195,10 +195,10 @@ FfnWs ffn_ws(int64_t M, int64_t K, int64_t H) {
 
 // --------------------------------------------------------------------------
 // GEMV launches.
-template <int MT, int RPL, typename TA, int SRC, int OUT>
-bl_status launch_gemv_t(const GemvParams& p, int grid, size_t smem, bool pdl, int dev,
-                        cudaStream_t st) {
-  auto* k = gemv_ternary_kernel<MT, RPL, TA, SRC, OUT>;
+template <int MT, typename TA, int SRC, int OUT>
+bl_status launch_gemv_t(const CUtensorMap& tw, const GemvParams& p, int grid, size_t smem,
+                        bool pdl, int dev, cudaStream_t st) {
+  auto* k = gemv_ternary_kernel<MT, TA, SRC, OUT>;
   BL_TRY(ensure_smem(k, dev, smem));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -210,44 +210,32 @@ bl_status launch_gemv_t(const GemvParams& p, int grid, size_t smem, bool pdl, in
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  BL_CUDA(cudaLaunchKernelEx(&cfg, k, p));
+  BL_CUDA(cudaLaunchKernelEx(&cfg, k, tw, p));
   return BL_OK;
 }
 
-template <int MT, typename TA, int SRC, int OUT>
-bl_status launch_gemv_rpl(const GemvParams& p, int rpl, int grid, size_t smem, bool pdl, int dev,
-                          cudaStream_t st) {
-  switch (rpl) {
-    case 1: return launch_gemv_t<MT, 1, TA, SRC, OUT>(p, grid, smem, pdl, dev, st);
-    case 2: return launch_gemv_t<MT, 2, TA, SRC, OUT>(p, grid, smem, pdl, dev, st);
-    case 3: return launch_gemv_t<MT, 3, TA, SRC, OUT>(p, grid, smem, pdl, dev, st);
-    default: return launch_gemv_t<MT, 4, TA, SRC, OUT>(p, grid, smem, pdl, dev, st);
-  }
-}
-
 template <typename TA, int SRC, int OUT>
-bl_status launch_gemv_mt(const GemvParams& p, int rpl, int grid, size_t smem, bool pdl, int dev,
-                         cudaStream_t st) {
+bl_status launch_gemv_mt(const CUtensorMap& tw, const GemvParams& p, int grid, size_t smem,
+                         bool pdl, int dev, cudaStream_t st) {
   // Token counts 1 and 2 get their own instantiations (fewer registers);
   // 3 and 4 share MT = 4 with runtime guards.
-  if (p.M == 1) return launch_gemv_rpl<1, TA, SRC, OUT>(p, rpl, grid, smem, pdl, dev, st);
-  if (p.M == 2) return launch_gemv_rpl<2, TA, SRC, OUT>(p, rpl, grid, smem, pdl, dev, st);
-  return launch_gemv_rpl<4, TA, SRC, OUT>(p, rpl, grid, smem, pdl, dev, st);
+  if (p.M == 1) return launch_gemv_t<1, TA, SRC, OUT>(tw, p, grid, smem, pdl, dev, st);
+  if (p.M == 2) return launch_gemv_t<2, TA, SRC, OUT>(tw, p, grid, smem, pdl, dev, st);
+  return launch_gemv_t<4, TA, SRC, OUT>(tw, p, grid, smem, pdl, dev, st);
 }
 
-constexpr size_t kGemvSmemCap = 200 * 1024;
+// Two CTAs per SM (228 KiB shared memory per SM, 1 KiB reserved per CTA).
+constexpr size_t kGemvSmemCap = 112 * 1024;
 
 // Choose rows per CTA: one wave over the SMs when shared memory allows,
-// at most 128 rows (4 per lane).
-bl_status gemv_plan(int64_t N, int64_t K, int M, int sms, int* rows, int* rpl, int* grid,
-                    size_t* smem) {
+// at most kGemvMaxRows rows.
+bl_status gemv_plan(int64_t N, int64_t K, int M, int sms, int* rows, int* grid, size_t* smem) {
   int64_t r = (N + sms - 1) / sms;
   if (r < 1) r = 1;
-  if (r > 128) r = 128;
+  if (r > kGemvMaxRows) r = kGemvMaxRows;
   while (r > 1 && gemv_smem_bytes(K, (int)r, M) > kGemvSmemCap) r = (r + 1) / 2;
   if (gemv_smem_bytes(K, (int)r, M) > kGemvSmemCap) return BL_ERR_SHAPE;
   *rows = (int)r;
-  *rpl = (int)((r + 31) / 32);
   *grid = (int)((N + r - 1) / r);
   *smem = gemv_smem_bytes(K, (int)r, M);
   return BL_OK;
@@ -256,26 +244,29 @@ bl_status gemv_plan(int64_t N, int64_t K, int M, int sms, int* rows, int* rpl, i
 // src: kSrcFloat (a_dtype says f32/bf16), kSrcFfnRequant, kSrcInt8.
 bl_status run_gemv(int src, int out, bl_dtype a_dtype, GemvParams p, bool pdl, int dev, int sms,
                    cudaStream_t st) {
-  int rows, rpl, grid;
+  int rows, grid;
   size_t smem;
-  BL_TRY(gemv_plan(p.N, p.K, p.M, sms, &rows, &rpl, &grid, &smem));
+  BL_TRY(gemv_plan(p.N, p.K, p.M, sms, &rows, &grid, &smem));
   p.rows_per_cta = rows;
-  p.pitch = gemv_pitch(p.K);
+  p.rows_pad = gemv_rows_pad(rows);
+  CUtensorMap tw;
+  BL_TRY(make_map_u8(&tw, p.W, (uint64_t)p.N, (uint64_t)(p.K / 4), 128, (uint32_t)p.rows_pad,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
   if (src == kSrcFloat) {
     if (a_dtype == BL_BF16) {
       return out == kOutDequant
-                 ? launch_gemv_mt<__nv_bfloat16, kSrcFloat, kOutDequant>(p, rpl, grid, smem, pdl, dev, st)
-                 : launch_gemv_mt<__nv_bfloat16, kSrcFloat, kOutRawI32>(p, rpl, grid, smem, pdl, dev, st);
+                 ? launch_gemv_mt<__nv_bfloat16, kSrcFloat, kOutDequant>(tw, p, grid, smem, pdl, dev, st)
+                 : launch_gemv_mt<__nv_bfloat16, kSrcFloat, kOutRawI32>(tw, p, grid, smem, pdl, dev, st);
     }
     return out == kOutDequant
-               ? launch_gemv_mt<float, kSrcFloat, kOutDequant>(p, rpl, grid, smem, pdl, dev, st)
-               : launch_gemv_mt<float, kSrcFloat, kOutRawI32>(p, rpl, grid, smem, pdl, dev, st);
+               ? launch_gemv_mt<float, kSrcFloat, kOutDequant>(tw, p, grid, smem, pdl, dev, st)
+               : launch_gemv_mt<float, kSrcFloat, kOutRawI32>(tw, p, grid, smem, pdl, dev, st);
   }
   if (src == kSrcFfnRequant)
-    return launch_gemv_mt<float, kSrcFfnRequant, kOutDequant>(p, rpl, grid, smem, pdl, dev, st);
+    return launch_gemv_mt<float, kSrcFfnRequant, kOutDequant>(tw, p, grid, smem, pdl, dev, st);
   return out == kOutDequant
-             ? launch_gemv_mt<float, kSrcInt8, kOutDequant>(p, rpl, grid, smem, pdl, dev, st)
-             : launch_gemv_mt<float, kSrcInt8, kOutRawI32>(p, rpl, grid, smem, pdl, dev, st);
+             ? launch_gemv_mt<float, kSrcInt8, kOutDequant>(tw, p, grid, smem, pdl, dev, st)
+             : launch_gemv_mt<float, kSrcInt8, kOutRawI32>(tw, p, grid, smem, pdl, dev, st);
 }
 
 // --------------------------------------------------------------------------

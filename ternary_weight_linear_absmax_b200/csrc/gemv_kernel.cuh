@@ -5,21 +5,30 @@
 // contraction, then one scale (γ_A·γ)/127) and "Como o BitNet quebra o Memory
 // Wall ..." (decode streams 0.25 byte per weight; the kernel is HBM-bound).
 //
-// Design (one launch per call):
-//  * Each CTA owns a contiguous slab of R weight rows. Its first warp issues
-//    one bulk copy (TMA, cp.async.bulk) per row into shared memory before
-//    anything else — with programmatic dependent launch this happens while
-//    the previous kernel on the stream is still running.
-//  * The CTA then waits for the previous grid (griddepcontrol.wait) and
-//    quantises the M tokens into shared memory (AbsMax prologue), or
-//    requantises the FFN intermediate, or copies pre-quantised int8 tokens.
-//  * Warps split K, lanes split rows: lane l of warp w handles rows l, l+32,
-//    ... and 64-weight chunks w, w+8, .... Weight rows sit in shared memory
-//    at a pitch chosen so a quarter-warp's 16-byte loads hit 8 distinct bank
-//    groups; activations are read as broadcasts.
-//  * Codes c = w+1 ∈ {0,1,2} are used directly as int8 operands of dp4a:
-//    Σ c·a = Σ w·a + Σ a, so the token's Σ a is subtracted once per row.
-//  * Partial sums of the 8 warps are combined in shared memory; the epilogue
+// Design (one launch per call, 512 threads per CTA, two CTAs per SM so the
+// next call's CTA can already be resident):
+//  * Each CTA owns a contiguous slab of R ≤ 128 weight rows. One thread
+//    issues K/512 tensor copies (TMA, 128-byte swizzle) of R rows × 128
+//    bytes each into shared memory before anything else. With programmatic
+//    dependent launch this happens while the previous kernel on the stream
+//    is still running, so in a decode chain the weight stream overlaps the
+//    previous layer's work.
+//  * The CTA then waits for the previous grid (griddepcontrol.wait) and runs
+//    the token prologue in one pass over global memory: AbsMax quantisation
+//    of the tokens, or the FFN ReLU² requantisation, or a copy of int8 tokens.
+//  * Thread t owns row t mod R and the chunk group t / R (every CG-th
+//    64-weight chunk of that row), which spreads R·K/64 chunk tasks evenly
+//    over the 512 threads. The swizzle places 16-byte chunk j of row r at
+//    position j ^ (r mod 8) of its 128-byte line, so consecutive lanes
+//    (consecutive rows, same chunk) load without bank conflicts; token words
+//    are broadcast loads.
+//  * Contraction with codes c = w+1 ∈ {0,1,2}: a packed word x holds, in byte
+//    i, the codes of weights 4j+i at bits 2j. For each j, x & (3·0x01010101
+//    << 2j) is a vector of four unsigned bytes c·4^j, so one LOP3 and one
+//    dp4a (unsigned × signed) per 4 weights accumulate 4^j·Σ c·a into acc[j];
+//    Σ c·a = acc[0] + acc[1]/4 + acc[2]/16 + acc[3]/64 exactly. Σ w·a is then
+//    Σ c·a − Σ a, with Σ a (the token's row sum) taken once.
+//  * Per-warp partial sums are combined in shared memory; the epilogue
 //    applies (γ_A·γ)/127 (and ReLU²) or writes the raw INT32 result.
 #pragma once
 
@@ -27,9 +36,13 @@
 
 namespace bl {
 
-constexpr int kGemvThreads = 256;
+constexpr int kGemvThreads = 512;
 constexpr int kGemvWarps = kGemvThreads / 32;
 constexpr int kGemvMaxTokens = 4;
+constexpr int kGemvMaxRows = 128;
+// 16-byte token vectors kept in registers per thread and token.
+template <int MT>
+__host__ __device__ constexpr int gemv_reg_vecs() { return MT == 1 ? 4 : (MT == 2 ? 2 : 1); }
 
 enum GemvSrc : int { kSrcFloat = 0, kSrcFfnRequant = 1, kSrcInt8 = 2 };
 enum GemvOut : int { kOutDequant = 0, kOutRawI32 = 1 };
@@ -40,55 +53,94 @@ struct GemvParams {
   const float* a_gamma_up;  // kSrcFfnRequant: γ_up (1 value)
   const int32_t* a_rowsum;  // kSrcInt8: Σ A_q per token, or nullptr
   const uint8_t* W;         // packed [N, K/4]
-  const float* gamma;       // γ of W (1 value)
+  const float* gamma;       // γ of W (1 value); may be null for raw output
   void* Y;                  // kOutDequant: float/bf16 [M,N]; kOutRawI32: int32 [M,N]
-  float* gamma_out;         // optional: per-token γ_A written by CTA 0
+  float* gamma_out;         // optional: per-token γ_A (or γ_r) written by CTA 0
   int64_t N;
   int64_t K;
   int rows_per_cta;
-  int pitch;  // bytes between weight rows in shared memory
+  int rows_pad;  // rows per CTA rounded up to 8 (rows of one swizzled box)
   int M;
   float eps;
   int relu2;
   int y_bf16;
 };
 
-__host__ __device__ inline int gemv_pitch(int64_t K) {
-  // Row pitch in 32-bit words ≡ 4 (mod 8): 16-byte loads of 8 consecutive
-  // lanes (8 consecutive rows) then cover all 32 banks exactly once.
-  const int w = (int)(K / 16);
-  return 4 * (w + ((4 - (w % 8)) + 8) % 8);
+// Shared memory holds the slab as K/512 boxes of rows_pad × 128 bytes.
+__host__ __device__ inline int gemv_boxes(int64_t K) { return (int)((K / 4 + 127) / 128); }
+__host__ __device__ inline int gemv_rows_pad(int rows) { return (rows + 7) & ~7; }
+
+// Chunk groups per row: as many as the 512 threads allow, at most one per
+// 64-weight chunk.
+__host__ __device__ inline int gemv_chunk_groups(int rows, int64_t K) {
+  int cg = kGemvThreads / (rows > 0 ? rows : 1);
+  const int nchunks = (int)(K / 64);
+  if (cg > nchunks) cg = nchunks;
+  return cg < 1 ? 1 : cg;
 }
 
-// Shared memory: [0,128) mbarrier + per-token scalars; then R weight rows at
-// the padded pitch; then the int8 tokens; then the per-warp partial sums.
-constexpr int kGemvHeader = 128;
+// Shared memory: [0,1024) mbarrier + per-token scalars; then the weight
+// boxes (1024-byte aligned, as the 128-byte swizzle requires); then the int8
+// tokens; then the per-warp partial sums.
+constexpr int kGemvHeader = 1024;
 
 __host__ __device__ inline size_t gemv_smem_bytes(int64_t K, int rows, int M) {
   size_t s = kGemvHeader;
-  s += (size_t)rows * gemv_pitch(K);                  // weights
-  s += (size_t)M * K;                                  // int8 activations
-  s += (size_t)kGemvWarps * M * rows * sizeof(int);    // warp partials
-  return (s + 127) & ~(size_t)127;
+  s += (size_t)gemv_boxes(K) * gemv_rows_pad(rows) * 128;  // weights
+  s += (size_t)M * K;                                      // int8 tokens
+  s += (size_t)kGemvThreads * M * sizeof(int);             // per-thread partial sums
+  return s + 1024;                                         // base alignment slack
 }
 
-template <int MT, int RPL, typename TA, int SRC, int OUT>
-__global__ void __launch_bounds__(kGemvThreads, 1) gemv_ternary_kernel(const GemvParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];
+// d = Σ_i ua[i]·sb[i] + c over the four bytes; a unsigned, b signed.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Block-wide max of MT values per thread: warp shuffles, one barrier, then
+// every thread reads the per-warp maxima (no second barrier).
+template <int MT>
+__device__ __forceinline__ void block_max_all(float (&v)[MT], float (*red)[MT]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    float t = warp_max(v[m]);
+    if (lane == 0) red[warp][m] = t;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    float t = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kGemvWarps; ++w) t = fmaxf(t, red[w][m]);
+    v[m] = t;
+  }
+}
+
+template <int MT, typename TA, int SRC, int OUT>
+__global__ void __launch_bounds__(kGemvThreads, 2)
+gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p) {
+  constexpr int kGemvRegVecs = gemv_reg_vecs<MT>();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  __shared__ float s_redf[kGemvWarps][MT];
+  __shared__ int s_redi[kGemvWarps][MT];
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int64_t K = p.K;
-  const int kbytes = (int)(K / 4);
   const int64_t r0 = (int64_t)blockIdx.x * p.rows_per_cta;
   const int R = (int)min((int64_t)p.rows_per_cta, p.N - r0);
   const int M = p.M;
 
   uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem);
-  float* s_sc = reinterpret_cast<float*>(smem + 16);   // [MT] dequant scale (γ_A·γ)/127
-  int* s_sum = reinterpret_cast<int*>(smem + 32);      // [MT] Σ A_q
-  float* s_tok = reinterpret_cast<float*>(smem + 48);  // [MT] token scale γ_A (or γ_r)
+  float* s_sc = reinterpret_cast<float*>(smem + 16);  // [MT] dequant scale (γ_A·γ)/127
   uint8_t* s_w = smem + kGemvHeader;
-  int8_t* s_a = reinterpret_cast<int8_t*>(s_w + (size_t)p.rows_per_cta * p.pitch);
+  const int nbox = gemv_boxes(K);
+  const int box_bytes = p.rows_pad * 128;
+  int8_t* s_a = reinterpret_cast<int8_t*>(s_w + (size_t)nbox * box_bytes);
   int* s_part = reinterpret_cast<int*>(s_a + (size_t)M * K);
 
   // 1. Stream this CTA's weight rows into shared memory (independent of the
@@ -98,275 +150,211 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_ternary_kernel(const Gem
     fence_barrier_init();
   }
   __syncthreads();
-  if (warp == 0) {
-    if (lane == 0) mbar_arrive_expect_tx(s_bar, (uint32_t)R * (uint32_t)kbytes);
-    __syncwarp();
-    for (int i = lane; i < R; i += 32)
-      bulk_g2s(s_w + (size_t)i * p.pitch, p.W + (r0 + i) * kbytes, (uint32_t)kbytes, s_bar);
+  if (tid == 0) {
+    mbar_arrive_expect_tx(s_bar, (uint32_t)nbox * (uint32_t)box_bytes);
+    for (int b = 0; b < nbox; ++b)
+      tma_load_2d(s_w + (size_t)b * box_bytes, &tm_w, b * 128, (int32_t)r0, s_bar);
+  } else if (tid == 32) {
+    // Warm L2 with the tokens (the reads themselves wait for the prior grid).
+    const size_t tok_bytes = (size_t)M * K *
+        (SRC == kSrcFloat ? sizeof(TA) : (SRC == kSrcFfnRequant ? 4 : 1));
+    for (size_t o = 0; o < tok_bytes; o += 65536)
+      prefetch_l2(reinterpret_cast<const uint8_t*>(p.A) + o,
+                  (uint32_t)min((size_t)65536, tok_bytes - o));
   }
+  // γ of W is as static as W itself (see BL_FLAG_PDL), so it is read before
+  // the dependency wait.
+  const float gamma_w = p.gamma != nullptr ? __ldg(p.gamma) : 0.0f;
   pdl_launch_dependents();
-  // 2. Activations and outputs are ordered after the previous kernel.
-  pdl_wait_prior_grid();
+  // 2. Tokens and outputs are ordered after the previous kernel. One warp
+  //    waits for the prior grid; the others wait at the CTA barrier, so a CTA
+  //    launched early spends no issue slots while its predecessor runs.
+  if (warp == 0) pdl_wait_prior_grid();
+  __syncthreads();
 
-  // 3. Token prologue → int8 tokens in shared memory, Σ A_q, scales.
-  if constexpr (SRC == kSrcFloat) {
-    __shared__ float red[kGemvWarps][MT];
-    const TA* A = reinterpret_cast<const TA*>(p.A);
-    constexpr int VEC = 16 / sizeof(TA);
+  // 3. Token prologue → int8 tokens in shared memory, Σ A_q and γ per token.
+  float tok_scale[MT];  // γ_A (float or int8 tokens) or γ_r (FFN requant)
+  int tok_sum[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) tok_sum[m] = 0;
+  if constexpr (SRC == kSrcFloat || SRC == kSrcFfnRequant) {
+    // Values per 16-byte vector and the value each element is quantised from.
+    constexpr int VEC = SRC == kSrcFloat ? 16 / (int)sizeof(TA) : 4;
     const int64_t nvec = K / VEC;
+    float scu[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) scu[m] = 0.0f;
+    if constexpr (SRC == kSrcFfnRequant) {
+      const float gup = *p.a_gamma_up;
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+        if (m < M) scu[m] = __fdiv_rn(__fmul_rn(p.a_scale[m], gup), 127.0f);
+    }
+    auto value = [&](const uint4& u, int i, int m) -> float {
+      if constexpr (SRC == kSrcFloat) {
+        return to_f32<TA>(reinterpret_cast<const TA*>(&u)[i]);
+      } else {
+        // r = max(h,0)² with h = fp32(acc · fp32((γ_X·γ_up)/127))
+        const float h =
+            fmaxf(__fmul_rn((float)reinterpret_cast<const int*>(&u)[i], scu[m]), 0.0f);
+        return __fmul_rn(h, h);
+      }
+    };
+    uint4 reg[MT][kGemvRegVecs];
     float mx[MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) mx[m] = 0.0f;
-    for (int64_t v = tid; v < nvec; v += kGemvThreads) {
+    for (int m = 0; m < MT; ++m) {
+      mx[m] = 0.0f;
+      if (m < M) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            reinterpret_cast<const uint8_t*>(p.A) + (size_t)m * (size_t)nvec * 16);
 #pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        if (m < M) {
-          uint4 u = __ldg(reinterpret_cast<const uint4*>(A + m * K) + v);
-          const TA* e = reinterpret_cast<const TA*>(&u);
+        for (int r = 0; r < kGemvRegVecs; ++r) {
+          const int64_t v = tid + (int64_t)r * kGemvThreads;
+          if (v < nvec) {
+            reg[m][r] = __ldg(src + v);
 #pragma unroll
-          for (int i = 0; i < VEC; ++i) mx[m] = fmaxf(mx[m], fabsf(to_f32<TA>(e[i])));
+            for (int i = 0; i < VEC; ++i) mx[m] = fmaxf(mx[m], fabsf(value(reg[m][r], i, m)));
+          }
+        }
+        for (int64_t v = tid + (int64_t)kGemvRegVecs * kGemvThreads; v < nvec; v += kGemvThreads) {
+          const uint4 u = __ldg(src + v);
+#pragma unroll
+          for (int i = 0; i < VEC; ++i) mx[m] = fmaxf(mx[m], fabsf(value(u, i, m)));
         }
       }
     }
+    block_max_all<MT>(mx, s_redf);
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
-      float t = warp_max(mx[m]);
-      if (lane == 0) red[warp][m] = t;
-    }
-    __syncthreads();
-    if (tid < MT) {
-      float t = 0.0f;
-      for (int w = 0; w < kGemvWarps; ++w) t = fmaxf(t, red[w][tid]);
-      s_tok[tid] = t;  // γ_A
-      if (tid < M && p.gamma_out != nullptr && blockIdx.x == 0) p.gamma_out[tid] = t;
-    }
-    __syncthreads();
-    int sum[MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) sum[m] = 0;
-    for (int64_t v = tid; v < nvec; v += kGemvThreads) {
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        if (m < M) {
-          const float s = __fdiv_rn(127.0f, __fadd_rn(s_tok[m], p.eps));
-          uint4 u = __ldg(reinterpret_cast<const uint4*>(A + m * K) + v);
-          const TA* e = reinterpret_cast<const TA*>(&u);
+      tok_scale[m] = mx[m];
+      if (m < M) {
+        const float s = __fdiv_rn(127.0f, __fadd_rn(mx[m], p.eps));
+        const uint4* src = reinterpret_cast<const uint4*>(
+            reinterpret_cast<const uint8_t*>(p.A) + (size_t)m * (size_t)nvec * 16);
+        auto emit = [&](const uint4& u, int64_t v) {
           int8_t q[VEC];
 #pragma unroll
           for (int i = 0; i < VEC; ++i) {
-            q[i] = quant_i8(to_f32<TA>(e[i]), s);
-            sum[m] += q[i];
+            q[i] = quant_i8(value(u, i, m), s);
+            tok_sum[m] += q[i];
           }
           if constexpr (VEC == 8)
             *reinterpret_cast<uint2*>(s_a + m * K + v * VEC) = *reinterpret_cast<uint2*>(q);
           else
             *reinterpret_cast<uint32_t*>(s_a + m * K + v * VEC) = *reinterpret_cast<uint32_t*>(q);
+        };
+#pragma unroll
+        for (int r = 0; r < kGemvRegVecs; ++r) {
+          const int64_t v = tid + (int64_t)r * kGemvThreads;
+          if (v < nvec) emit(reg[m][r], v);
         }
+        for (int64_t v = tid + (int64_t)kGemvRegVecs * kGemvThreads; v < nvec; v += kGemvThreads)
+          emit(__ldg(src + v), v);
       }
-    }
-    __shared__ int redi[kGemvWarps][MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      int t = warp_sum_i(sum[m]);
-      if (lane == 0) redi[warp][m] = t;
-    }
-    __syncthreads();
-    if (tid < MT) {
-      int t = 0;
-      for (int w = 0; w < kGemvWarps; ++w) t += redi[w][tid];
-      s_sum[tid] = t;
-    }
-  } else if constexpr (SRC == kSrcFfnRequant) {
-    // h = fp32(acc·fp32((γ_X·γ_up)/127)); r = max(h,0)²; γ_r = max r;
-    // q = Clip(Round(r·127/(γ_r+ε))).
-    __shared__ float red[kGemvWarps][MT];
-    const int32_t* A = reinterpret_cast<const int32_t*>(p.A);
-    const float gup = *p.a_gamma_up;
-    float scu[MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m)
-      scu[m] = m < M ? __fdiv_rn(__fmul_rn(p.a_scale[m], gup), 127.0f) : 0.0f;
-    const int64_t nvec = K / 4;
-    float mx[MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) mx[m] = 0.0f;
-    for (int64_t v = tid; v < nvec; v += kGemvThreads) {
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        if (m < M) {
-          int4 u = __ldg(reinterpret_cast<const int4*>(A + m * K) + v);
-          const int e[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            float h = fmaxf(__fmul_rn((float)e[i], scu[m]), 0.0f);
-            mx[m] = fmaxf(mx[m], __fmul_rn(h, h));
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      float t = warp_max(mx[m]);
-      if (lane == 0) red[warp][m] = t;
-    }
-    __syncthreads();
-    if (tid < MT) {
-      float t = 0.0f;
-      for (int w = 0; w < kGemvWarps; ++w) t = fmaxf(t, red[w][tid]);
-      s_tok[tid] = t;  // γ_r
-      if (tid < M && p.gamma_out != nullptr && blockIdx.x == 0) p.gamma_out[tid] = t;
-    }
-    __syncthreads();
-    int sum[MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) sum[m] = 0;
-    for (int64_t v = tid; v < nvec; v += kGemvThreads) {
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        if (m < M) {
-          const float s = __fdiv_rn(127.0f, __fadd_rn(s_tok[m], p.eps));
-          int4 u = __ldg(reinterpret_cast<const int4*>(A + m * K) + v);
-          const int e[4] = {u.x, u.y, u.z, u.w};
-          int8_t q[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            float h = fmaxf(__fmul_rn((float)e[i], scu[m]), 0.0f);
-            q[i] = quant_i8(__fmul_rn(h, h), s);
-            sum[m] += q[i];
-          }
-          *reinterpret_cast<uint32_t*>(s_a + m * K + v * 4) = *reinterpret_cast<uint32_t*>(q);
-        }
-      }
-    }
-    __shared__ int redi[kGemvWarps][MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      int t = warp_sum_i(sum[m]);
-      if (lane == 0) redi[warp][m] = t;
-    }
-    __syncthreads();
-    if (tid < MT) {
-      int t = 0;
-      for (int w = 0; w < kGemvWarps; ++w) t += redi[w][tid];
-      s_sum[tid] = t;
     }
   } else {  // kSrcInt8
     const int8_t* A = reinterpret_cast<const int8_t*>(p.A);
     const int64_t nvec = K / 16;
-    int sum[MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) sum[m] = 0;
-    for (int64_t v = tid; v < nvec; v += kGemvThreads) {
+    for (int m = 0; m < MT; ++m) {
+      tok_scale[m] = (m < M && p.a_scale != nullptr) ? p.a_scale[m] : 0.0f;
+      if (m < M) {
+        for (int64_t v = tid; v < nvec; v += kGemvThreads) {
+          uint4 u = __ldg(reinterpret_cast<const uint4*>(A + m * K) + v);
+          *reinterpret_cast<uint4*>(s_a + m * K + v * 16) = u;
+          tok_sum[m] = dp4a(u.x, 0x01010101u, tok_sum[m]);
+          tok_sum[m] = dp4a(u.y, 0x01010101u, tok_sum[m]);
+          tok_sum[m] = dp4a(u.z, 0x01010101u, tok_sum[m]);
+          tok_sum[m] = dp4a(u.w, 0x01010101u, tok_sum[m]);
+        }
+      }
+    }
+  }
+  // Per-warp token sums; combined in the epilogue after the next barrier.
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    const int t = warp_sum_i(tok_sum[m]);
+    if (lane == 0) s_redi[warp][m] = t;
+  }
+  if (tid < MT) {
+    float ts = 0.0f;
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+      if (m == tid) ts = tok_scale[m];
+    if constexpr (SRC != kSrcInt8) {
+      if (tid < M && p.gamma_out != nullptr && blockIdx.x == 0) p.gamma_out[tid] = ts;
+    }
+    s_sc[tid] = __fdiv_rn(__fmul_rn(ts, gamma_w), 127.0f);  // (γ_A·γ)/127
+  }
+  __syncthreads();
+
+  // 4. Weights must have landed: every thread observes the completed phase.
+  if (!mbar_wait(s_bar, 0)) {
+    // Gave up: the error flag is raised and this CTA's outputs stay
+    // untouched. The wait that gave up was the wait for its own copies.
+    return;
+  }
+
+  // 5. Contraction. Thread t < R·CG owns row t mod R and chunk group
+  //    t / R, i.e. the 64-weight chunks cg, cg + CG, ... of that row.
+  //    Consecutive lanes take consecutive rows at the same chunk: the
+  //    swizzle keeps their weight loads conflict-free and the token loads
+  //    are broadcasts.
+  const int CG = gemv_chunk_groups(R, K);
+  const int nchunks = (int)(K / 64);
+  const bool active = tid < R * CG;
+  const int row = active ? tid % R : 0;
+  const int cg = active ? tid / R : 0;
+  int acc[MT][4];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[m][j] = 0;
+  if (active) {
+    const uint8_t* wrow = s_w + (size_t)row * 128;
+    const int sw = row & 7;
+#pragma unroll 4
+    for (int c = cg; c < nchunks; c += CG) {
+      // chunk c: box c/8, 16-byte slot (c mod 8) XOR (row mod 8)
+      const uint4 wv = *reinterpret_cast<const uint4*>(wrow + (size_t)(c >> 3) * box_bytes +
+                                                       (((c & 7) ^ sw) << 4));
+      const uint32_t x[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
         if (m < M) {
-          uint4 u = __ldg(reinterpret_cast<const uint4*>(A + m * K) + v);
-          *reinterpret_cast<uint4*>(s_a + m * K + v * 16) = u;
-          sum[m] = dp4a(u.x, 0x01010101u, sum[m]);
-          sum[m] = dp4a(u.y, 0x01010101u, sum[m]);
-          sum[m] = dp4a(u.z, 0x01010101u, sum[m]);
-          sum[m] = dp4a(u.w, 0x01010101u, sum[m]);
-        }
-      }
-    }
-    __shared__ int redi[kGemvWarps][MT];
+          const uint4* ap = reinterpret_cast<const uint4*>(s_a + m * K + c * 64);
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      int t = warp_sum_i(sum[m]);
-      if (lane == 0) redi[warp][m] = t;
-    }
-    __syncthreads();
-    if (tid < MT) {
-      int t = 0;
-      for (int w = 0; w < kGemvWarps; ++w) t += redi[w][tid];
-      s_sum[tid] = (p.a_rowsum != nullptr && tid < M) ? p.a_rowsum[tid] : t;
-      s_tok[tid] = (tid < M && p.a_scale != nullptr) ? p.a_scale[tid] : 0.0f;
-    }
-  }
-  if (tid < MT) {
-    const float g = p.gamma != nullptr ? *p.gamma : 0.0f;  // absent for raw INT32 output
-    s_sc[tid] = __fdiv_rn(__fmul_rn(s_tok[tid], g), 127.0f);  // (γ_A·γ)/127
-  }
-  __syncthreads();
-
-  // 4. Weights must have landed.
-  __shared__ int s_ok;
-  if (tid == 0) s_ok = mbar_wait(s_bar, 0) ? 1 : 0;
-  __syncthreads();
-  // On give-up the error flag is raised and the outputs are left untouched.
-  // The wait that gave up was the wait for this CTA's own copies.
-  if (!s_ok) return;
-  // Each thread observes the completed phase itself (acquire of the
-  // bulk-copy writes); the phase is already complete, so this returns at once.
-  mbar_wait(s_bar, 0);
-
-  // 5. Contraction.
-  int acc[RPL][MT];
-#pragma unroll
-  for (int t = 0; t < RPL; ++t)
-#pragma unroll
-    for (int m = 0; m < MT; ++m) acc[t][m] = 0;
-  const int nchunks = (int)(K / 64);
-  for (int c = warp; c < nchunks; c += kGemvWarps) {
-    uint32_t a[MT][16];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      if (m < M) {
-        const uint4* src = reinterpret_cast<const uint4*>(s_a + m * K + c * 64);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint4 u = src[v];
-          a[m][4 * v + 0] = u.x;
-          a[m][4 * v + 1] = u.y;
-          a[m][4 * v + 2] = u.z;
-          a[m][4 * v + 3] = u.w;
-        }
-      } else {
-#pragma unroll
-        for (int v = 0; v < 16; ++v) a[m][v] = 0u;
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < RPL; ++t) {
-      const int i = lane + 32 * t;
-      if (i < R) {
-        const uint4 wv = *reinterpret_cast<const uint4*>(s_w + (size_t)i * p.pitch + c * 16);
-        const uint32_t x[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t e0, e1, e2, e3;
-          expand_word(x[q], e0, e1, e2, e3);
-#pragma unroll
-          for (int m = 0; m < MT; ++m) {
-            acc[t][m] = dp4a(e0, a[m][4 * q + 0], acc[t][m]);
-            acc[t][m] = dp4a(e1, a[m][4 * q + 1], acc[t][m]);
-            acc[t][m] = dp4a(e2, a[m][4 * q + 2], acc[t][m]);
-            acc[t][m] = dp4a(e3, a[m][4 * q + 3], acc[t][m]);
+          for (int q = 0; q < 4; ++q) {
+            const uint4 a = ap[q];  // token words 16c+4q .. 16c+4q+3
+            acc[m][0] = dp4a_us(x[q] & 0x03030303u, a.x, acc[m][0]);
+            acc[m][1] = dp4a_us(x[q] & 0x0C0C0C0Cu, a.y, acc[m][1]);
+            acc[m][2] = dp4a_us(x[q] & 0x30303030u, a.z, acc[m][2]);
+            acc[m][3] = dp4a_us(x[q] & 0xC0C0C0C0u, a.w, acc[m][3]);
           }
         }
       }
     }
-  }
-  const int RP = p.rows_per_cta;
+    // Σ c·a over this thread's chunks; acc[j] is a multiple of 4^j, so the
+    // arithmetic shifts are exact.
 #pragma unroll
-  for (int t = 0; t < RPL; ++t) {
-    const int i = lane + 32 * t;
-    if (i < R) {
-#pragma unroll
-      for (int m = 0; m < MT; ++m)
-        if (m < M) s_part[(warp * M + m) * RP + i] = acc[t][m];
-    }
+    for (int m = 0; m < MT; ++m)
+      if (m < M)
+        s_part[(m * CG + cg) * R + row] =
+            acc[m][0] + (acc[m][1] >> 2) + (acc[m][2] >> 4) + (acc[m][3] >> 6);
   }
   __syncthreads();
 
-  // 6. Epilogue: combine the warps, undo the code offset, scale.
+  // 6. Epilogue: combine the group's warps, undo the code offset, scale.
   for (int e = tid; e < M * R; e += kGemvThreads) {
-    const int m = e / R, i = e - m * R;
+    const int m = e / R, r = e - m * R;
     int d = 0;
+    for (int k = 0; k < CG; ++k) d += s_part[(m * CG + k) * R + r];
+    int ssum = 0;
 #pragma unroll
-    for (int w = 0; w < kGemvWarps; ++w) d += s_part[(w * M + m) * RP + i];
-    const int v = d - s_sum[m];
-    const int64_t o = (int64_t)m * p.N + r0 + i;
+    for (int w = 0; w < kGemvWarps; ++w) ssum += s_redi[w][m];
+    const int v = d - ssum;
+    const int64_t o = (int64_t)m * p.N + r0 + r;
     if constexpr (OUT == kOutRawI32) {
       reinterpret_cast<int32_t*>(p.Y)[o] = v;
     } else {
