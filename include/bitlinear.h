@@ -172,6 +172,37 @@ bl_status bl_linear_ex(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
                        bl_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * bl_linear_noalloc — bl_linear for callers that cannot allocate device memory.
+ * The pages have no counterpart: this is a deployment variant, not part of
+ * the method.
+ * Some callers own no device allocator on the path that runs the layer: a
+ * plugin whose host runtime hands it only its input and output buffers and
+ * owns every other byte of device memory, or a serving loop that must not
+ * call cudaMalloc on its hot path (cudaMalloc may synchronise the device and
+ * grows memory outside a fixed budget). This entry point takes the same
+ * arguments as bl_linear minus the workspace and allocates nothing: the
+ * scratch it needs for more than bl_gemv_max_tokens() tokens (the int8
+ * tokens, their scales and row sums: M·K + 8·M bytes, 256-byte aligned
+ * pieces) lives in one fixed 4 MiB array inside the library. Every GPU that
+ * loads the library holds that array until the process exits.
+ *   * Sizes whose scratch exceeds 4 MiB (bl_linear_workspace_bytes(M, K, N) >
+ *     4 MiB, e.g. M·K above about 4.1 million) are refused with
+ *     BL_ERR_WORKSPACE before anything is launched; use bl_linear then.
+ *   * The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   * All calls on a device share the array, which keeps whatever the last
+ *     call left in it. Nothing in it needs to start at zero (each call writes
+ *     every byte it reads), but calls whose kernels overlap on the GPU (for
+ *     example on two streams at once) race on it: order them on one stream.
+ * Arguments, layouts and the other errors are those of bl_linear.
+ */
+bl_status bl_linear_noalloc(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
+                            const uint8_t* W_packed, const float* gamma, int64_t N,
+                            float eps, int relu2, void* Y, bl_dtype y_dtype,
+                            bl_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * bl_ffn_relu2 — ternary FFN block (BitLinear up → ReLU² → BitLinear down).
  * Composition of the BLOG formulas with ReLUSquared (bit_layers.py): per
  * token, h = dequantised up-projection (fp32), r = max(h,0)² (fp32), AbsMax

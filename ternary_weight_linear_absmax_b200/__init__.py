@@ -22,7 +22,7 @@ from ._lib import BL_BF16, BL_F32, BL_FLAG_PDL, BitLinearError, check, load
 
 __all__ = [
     "bl_quant_weights", "bl_quant_acts", "bl_zero_gemm", "bl_linear_q", "bl_linear",
-    "bl_ffn_relu2", "bl_check_device_error", "bl_selftest_wait_timeout",
+    "bl_linear_noalloc", "bl_ffn_relu2", "bl_check_device_error", "bl_selftest_wait_timeout",
     "bl_gemv_max_tokens", "workspace_bytes", "BitLinearError", "load", "BL_FLAG_PDL",
 ]
 
@@ -156,6 +156,26 @@ def bl_linear(A, W_packed, gamma, eps: float = 1e-5, *, relu2=False, out_dtype=t
                          N, float(eps), int(bool(relu2)), out.data_ptr(), _dt(out, "out"),
                          _ptr(workspace), _nbytes(workspace), BL_FLAG_PDL if pdl else 0,
                          _stream(stream)), "bl_linear")
+    return out
+
+
+def bl_linear_noalloc(A, W_packed, gamma, eps: float = 1e-5, *, relu2=False,
+                      out_dtype=torch.bfloat16, out=None, stream=None):
+    """BitLinear forward that allocates no device memory inside the library
+    (for callers without an allocator): the scratch comes from a fixed 4 MiB
+    array in the library; larger problems raise BL_ERR_WORKSPACE. Only the
+    output (when ``out`` is None) is allocated here, by torch."""
+    _cuda(A, "A")
+    _cuda(W_packed, "W_packed")
+    _cuda(gamma, "gamma")
+    M, K = A.shape
+    N = W_packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    check(load().bl_linear_noalloc(A.data_ptr(), _dt(A, "A"), M, K, W_packed.data_ptr(),
+                                   gamma.data_ptr(), N, float(eps), int(bool(relu2)),
+                                   out.data_ptr(), _dt(out, "out"), _stream(stream)),
+          "bl_linear_noalloc")
     return out
 
 

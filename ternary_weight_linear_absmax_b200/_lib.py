@@ -40,6 +40,8 @@ SIGNATURES = {
                          _sz, _vp]),
     "bl_linear_ex": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _i64, _f32, _int, _vp, _int, _vp,
                             _sz, _uint, _vp]),
+    "bl_linear_noalloc": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _i64, _f32, _int, _vp, _int,
+                                 _vp]),
     "bl_ffn_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_ffn_relu2": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _f32, _vp, _int,
                             _vp, _sz, _vp]),

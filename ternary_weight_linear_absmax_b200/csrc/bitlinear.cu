@@ -686,6 +686,86 @@ bl_status bl_check_device_error(bl_stream_t stream) {
 
 }  // extern "C"
 
+// ==========================================================================
+// bl_linear_noalloc: bl_linear for callers that cannot allocate device
+// memory. Its scratch (the quantised tokens, their scales and row sums) lives
+// in the fixed array below instead of a caller-provided workspace.
+// ==========================================================================
+namespace {
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;  // 4 MiB per device
+}  // namespace
+
+// Held by every GPU that loads this library, until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+void* g_noalloc_ptr[bl::kMaxDevices] = {};
+
+// Device address of the scratch array for the current device. In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+bl_status noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(bl::g_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+      return BL_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return BL_OK;
+}
+}  // namespace
+
+extern "C" bl_status bl_linear_noalloc(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
+                                       const uint8_t* W_packed, const float* gamma, int64_t N,
+                                       float eps, int relu2, void* Y, bl_dtype y_dtype,
+                                       bl_stream_t stream) {
+  BL_TRY(check_dtype(a_dtype));
+  BL_TRY(check_dtype(y_dtype));
+  BL_TRY(check_k(K));
+  BL_TRY(check_rows(M));
+  BL_TRY(check_rows(N));
+  BL_TRY(check_eps(eps));
+  if (M == 0 || N == 0) return BL_OK;
+  BL_TRY(check_ptr(A));
+  BL_TRY(check_ptr(W_packed));
+  if (gamma == nullptr) return BL_ERR_INVALID_ARG;
+  BL_TRY(check_ptr(Y));
+  // Scratch this call needs; refuse what the fixed array cannot hold.
+  const size_t need = bl_linear_workspace_bytes(M, K, N);
+  if (need > kNoAllocScratchBytes) return BL_ERR_WORKSPACE;
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (need == 0) {  // a few tokens: the fused GEMV needs no scratch at all
+    GemvParams p = {};
+    p.A = A;
+    p.W = W_packed;
+    p.gamma = gamma;
+    p.Y = Y;
+    p.N = N;
+    p.K = K;
+    p.M = (int)M;
+    p.eps = eps;
+    p.relu2 = relu2 ? 1 : 0;
+    p.y_bf16 = y_dtype == BL_BF16;
+    return run_gemv(kSrcFloat, kOutDequant, a_dtype, p, false, dev, sms, st);
+  }
+  void* scratch = nullptr;
+  BL_TRY(noalloc_scratch(dev, &scratch));
+  // Every scratch byte read below is first written by this call's quantiser,
+  // so nothing has to start at zero.
+  const ActWs w = act_ws(M, K);
+  uint8_t* base = reinterpret_cast<uint8_t*>(scratch);
+  int8_t* Aq = reinterpret_cast<int8_t*>(base + w.aq);
+  float* gA = reinterpret_cast<float*>(base + w.gamma);
+  int32_t* rs = reinterpret_cast<int32_t*>(base + w.rowsum);
+  BL_TRY(run_quant_acts(A, a_dtype, M, K, eps, Aq, gA, rs, st));
+  return run_tc(Aq, W_packed, M, K, N, gamma, gA, rs, Y, kTcDequant, relu2 ? 1 : 0,
+                y_dtype == BL_BF16, dev, st);
+}
+
 namespace bl {
 namespace {
 __global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns) {
