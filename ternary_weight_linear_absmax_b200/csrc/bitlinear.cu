@@ -272,26 +272,26 @@ bl_status run_gemv(int src, int out, bl_dtype a_dtype, GemvParams p, bool pdl, i
 // --------------------------------------------------------------------------
 // Tensor-core launches.
 template <int BN, int OUT>
-bl_status launch_tc_t(const CUtensorMap& ta, const CUtensorMap& tw, const TcParams& p, int dev,
-                      cudaStream_t st) {
+bl_status launch_tc_t(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
+                      const TcParams& p, int dev, cudaStream_t st) {
   auto* k = tc_ternary_gemm_kernel<BN, OUT>;
   constexpr size_t smem = TcConfig<BN>::kSmemBytes;
   BL_TRY(ensure_smem(k, dev, smem));
   dim3 grid((unsigned)((p.N + 127) / 128), (unsigned)((p.M + BN - 1) / BN));
-  k<<<grid, kTcThreads, smem, st>>>(ta, tw, p);
+  k<<<grid, kTcThreads, smem, st>>>(ta, tw, ty, p);
   BL_CUDA(cudaGetLastError());
   return BL_OK;
 }
 
 template <int OUT>
-bl_status launch_tc_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tw, const TcParams& p,
-                       int dev, cudaStream_t st) {
+bl_status launch_tc_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tw,
+                       const CUtensorMap& ty, const TcParams& p, int dev, cudaStream_t st) {
   switch (bn) {
-    case 16: return launch_tc_t<16, OUT>(ta, tw, p, dev, st);
-    case 32: return launch_tc_t<32, OUT>(ta, tw, p, dev, st);
-    case 64: return launch_tc_t<64, OUT>(ta, tw, p, dev, st);
-    case 128: return launch_tc_t<128, OUT>(ta, tw, p, dev, st);
-    default: return launch_tc_t<256, OUT>(ta, tw, p, dev, st);
+    case 16: return launch_tc_t<16, OUT>(ta, tw, ty, p, dev, st);
+    case 32: return launch_tc_t<32, OUT>(ta, tw, ty, p, dev, st);
+    case 64: return launch_tc_t<64, OUT>(ta, tw, ty, p, dev, st);
+    case 128: return launch_tc_t<128, OUT>(ta, tw, ty, p, dev, st);
+    default: return launch_tc_t<256, OUT>(ta, tw, ty, p, dev, st);
   }
 }
 
@@ -314,7 +314,28 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
                      CU_TENSOR_MAP_SWIZZLE_128B));
   BL_TRY(make_map_u8(&tw, Wp, (uint64_t)N, (uint64_t)(K / 4), kTcBK / 4, 128,
                      CU_TENSOR_MAP_SWIZZLE_NONE));
+  // Output tensor map for the staged tensor-store epilogue (rows of N
+  // elements must be a multiple of 16 bytes).
+  const int esz = (out == kTcRawI32 || !y_bf16) ? 4 : 2;
+  CUtensorMap ty;
+  std::memset(&ty, 0, sizeof(ty));
+  int tma_store = 0;
+  if (((uint64_t)N * esz) % 16 == 0) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return BL_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)N * esz};
+    cuuint32_t box[2] = {128, (cuuint32_t)bn};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&ty, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32,
+                     2, Y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return BL_ERR_CUDA;
+    tma_store = 1;
+  }
   TcParams p;
+  p.tma_store = tma_store;
   p.gamma = gamma;
   p.gammaA = gammaA;
   p.rowsum = rowsum;
@@ -324,8 +345,8 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
   p.K = K;
   p.relu2 = relu2;
   p.y_bf16 = y_bf16;
-  return out == kTcDequant ? launch_tc_bn<kTcDequant>(bn, ta, tw, p, dev, st)
-                           : launch_tc_bn<kTcRawI32>(bn, ta, tw, p, dev, st);
+  return out == kTcDequant ? launch_tc_bn<kTcDequant>(bn, ta, tw, ty, p, dev, st)
+                           : launch_tc_bn<kTcRawI32>(bn, ta, tw, ty, p, dev, st);
 }
 
 bl_status run_quant_acts(const void* A, bl_dtype dt, int64_t M, int64_t K, float eps, int8_t* Aq,

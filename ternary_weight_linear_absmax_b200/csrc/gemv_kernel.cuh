@@ -16,19 +16,19 @@
 //  * The CTA then waits for the previous grid (griddepcontrol.wait) and runs
 //    the token prologue in one pass over global memory: AbsMax quantisation
 //    of the tokens, or the FFN ReLU² requantisation, or a copy of int8 tokens.
-//  * Thread t owns row t mod R and the chunk group t / R (every CG-th
-//    64-weight chunk of that row), which spreads R·K/64 chunk tasks evenly
-//    over the 512 threads. The swizzle places 16-byte chunk j of row r at
-//    position j ^ (r mod 8) of its 128-byte line, so consecutive lanes
-//    (consecutive rows, same chunk) load without bank conflicts; token words
-//    are broadcast loads.
+//  * Each thread owns two rows (r and r + ⌈R/2⌉) and a chunk group (every
+//    CG-th 64-weight chunk of K), so the R·K/64 chunk tasks spread evenly over
+//    the 512 threads and each token load serves two rows. The swizzle places
+//    16-byte chunk j of row r at position j ^ (r mod 8) of its 128-byte line,
+//    so consecutive lanes (consecutive rows, same chunk) load without bank
+//    conflicts; token words are broadcast loads.
 //  * Contraction with codes c = w+1 ∈ {0,1,2}: a packed word x holds, in byte
 //    i, the codes of weights 4j+i at bits 2j. For each j, x & (3·0x01010101
 //    << 2j) is a vector of four unsigned bytes c·4^j, so one LOP3 and one
 //    dp4a (unsigned × signed) per 4 weights accumulate 4^j·Σ c·a into acc[j];
 //    Σ c·a = acc[0] + acc[1]/4 + acc[2]/16 + acc[3]/64 exactly. Σ w·a is then
 //    Σ c·a − Σ a, with Σ a (the token's row sum) taken once.
-//  * Per-warp partial sums are combined in shared memory; the epilogue
+//  * Partial sums are combined in shared memory; the epilogue
 //    applies (γ_A·γ)/127 (and ReLU²) or writes the raw INT32 result.
 #pragma once
 
@@ -88,7 +88,7 @@ __host__ __device__ inline size_t gemv_smem_bytes(int64_t K, int rows, int M) {
   size_t s = kGemvHeader;
   s += (size_t)gemv_boxes(K) * gemv_rows_pad(rows) * 128;  // weights
   s += (size_t)M * K;                                      // int8 tokens
-  s += (size_t)kGemvThreads * M * sizeof(int);             // per-thread partial sums
+  s += (size_t)2 * kGemvThreads * M * sizeof(int);         // partial sums (2 rows/thread)
   return s + 1024;                                         // base alignment slack
 }
 
@@ -99,35 +99,16 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
   return d;
 }
 
-// Block-wide max of MT values per thread: warp shuffles, one barrier, then
-// every thread reads the per-warp maxima (no second barrier).
-template <int MT>
-__device__ __forceinline__ void block_max_all(float (&v)[MT], float (*red)[MT]) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-#pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    float t = warp_max(v[m]);
-    if (lane == 0) red[warp][m] = t;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    float t = 0.0f;
-#pragma unroll
-    for (int w = 0; w < kGemvWarps; ++w) t = fmaxf(t, red[w][m]);
-    v[m] = t;
-  }
-}
-
 template <int MT, typename TA, int SRC, int OUT>
 __global__ void __launch_bounds__(kGemvThreads, 2)
 gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p) {
-  constexpr int kGemvRegVecs = gemv_reg_vecs<MT>();
+  constexpr int RV = gemv_reg_vecs<MT>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  __shared__ float s_redf[kGemvWarps][MT];
-  __shared__ int s_redi[kGemvWarps][MT];
+  __shared__ unsigned s_max[MT];  // per-token max as float bits (all values are ≥ 0)
+  __shared__ int s_sum[MT];       // per-token Σ A_q
+  __shared__ float s_sc[MT];      // per-token dequant scale (γ_A·γ)/127
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int64_t K = p.K;
@@ -136,7 +117,6 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
   const int M = p.M;
 
   uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem);
-  float* s_sc = reinterpret_cast<float*>(smem + 16);  // [MT] dequant scale (γ_A·γ)/127
   uint8_t* s_w = smem + kGemvHeader;
   const int nbox = gemv_boxes(K);
   const int box_bytes = p.rows_pad * 128;
@@ -148,6 +128,10 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
   if (tid == 0) {
     mbar_init(s_bar, 1);
     fence_barrier_init();
+  }
+  if (tid < MT) {
+    s_max[tid] = 0u;
+    s_sum[tid] = 0;
   }
   __syncthreads();
   if (tid == 0) {
@@ -172,13 +156,9 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
   if (warp == 0) pdl_wait_prior_grid();
   __syncthreads();
 
-  // 3. Token prologue → int8 tokens in shared memory, Σ A_q and γ per token.
-  float tok_scale[MT];  // γ_A (float or int8 tokens) or γ_r (FFN requant)
-  int tok_sum[MT];
-#pragma unroll
-  for (int m = 0; m < MT; ++m) tok_sum[m] = 0;
+  // 3. Token prologue → int8 tokens in shared memory, Σ A_q and the scales.
+  //    Warp reductions use redux.sync; warps combine through shared atomics.
   if constexpr (SRC == kSrcFloat || SRC == kSrcFfnRequant) {
-    // Values per 16-byte vector and the value each element is quantised from.
     constexpr int VEC = SRC == kSrcFloat ? 16 / (int)sizeof(TA) : 4;
     const int64_t nvec = K / VEC;
     float scu[MT];
@@ -190,6 +170,7 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
       for (int m = 0; m < MT; ++m)
         if (m < M) scu[m] = __fdiv_rn(__fmul_rn(p.a_scale[m], gup), 127.0f);
     }
+    // The value each element is quantised from.
     auto value = [&](const uint4& u, int i, int m) -> float {
       if constexpr (SRC == kSrcFloat) {
         return to_f32<TA>(reinterpret_cast<const TA*>(&u)[i]);
@@ -200,44 +181,48 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
         return __fmul_rn(h, h);
       }
     };
-    uint4 reg[MT][kGemvRegVecs];
-    float mx[MT];
+    auto row_ptr = [&](int m) {
+      return reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.A) +
+                                            (size_t)m * (size_t)nvec * 16);
+    };
+    uint4 reg[MT][RV];
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
-      mx[m] = 0.0f;
+      float mx = 0.0f;
       if (m < M) {
-        const uint4* src = reinterpret_cast<const uint4*>(
-            reinterpret_cast<const uint8_t*>(p.A) + (size_t)m * (size_t)nvec * 16);
+        const uint4* src = row_ptr(m);
 #pragma unroll
-        for (int r = 0; r < kGemvRegVecs; ++r) {
+        for (int r = 0; r < RV; ++r) {
           const int64_t v = tid + (int64_t)r * kGemvThreads;
           if (v < nvec) {
             reg[m][r] = __ldg(src + v);
 #pragma unroll
-            for (int i = 0; i < VEC; ++i) mx[m] = fmaxf(mx[m], fabsf(value(reg[m][r], i, m)));
+            for (int i = 0; i < VEC; ++i) mx = fmaxf(mx, fabsf(value(reg[m][r], i, m)));
           }
         }
-        for (int64_t v = tid + (int64_t)kGemvRegVecs * kGemvThreads; v < nvec; v += kGemvThreads) {
+        for (int64_t v = tid + (int64_t)RV * kGemvThreads; v < nvec; v += kGemvThreads) {
           const uint4 u = __ldg(src + v);
 #pragma unroll
-          for (int i = 0; i < VEC; ++i) mx[m] = fmaxf(mx[m], fabsf(value(u, i, m)));
+          for (int i = 0; i < VEC; ++i) mx = fmaxf(mx, fabsf(value(u, i, m)));
         }
       }
+      const unsigned wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
+      if (lane == 0 && m < M) atomicMax(&s_max[m], wmax);
     }
-    block_max_all<MT>(mx, s_redf);
+    __syncthreads();
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
-      tok_scale[m] = mx[m];
+      int tsum = 0;
       if (m < M) {
-        const float s = __fdiv_rn(127.0f, __fadd_rn(mx[m], p.eps));
-        const uint4* src = reinterpret_cast<const uint4*>(
-            reinterpret_cast<const uint8_t*>(p.A) + (size_t)m * (size_t)nvec * 16);
+        const float g = __uint_as_float(s_max[m]);  // γ_A (or γ_r)
+        const float s = __fdiv_rn(127.0f, __fadd_rn(g, p.eps));
+        const uint4* src = row_ptr(m);
         auto emit = [&](const uint4& u, int64_t v) {
           int8_t q[VEC];
 #pragma unroll
           for (int i = 0; i < VEC; ++i) {
             q[i] = quant_i8(value(u, i, m), s);
-            tok_sum[m] += q[i];
+            tsum += q[i];
           }
           if constexpr (VEC == 8)
             *reinterpret_cast<uint2*>(s_a + m * K + v * VEC) = *reinterpret_cast<uint2*>(q);
@@ -245,47 +230,43 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
             *reinterpret_cast<uint32_t*>(s_a + m * K + v * VEC) = *reinterpret_cast<uint32_t*>(q);
         };
 #pragma unroll
-        for (int r = 0; r < kGemvRegVecs; ++r) {
+        for (int r = 0; r < RV; ++r) {
           const int64_t v = tid + (int64_t)r * kGemvThreads;
           if (v < nvec) emit(reg[m][r], v);
         }
-        for (int64_t v = tid + (int64_t)kGemvRegVecs * kGemvThreads; v < nvec; v += kGemvThreads)
+        for (int64_t v = tid + (int64_t)RV * kGemvThreads; v < nvec; v += kGemvThreads)
           emit(__ldg(src + v), v);
+        if (tid == 0) {
+          s_sc[m] = __fdiv_rn(__fmul_rn(g, gamma_w), 127.0f);  // (γ_A·γ)/127
+          if (p.gamma_out != nullptr && blockIdx.x == 0) p.gamma_out[m] = g;
+        }
       }
+      const int wsum = __reduce_add_sync(0xffffffffu, tsum);
+      if (lane == 0 && m < M) atomicAdd(&s_sum[m], wsum);
     }
   } else {  // kSrcInt8
     const int8_t* A = reinterpret_cast<const int8_t*>(p.A);
     const int64_t nvec = K / 16;
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
-      tok_scale[m] = (m < M && p.a_scale != nullptr) ? p.a_scale[m] : 0.0f;
+      int tsum = 0;
       if (m < M) {
         for (int64_t v = tid; v < nvec; v += kGemvThreads) {
-          uint4 u = __ldg(reinterpret_cast<const uint4*>(A + m * K) + v);
+          const uint4 u = __ldg(reinterpret_cast<const uint4*>(A + m * K) + v);
           *reinterpret_cast<uint4*>(s_a + m * K + v * 16) = u;
-          tok_sum[m] = dp4a(u.x, 0x01010101u, tok_sum[m]);
-          tok_sum[m] = dp4a(u.y, 0x01010101u, tok_sum[m]);
-          tok_sum[m] = dp4a(u.z, 0x01010101u, tok_sum[m]);
-          tok_sum[m] = dp4a(u.w, 0x01010101u, tok_sum[m]);
+          tsum = dp4a(u.x, 0x01010101u, tsum);
+          tsum = dp4a(u.y, 0x01010101u, tsum);
+          tsum = dp4a(u.z, 0x01010101u, tsum);
+          tsum = dp4a(u.w, 0x01010101u, tsum);
+        }
+        if (tid == 0) {
+          const float g = p.a_scale != nullptr ? p.a_scale[m] : 0.0f;
+          s_sc[m] = __fdiv_rn(__fmul_rn(g, gamma_w), 127.0f);
         }
       }
+      const int wsum = __reduce_add_sync(0xffffffffu, tsum);
+      if (lane == 0 && m < M) atomicAdd(&s_sum[m], wsum);
     }
-  }
-  // Per-warp token sums; combined in the epilogue after the next barrier.
-#pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    const int t = warp_sum_i(tok_sum[m]);
-    if (lane == 0) s_redi[warp][m] = t;
-  }
-  if (tid < MT) {
-    float ts = 0.0f;
-#pragma unroll
-    for (int m = 0; m < MT; ++m)
-      if (m == tid) ts = tok_scale[m];
-    if constexpr (SRC != kSrcInt8) {
-      if (tid < M && p.gamma_out != nullptr && blockIdx.x == 0) p.gamma_out[tid] = ts;
-    }
-    s_sc[tid] = __fdiv_rn(__fmul_rn(ts, gamma_w), 127.0f);  // (γ_A·γ)/127
   }
   __syncthreads();
 
@@ -296,30 +277,39 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
     return;
   }
 
-  // 5. Contraction. Thread t < R·CG owns row t mod R and chunk group
-  //    t / R, i.e. the 64-weight chunks cg, cg + CG, ... of that row.
-  //    Consecutive lanes take consecutive rows at the same chunk: the
-  //    swizzle keeps their weight loads conflict-free and the token loads
-  //    are broadcasts.
-  const int CG = gemv_chunk_groups(R, K);
+  // 5. Contraction. Thread t < RH·CG owns rows r = t mod RH and r + RH
+  //    (RH = ⌈R/2⌉) and the chunk group cg = t / RH: the 64-weight chunks
+  //    cg, cg + CG, ... of both rows. The two rows share every token load and
+  //    keep 8 independent accumulators per token. Consecutive lanes take
+  //    consecutive rows at the same chunk: the swizzle keeps their weight
+  //    loads conflict-free and the token loads are broadcasts.
+  const int RH = (R + 1) >> 1;
+  const int CG = gemv_chunk_groups(RH, K);
   const int nchunks = (int)(K / 64);
-  const bool active = tid < R * CG;
-  const int row = active ? tid % R : 0;
-  const int cg = active ? tid / R : 0;
-  int acc[MT][4];
+  const bool active = tid < RH * CG;
+  const int ra = active ? tid % RH : 0;
+  const int cg = active ? tid / RH : 0;
+  const bool has_b = ra + RH < R;
+  const int rb = has_b ? ra + RH : ra;
+  int acc[2][MT][4];
 #pragma unroll
-  for (int m = 0; m < MT; ++m)
+  for (int h = 0; h < 2; ++h)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[m][j] = 0;
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[h][m][j] = 0;
   if (active) {
-    const uint8_t* wrow = s_w + (size_t)row * 128;
-    const int sw = row & 7;
-#pragma unroll 4
+    const uint8_t* wa = s_w + (size_t)ra * 128;
+    const uint8_t* wb = s_w + (size_t)rb * 128;
+    const int swa = ra & 7, swb = rb & 7;
+#pragma unroll 2
     for (int c = cg; c < nchunks; c += CG) {
       // chunk c: box c/8, 16-byte slot (c mod 8) XOR (row mod 8)
-      const uint4 wv = *reinterpret_cast<const uint4*>(wrow + (size_t)(c >> 3) * box_bytes +
-                                                       (((c & 7) ^ sw) << 4));
-      const uint32_t x[4] = {wv.x, wv.y, wv.z, wv.w};
+      const size_t box = (size_t)(c >> 3) * box_bytes;
+      const uint4 va = *reinterpret_cast<const uint4*>(wa + box + (((c & 7) ^ swa) << 4));
+      const uint4 vb = *reinterpret_cast<const uint4*>(wb + box + (((c & 7) ^ swb) << 4));
+      const uint32_t xa[4] = {va.x, va.y, va.z, va.w};
+      const uint32_t xb[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
         if (m < M) {
@@ -327,10 +317,14 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const uint4 a = ap[q];  // token words 16c+4q .. 16c+4q+3
-            acc[m][0] = dp4a_us(x[q] & 0x03030303u, a.x, acc[m][0]);
-            acc[m][1] = dp4a_us(x[q] & 0x0C0C0C0Cu, a.y, acc[m][1]);
-            acc[m][2] = dp4a_us(x[q] & 0x30303030u, a.z, acc[m][2]);
-            acc[m][3] = dp4a_us(x[q] & 0xC0C0C0C0u, a.w, acc[m][3]);
+            acc[0][m][0] = dp4a_us(xa[q] & 0x03030303u, a.x, acc[0][m][0]);
+            acc[1][m][0] = dp4a_us(xb[q] & 0x03030303u, a.x, acc[1][m][0]);
+            acc[0][m][1] = dp4a_us(xa[q] & 0x0C0C0C0Cu, a.y, acc[0][m][1]);
+            acc[1][m][1] = dp4a_us(xb[q] & 0x0C0C0C0Cu, a.y, acc[1][m][1]);
+            acc[0][m][2] = dp4a_us(xa[q] & 0x30303030u, a.z, acc[0][m][2]);
+            acc[1][m][2] = dp4a_us(xb[q] & 0x30303030u, a.z, acc[1][m][2]);
+            acc[0][m][3] = dp4a_us(xa[q] & 0xC0C0C0C0u, a.w, acc[0][m][3]);
+            acc[1][m][3] = dp4a_us(xb[q] & 0xC0C0C0C0u, a.w, acc[1][m][3]);
           }
         }
       }
@@ -338,22 +332,23 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
     // Σ c·a over this thread's chunks; acc[j] is a multiple of 4^j, so the
     // arithmetic shifts are exact.
 #pragma unroll
-    for (int m = 0; m < MT; ++m)
-      if (m < M)
-        s_part[(m * CG + cg) * R + row] =
-            acc[m][0] + (acc[m][1] >> 2) + (acc[m][2] >> 4) + (acc[m][3] >> 6);
+    for (int m = 0; m < MT; ++m) {
+      if (m < M) {
+        int* part = s_part + (m * CG + cg) * R;
+        part[ra] = acc[0][m][0] + (acc[0][m][1] >> 2) + (acc[0][m][2] >> 4) + (acc[0][m][3] >> 6);
+        if (has_b)
+          part[rb] = acc[1][m][0] + (acc[1][m][1] >> 2) + (acc[1][m][2] >> 4) + (acc[1][m][3] >> 6);
+      }
+    }
   }
   __syncthreads();
 
-  // 6. Epilogue: combine the group's warps, undo the code offset, scale.
+  // 6. Epilogue: combine the chunk groups, undo the code offset, scale.
   for (int e = tid; e < M * R; e += kGemvThreads) {
     const int m = e / R, r = e - m * R;
     int d = 0;
     for (int k = 0; k < CG; ++k) d += s_part[(m * CG + k) * R + r];
-    int ssum = 0;
-#pragma unroll
-    for (int w = 0; w < kGemvWarps; ++w) ssum += s_redi[w][m];
-    const int v = d - ssum;
+    const int v = d - s_sum[m];
     const int64_t o = (int64_t)m * p.N + r0 + r;
     if constexpr (OUT == kOutRawI32) {
       reinterpret_cast<int32_t*>(p.Y)[o] = v;

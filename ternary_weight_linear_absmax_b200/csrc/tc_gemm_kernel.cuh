@@ -44,6 +44,8 @@ struct TcParams {
   int64_t M, N, K;
   int relu2;
   int y_bf16;
+  int tma_store;  // 1: the epilogue stages the tile in shared memory and writes it with one
+                  //    tensor store through tm_y (needs N·element bytes % 16 == 0)
 };
 
 template <int BN>
@@ -52,13 +54,18 @@ struct TcConfig {
   static constexpr int kWStage = 128 * 32;       // bytes of packed weights per stage
   static constexpr int kSStages = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
   static constexpr int kTStages = 4;             // TMEM A stages (32 columns each)
-  static constexpr int kDCols = BN < 32 ? 32 : BN;
-  static constexpr int kACol = kDCols;
-  static constexpr int kColsNeeded = kDCols + kTStages * 32;
+  // Independent accumulators: consecutive MMAs into one accumulator are
+  // serialised by its read-modify-write, which dominates for small N. The
+  // four MMAs of a stage rotate over kAcc accumulators, summed in the
+  // epilogue (exact integer addition).
+  static constexpr int kAcc = BN <= 64 ? 4 : (BN <= 128 ? 2 : 1);
+  static constexpr int kDCols = BN < 32 ? 32 : BN;  // columns per accumulator
+  static constexpr int kACol = kAcc * kDCols;
+  static constexpr int kColsNeeded = kACol + kTStages * 32;
   static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
                                    : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
   static constexpr int kRingBytes = kSStages * (kBStage + kWStage);
-  static constexpr int kBarBytes = (2 * kSStages + 2 * kTStages + 1) * 8;
+  static constexpr int kBarBytes = (2 * kSStages + 2 * kTStages + 2) * 8;
   static constexpr int kParamBytes = BN * 8;
   // 1 KiB slack for aligning the dynamic buffer to 1024 bytes. At least
   // 116 KiB are requested so that only one CTA is resident per SM: every CTA
@@ -84,10 +91,115 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
   }
 }
 
+// Epilogue body for one chunk of CW accumulator columns (tokens) of this
+// thread's row: undo the code offset, scale (and ReLU²), convert, and write
+// either into the staged [BN x 128] tile or straight to global memory. The
+// flags are template parameters so the unrolled body has no branches and the
+// CW columns form independent instruction chains.
+template <int CW, int OUT, bool RELU, bool BF16, bool STAGE>
+__device__ __forceinline__ void tc_epilogue_chunk(const uint32_t (&d)[CW], int c0, int row,
+                                                  const float* s_sc, const int* s_rs,
+                                                  uint8_t* stage, const TcParams& p, int64_t m0,
+                                                  int64_t n) {
+  // Read all per-token scalars first: the stores below go to shared memory
+  // too, and without this split they would order every following load.
+  float sc[CW];
+  int rs[CW];
+#pragma unroll
+  for (int j = 0; j < CW; ++j) {
+    sc[j] = s_sc[c0 + j];
+    rs[j] = s_rs[c0 + j];
+  }
+  uint32_t bits[CW];
+#pragma unroll
+  for (int j = 0; j < CW; ++j) {
+    const int v = (int)d[j] - rs[j];
+    if constexpr (OUT == kTcRawI32) {
+      bits[j] = (uint32_t)v;
+    } else {
+      float y = __fmul_rn((float)v, sc[j]);
+      if constexpr (RELU) {
+        y = fmaxf(y, 0.0f);
+        y = __fmul_rn(y, y);
+      }
+      if constexpr (BF16)
+        bits[j] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y));
+      else
+        bits[j] = __float_as_uint(y);
+    }
+  }
+  constexpr bool kHalf = (OUT != kTcRawI32) && BF16;
+#pragma unroll
+  for (int j = 0; j < CW; ++j) {
+    const int jj = c0 + j;
+    if constexpr (STAGE) {
+      if constexpr (kHalf)
+        reinterpret_cast<uint16_t*>(stage)[jj * 128 + row] = (uint16_t)bits[j];
+      else
+        reinterpret_cast<uint32_t*>(stage)[jj * 128 + row] = bits[j];
+    } else {
+      const int64_t m = m0 + jj;
+      if (m < p.M && n < p.N) {
+        const int64_t o = m * p.N + n;
+        if constexpr (kHalf)
+          reinterpret_cast<uint16_t*>(p.Y)[o] = (uint16_t)bits[j];
+        else
+          reinterpret_cast<uint32_t*>(p.Y)[o] = bits[j];
+      }
+    }
+  }
+}
+
+// Whole-tile epilogue for one thread's TMEM lane: loads CW columns at a time
+// (summing the kAcc accumulators), with the next chunk's load issued before
+// the current chunk is processed.
+template <int BN, int OUT, bool RELU, bool BF16, bool STAGE>
+__device__ __forceinline__ void tc_epilogue(uint32_t t_lane, int row, const float* s_sc,
+                                            const int* s_rs, uint8_t* stage, const TcParams& p,
+                                            int64_t m0, int64_t n) {
+  using C = TcConfig<BN>;
+  constexpr int CW = BN >= 32 ? 32 : 16;
+  auto load = [&](int c0, uint32_t (&d)[CW]) {
+    if constexpr (CW == 32)
+      tmem_ld_32x32b_x32(t_lane + c0, d);
+    else
+      tmem_ld_32x32b_x16(t_lane + c0, d);
+    if constexpr (C::kAcc > 1) {
+      tmem_wait_ld();
+#pragma unroll
+      for (int a = 1; a < C::kAcc; ++a) {
+        uint32_t e[CW];
+        if constexpr (CW == 32)
+          tmem_ld_32x32b_x32(t_lane + a * C::kDCols + c0, e);
+        else
+          tmem_ld_32x32b_x16(t_lane + a * C::kDCols + c0, e);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < CW; ++j) d[j] = (uint32_t)((int)d[j] + (int)e[j]);
+      }
+    }
+  };
+  uint32_t cur[CW], nxt[CW];
+  load(0, cur);
+  tmem_wait_ld();
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += CW) {
+    const bool more = c0 + CW < BN;
+    if (more) load(c0 + CW, nxt);  // in flight while this chunk is processed
+    tc_epilogue_chunk<CW, OUT, RELU, BF16, STAGE>(cur, c0, row, s_sc, s_rs, stage, p, m0, n);
+    if (more) {
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < CW; ++j) cur[j] = nxt[j];
+    }
+  }
+}
+
 template <int BN, int OUT>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
-                       const __grid_constant__ CUtensorMap tm_w, const TcParams p) {
+                       const __grid_constant__ CUtensorMap tm_w,
+                       const __grid_constant__ CUtensorMap tm_y, const TcParams p) {
   using C = TcConfig<BN>;
   constexpr int SS = C::kSStages, TS = C::kTStages;
   extern __shared__ uint8_t smem_raw[];
@@ -101,6 +213,7 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
   uint64_t* afull = bars + 2 * SS;                  // [TS] A operand in TMEM ready
   uint64_t* aempty = bars + 2 * SS + TS;            // [TS] MMA done with A stage
   uint64_t* done = bars + 2 * SS + 2 * TS;          // accumulator complete
+  uint64_t* staged = bars + 2 * SS + 2 * TS + 1;    // output tile staged (128 arrivals)
   float* s_sc = reinterpret_cast<float*>(smem + C::kRingBytes + C::kBarBytes);
   int* s_rs = reinterpret_cast<int*>(s_sc + BN);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_rs + BN);
@@ -133,6 +246,7 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
       mbar_init(&aempty[t], 1);
     }
     mbar_init(done, 1);
+    mbar_init(staged, 128);
     *s_abort = 0;
     fence_barrier_init();
     prefetch_tensormap(&tm_act);
@@ -148,43 +262,45 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
   const uint32_t tmem = *s_tmem;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      int kb = 0;
-      for (; kb < KB; ++kb) {
-        const int s = kb % SS;
-        if (kb >= SS && !wait_or_abort(&empty[s], ((kb / SS) + 1) & 1, s_abort)) break;
-        mbar_arrive_expect_tx(&full[s], C::kBStage + C::kWStage);
-        tma_load_2d(s_b + s * C::kBStage, &tm_act, kb * kTcBK, (int32_t)m0, &full[s]);
-        tma_load_2d(s_w + s * C::kWStage, &tm_w, kb * (kTcBK / 4), (int32_t)n0, &full[s]);
-      }
-      if (*s_abort) {
-        // Drain copies that may still be in flight (bounded) before exit.
-        for (int d = max(0, kb - SS); d < kb; ++d)
-          mbar_wait_for(&full[d % SS], (d / SS) & 1, 100000000ull);
-      }
+    // ---------------- TMA producer (whole warp, one elected lane issues) ---
+    int kb = 0;
+    for (; kb < KB; ++kb) {
+      const int s = kb % SS;
+      bool ok = kb < SS || wait_or_abort(&empty[s], ((kb / SS) + 1) & 1, s_abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tma_load_2x2d_warp(&full[s], C::kBStage + C::kWStage, s_b + s * C::kBStage, &tm_act,
+                         kb * kTcBK, (int32_t)m0, s_w + s * C::kWStage, &tm_w, kb * (kTcBK / 4),
+                         (int32_t)n0);
+    }
+    if (*s_abort && lane == 0) {
+      // Drain copies that may still be in flight (bounded) before exit.
+      for (int d = max(0, kb - SS); d < kb; ++d)
+        mbar_wait_for(&full[d % SS], (d / SS) & 1, 100000000ull);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(128, BN);
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % SS, t = kb % TS;
-        if (!wait_or_abort(&full[s], (kb / SS) & 1, s_abort)) break;
-        if (!wait_or_abort(&afull[t], (kb / TS) & 1, s_abort)) break;
-        tc_fence_after();
-        const uint32_t b_addr = smem_u32(s_b + s * C::kBStage);
+    // ---------------- MMA issuer (whole warp, one elected lane issues) -----
+    constexpr uint32_t idesc = idesc_i8(128, BN);
+    const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+    const uint32_t b_base = __shfl_sync(0xffffffffu, smem_u32(s_b), 0);
+    for (int kb = 0; kb < KB; ++kb) {
+      const int s = kb % SS, t = kb % TS;
+      bool ok = wait_or_abort(&full[s], (kb / SS) & 1, s_abort);
+      if (ok) ok = wait_or_abort(&afull[t], (kb / TS) & 1, s_abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const uint64_t bdesc = smem_desc_sw128(b_base + s * C::kBStage);
+      const uint32_t a_col = tm + C::kACol + t * 32;
 #pragma unroll
-        for (int kk = 0; kk < kTcBK / 32; ++kk) {
-          const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 32);
-          mma_i8_ts(tmem, tmem + C::kACol + t * 32 + kk * 8, bdesc, idesc,
-                    (kb > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&empty[s]);
-        mma_commit(&aempty[t]);
+      for (int kk = 0; kk < kTcBK / 32; ++kk) {
+        const int acc = kk % C::kAcc;
+        // +2 in the descriptor's address field = +32 bytes along K
+        mma_i8_ts_warp(tm + acc * C::kDCols, a_col + kk * 8, bdesc + (uint64_t)(kk * 2), idesc,
+                       (kb > 0 || kk >= C::kAcc) ? 1u : 0u);
       }
-      mma_commit(done);  // also on abort: tracks every MMA issued
+      mma_commit_warp(&empty[s]);
+      mma_commit_warp(&aempty[t]);
     }
+    mma_commit_warp(done);  // also on abort: tracks every MMA issued
   } else {
     // ---------------- expansion (warps 2..5) ----------------
     const int q = warp & 3;         // TMEM lane quarter this warp may access
@@ -214,33 +330,38 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
     if (ok) {
       tc_fence_after();
       const int64_t n = n0 + row;
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        uint32_t d[16];
-        tmem_ld_32x32b_x16(tmem + lane_addr + c0, d);
-        tmem_wait_ld();
-        if (n < p.N) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int64_t m = m0 + c0 + j;
-            if (m < p.M) {
-              const int v = (int)d[j] - s_rs[c0 + j];
-              const int64_t o = m * p.N + n;
-              if constexpr (OUT == kTcRawI32) {
-                reinterpret_cast<int32_t*>(p.Y)[o] = v;
-              } else {
-                float y = __fmul_rn((float)v, s_sc[c0 + j]);
-                if (p.relu2) {
-                  y = fmaxf(y, 0.0f);
-                  y = __fmul_rn(y, y);
-                }
-                if (p.y_bf16)
-                  reinterpret_cast<__nv_bfloat16*>(p.Y)[o] = __float2bfloat16_rn(y);
-                else
-                  reinterpret_cast<float*>(p.Y)[o] = y;
-              }
-            }
-          }
+      // The staging tile reuses the ring: once `done` has been observed every
+      // load has landed and every MMA has finished reading it.
+      const uint32_t t_lane = tmem + lane_addr;
+      if constexpr (OUT == kTcRawI32) {
+        if (p.tma_store)
+          tc_epilogue<BN, OUT, false, false, true>(t_lane, row, s_sc, s_rs, smem, p, m0, n);
+        else
+          tc_epilogue<BN, OUT, false, false, false>(t_lane, row, s_sc, s_rs, smem, p, m0, n);
+      } else {
+        const int sel = (p.tma_store ? 4 : 0) | (p.y_bf16 ? 2 : 0) | (p.relu2 ? 1 : 0);
+        switch (sel) {
+          case 0: tc_epilogue<BN, OUT, false, false, false>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
+          case 1: tc_epilogue<BN, OUT, true, false, false>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
+          case 2: tc_epilogue<BN, OUT, false, true, false>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
+          case 3: tc_epilogue<BN, OUT, true, true, false>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
+          case 4: tc_epilogue<BN, OUT, false, false, true>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
+          case 5: tc_epilogue<BN, OUT, true, false, true>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
+          case 6: tc_epilogue<BN, OUT, false, true, true>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
+          default: tc_epilogue<BN, OUT, true, true, true>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
+        }
+      }
+      if (p.tma_store) fence_proxy_async_smem();  // staged writes -> visible to the tensor store
+    }
+    // Every epilogue thread arrives (also when it skipped the epilogue), so
+    // the storing thread's bounded wait can only time out on a failed CTA.
+    if (p.tma_store) {
+      mbar_arrive(staged);
+      if (warp == 2 && lane == 0 && ok) {
+        if (mbar_wait(staged, 0) && !*s_abort) {
+          tma_store_2d(&tm_y, (int32_t)n0, (int32_t)m0, smem);
+          bulk_commit_group();
+          bulk_wait_group_read0();  // shared source read before the CTA may exit
         }
       }
     }
