@@ -312,8 +312,8 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
   CUtensorMap ta, tw;
   BL_TRY(make_map_u8(&ta, Aq, (uint64_t)M, (uint64_t)K, kTcBK, (uint32_t)bn,
                      CU_TENSOR_MAP_SWIZZLE_128B));
-  BL_TRY(make_map_u8(&tw, Wp, (uint64_t)N, (uint64_t)(K / 4), kTcBK / 4, 128,
-                     CU_TENSOR_MAP_SWIZZLE_NONE));
+  BL_TRY(make_map_u8(&tw, Wp, (uint64_t)N, (uint64_t)(K / 4), 128, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
   // Output tensor map for the staged tensor-store epilogue (rows of N
   // elements must be a multiple of 16 bytes).
   const int esz = (out == kTcRawI32 || !y_bf16) ? 4 : 2;

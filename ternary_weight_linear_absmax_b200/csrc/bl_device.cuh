@@ -234,6 +234,33 @@ __device__ __forceinline__ void tma_load_2x2d_warp(uint64_t* bar, uint32_t tx, v
       : "memory");
 }
 
+// One elected lane of a converged warp arms `bar` for `tx` bytes and issues
+// one 2-D tensor load that completes on it.
+__device__ __forceinline__ void tma_load_1x2d_warp(uint64_t* bar, uint32_t tx, void* dst,
+                                                   const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t"
+      "@e cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%2], [%3, {%4, %5}], [%0];\n\t}" ::"r"(smem_u32(bar)),
+      "r"(tx), "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// One elected lane prefetches a 2-D tensor tile into L2 (no shared memory,
+// no barrier).
+__device__ __forceinline__ void tma_prefetch_2d_warp(const CUtensorMap* map, int32_t x,
+                                                     int32_t y) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];\n\t}" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y)
+      : "memory");
+}
+
 // 2-D tensor store shared -> global (bulk group), its commit and the wait
 // until the shared-memory source has been read. Stores start at
 // non-negative coordinates; elements outside the tensor are not written.

@@ -346,9 +346,18 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
   // 6. Epilogue: combine the chunk groups, undo the code offset, scale.
   for (int e = tid; e < M * R; e += kGemvThreads) {
     const int m = e / R, r = e - m * R;
-    int d = 0;
-    for (int k = 0; k < CG; ++k) d += s_part[(m * CG + k) * R + r];
-    const int v = d - s_sum[m];
+    // Four independent partial sums keep the shared loads in flight together.
+    const int* pp = s_part + m * CG * R + r;
+    int d0 = 0, d1 = 0, d2 = 0, d3 = 0;
+    int k = 0;
+    for (; k + 4 <= CG; k += 4) {
+      d0 += pp[(k + 0) * R];
+      d1 += pp[(k + 1) * R];
+      d2 += pp[(k + 2) * R];
+      d3 += pp[(k + 3) * R];
+    }
+    for (; k < CG; ++k) d0 += pp[k * R];
+    const int v = (d0 + d1) + (d2 + d3) - s_sum[m];
     const int64_t o = (int64_t)m * p.N + r0 + r;
     if constexpr (OUT == kOutRawI32) {
       reinterpret_cast<int32_t*>(p.Y)[o] = v;

@@ -50,10 +50,17 @@ struct TcParams {
 
 template <int BN>
 struct TcConfig {
-  static constexpr int kBStage = BN * kTcBK;     // bytes of token tile per stage
-  static constexpr int kWStage = 128 * 32;       // bytes of packed weights per stage
-  static constexpr int kSStages = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
-  static constexpr int kTStages = 4;             // TMEM A stages (32 columns each)
+  // Token ring: one 128-byte-wide K block (BN rows, 128-byte swizzle) per stage.
+  static constexpr int kBStage = BN * kTcBK;
+  // Deep enough that the producer can run ahead over every weight stage
+  // (4 K blocks per weight stage): small token tiles are cheap to stage.
+  static constexpr int kSStages = BN >= 256 ? 4 : (BN >= 128 ? 6 : (BN >= 64 ? 12 : (BN >= 32 ? 16 : 24)));
+  // Weight ring: 128 rows × 128 packed bytes (4 K blocks) per stage, 128-byte
+  // swizzle. Wide rows keep the number of TMA requests per byte low, which is
+  // what bounds the stream when few tokens share each weight byte.
+  static constexpr int kWStage = 128 * 128;
+  static constexpr int kWStages = BN >= 256 ? 2 : (BN >= 128 ? 3 : (BN >= 64 ? 4 : 6));
+  static constexpr int kTStages = 4;  // TMEM A stages (32 columns = one K block each)
   // Independent accumulators: consecutive MMAs into one accumulator are
   // serialised by its read-modify-write, which dominates for small N. The
   // four MMAs of a stage rotate over kAcc accumulators, summed in the
@@ -64,14 +71,16 @@ struct TcConfig {
   static constexpr int kColsNeeded = kACol + kTStages * 32;
   static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
                                    : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
-  static constexpr int kRingBytes = kSStages * (kBStage + kWStage);
-  static constexpr int kBarBytes = (2 * kSStages + 2 * kTStages + 2) * 8;
+  static constexpr int kRingBytes = kSStages * kBStage + kWStages * kWStage;
+  static constexpr int kBarBytes = (2 * kSStages + 2 * kWStages + 2 * kTStages + 2) * 8;
   static constexpr int kParamBytes = BN * 8;
   // 1 KiB slack for aligning the dynamic buffer to 1024 bytes. At least
   // 116 KiB are requested so that only one CTA is resident per SM: every CTA
   // then gets its TMEM columns without waiting on another CTA's allocation.
   static constexpr int kSmemUsed = 1024 + kRingBytes + kBarBytes + kParamBytes + 64;
   static constexpr int kSmemBytes = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
+  // The output staging tile reuses the ring.
+  static_assert(BN * 128 * 4 <= kRingBytes, "staging tile must fit in the ring");
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
@@ -201,19 +210,21 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
                        const __grid_constant__ CUtensorMap tm_w,
                        const __grid_constant__ CUtensorMap tm_y, const TcParams p) {
   using C = TcConfig<BN>;
-  constexpr int SS = C::kSStages, TS = C::kTStages;
+  constexpr int SS = C::kSStages, WS = C::kWStages, TS = C::kTStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* s_b = smem;                              // SS × BN×128 (1024-aligned stages)
-  uint8_t* s_w = smem + SS * C::kBStage;            // SS × 128×32
+  uint8_t* s_w = smem + SS * C::kBStage;            // WS × 128×128 (1024-aligned stages)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kRingBytes);
-  uint64_t* full = bars;                            // [SS] TMA landed
-  uint64_t* empty = bars + SS;                      // [SS] MMA done with stage
-  uint64_t* afull = bars + 2 * SS;                  // [TS] A operand in TMEM ready
-  uint64_t* aempty = bars + 2 * SS + TS;            // [TS] MMA done with A stage
-  uint64_t* done = bars + 2 * SS + 2 * TS;          // accumulator complete
-  uint64_t* staged = bars + 2 * SS + 2 * TS + 1;    // output tile staged (128 arrivals)
+  uint64_t* full = bars;                            // [SS] token tile landed
+  uint64_t* empty = bars + SS;                      // [SS] MMA done with token stage
+  uint64_t* wfull = bars + 2 * SS;                  // [WS] weight tile landed
+  uint64_t* wempty = bars + 2 * SS + WS;            // [WS] expansion done with weight stage
+  uint64_t* afull = bars + 2 * SS + 2 * WS;         // [TS] A operand in TMEM ready
+  uint64_t* aempty = afull + TS;                    // [TS] MMA done with A stage
+  uint64_t* done = aempty + TS;                     // accumulator complete
+  uint64_t* staged = done + 1;                      // output tile staged (128 arrivals)
   float* s_sc = reinterpret_cast<float*>(smem + C::kRingBytes + C::kBarBytes);
   int* s_rs = reinterpret_cast<int*>(s_sc + BN);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_rs + BN);
@@ -241,6 +252,10 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
+    for (int v = 0; v < WS; ++v) {
+      mbar_init(&wfull[v], 1);
+      mbar_init(&wempty[v], 128);
+    }
     for (int t = 0; t < TS; ++t) {
       mbar_init(&afull[t], 128);
       mbar_init(&aempty[t], 1);
@@ -263,19 +278,30 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
 
   if (warp == 0) {
     // ---------------- TMA producer (whole warp, one elected lane issues) ---
-    int kb = 0;
+    int kb = 0, wissued = 0;
     for (; kb < KB; ++kb) {
+      if ((kb & 3) == 0) {  // a new weight stage covers K blocks kb .. kb+3
+        const int ws = kb >> 2, v = ws % WS;
+        bool ok = ws < WS || wait_or_abort(&wempty[v], ((ws / WS) + 1) & 1, s_abort);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tma_load_1x2d_warp(&wfull[v], C::kWStage, s_w + v * C::kWStage, &tm_w, ws * 128,
+                           (int32_t)n0);
+        ++wissued;
+      }
       const int s = kb % SS;
       bool ok = kb < SS || wait_or_abort(&empty[s], ((kb / SS) + 1) & 1, s_abort);
       if (!__all_sync(0xffffffffu, ok)) break;
-      tma_load_2x2d_warp(&full[s], C::kBStage + C::kWStage, s_b + s * C::kBStage, &tm_act,
-                         kb * kTcBK, (int32_t)m0, s_w + s * C::kWStage, &tm_w, kb * (kTcBK / 4),
-                         (int32_t)n0);
+      tma_load_1x2d_warp(&full[s], C::kBStage, s_b + s * C::kBStage, &tm_act, kb * kTcBK,
+                         (int32_t)m0);
+      // Warm L2 with the token tile this stage will hold next time round.
+      if (kb + SS < KB) tma_prefetch_2d_warp(&tm_act, (kb + SS) * kTcBK, (int32_t)m0);
     }
     if (*s_abort && lane == 0) {
       // Drain copies that may still be in flight (bounded) before exit.
       for (int d = max(0, kb - SS); d < kb; ++d)
         mbar_wait_for(&full[d % SS], (d / SS) & 1, 100000000ull);
+      for (int d = max(0, wissued - WS); d < wissued; ++d)
+        mbar_wait_for(&wfull[d % WS], (d / WS) & 1, 100000000ull);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer (whole warp, one elected lane issues) -----
@@ -307,19 +333,23 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
     const int row = 32 * q + lane;  // weight row within the tile
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     for (int kb = 0; kb < KB; ++kb) {
-      const int s = kb % SS, t = kb % TS;
+      const int t = kb % TS, ws = kb >> 2, v = ws % WS, sub = kb & 3;
       // tcgen05.st is warp-collective: the whole warp continues or stops.
-      bool ok = wait_or_abort(&full[s], (kb / SS) & 1, s_abort);
+      bool ok = wait_or_abort(&wfull[v], (ws / WS) & 1, s_abort);
       if (ok && kb >= TS) ok = wait_or_abort(&aempty[t], ((kb / TS) + 1) & 1, s_abort);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const uint4* src = reinterpret_cast<const uint4*>(s_w + s * C::kWStage + row * 32);
-      const uint4 u0 = src[0], u1 = src[1];
+      // This K block is 16-byte chunks 2·sub and 2·sub+1 of the row's 128-byte
+      // line; the 128-byte swizzle stores chunk j at slot j ^ (row mod 8).
+      const uint8_t* line = s_w + v * C::kWStage + row * 128;
+      const uint4 u0 = *reinterpret_cast<const uint4*>(line + (((2 * sub) ^ (row & 7)) << 4));
+      const uint4 u1 = *reinterpret_cast<const uint4*>(line + (((2 * sub + 1) ^ (row & 7)) << 4));
+      if (sub == 3 || kb == KB - 1) mbar_arrive(&wempty[v]);  // done reading this stage
       const uint32_t x[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-      uint32_t v[32];
+      uint32_t vv[32];
 #pragma unroll
-      for (int g = 0; g < 8; ++g) expand_word(x[g], v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-      tmem_st_32x32b_x32(tmem + lane_addr + C::kACol + t * 32, v);
+      for (int g = 0; g < 8; ++g) expand_word(x[g], vv[4 * g], vv[4 * g + 1], vv[4 * g + 2], vv[4 * g + 3]);
+      tmem_st_32x32b_x32(tmem + lane_addr + C::kACol + t * 32, vv);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&afull[t]);
