@@ -673,7 +673,9 @@ bl_status bl_ffn_relu2(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, in
     dn.M = (int)M;
     dn.eps = eps;
     dn.y_bf16 = y_dtype == BL_BF16;
-    return run_gemv(kSrcFfnRequant, kOutDequant, BL_F32, dn, false, dev, sms, st);
+    // The kernel before this one is the up-projection above, which does not
+    // write W_down: the down-projection may stream its weights early (PDL).
+    return run_gemv(kSrcFfnRequant, kOutDequant, BL_F32, dn, true, dev, sms, st);
   }
   int8_t* Xq = reinterpret_cast<int8_t*>(base + w.x.aq);
   float* gX = reinterpret_cast<float*>(base + w.x.gamma);

@@ -303,6 +303,17 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
       : "memory");
 }
 
+// Store 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+
 // Load 32 consecutive 32-bit columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
@@ -385,11 +396,29 @@ __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
   return __bfloat162float(v);
 }
 
+// Clip(Round(a·s), -128, 127) with one fp32 product and round-half-to-even,
+// returned in the low byte of a word. Clipping before rounding gives the
+// same integer because the bounds are integers. Adding 1.5·2^23 to a value
+// in [-128, 127] lands in [2^23, 2^24), where the fp32 spacing is 1, so the
+// correctly rounded sum is 1.5·2^23 + Round(v) with ties to even (1.5·2^23 is
+// even); its bit pattern is 0x4B400000 + Round(v), whose low byte is the
+// two's-complement int8. This keeps the rounding off the conversion unit.
+__device__ __forceinline__ uint32_t quant_i8_bits(float a, float s) {
+  float v = __fmul_rn(a, s);
+  v = fminf(fmaxf(v, -128.0f), 127.0f);
+  return __float_as_uint(__fadd_rn(v, 12582912.0f));
+}
+
 __device__ __forceinline__ int8_t quant_i8(float a, float s) {
-  // Clip(Round(a·s), -128, 127): one fp32 product, round half to even.
-  float q = rintf(__fmul_rn(a, s));
-  q = fminf(fmaxf(q, -128.0f), 127.0f);
-  return (int8_t)(int)q;
+  return (int8_t)(quant_i8_bits(a, s) & 0xFFu);
+}
+
+// Packs the low bytes of four words into one word (byte i from word i).
+__device__ __forceinline__ uint32_t pack4_low_bytes(uint32_t b0, uint32_t b1, uint32_t b2,
+                                                    uint32_t b3) {
+  const uint32_t lo = __byte_perm(b0, b1, 0x0040);
+  const uint32_t hi = __byte_perm(b2, b3, 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
 }
 
 // Warp reductions

@@ -88,7 +88,7 @@ __host__ __device__ inline size_t gemv_smem_bytes(int64_t K, int rows, int M) {
   size_t s = kGemvHeader;
   s += (size_t)gemv_boxes(K) * gemv_rows_pad(rows) * 128;  // weights
   s += (size_t)M * K;                                      // int8 tokens
-  s += (size_t)2 * kGemvThreads * M * sizeof(int);         // partial sums (2 rows/thread)
+  s += (size_t)M * rows * sizeof(int);                     // per-row sums
   return s + 1024;                                         // base alignment slack
 }
 
@@ -133,6 +133,7 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
     s_max[tid] = 0u;
     s_sum[tid] = 0;
   }
+  for (int i = tid; i < M * p.rows_per_cta; i += kGemvThreads) s_part[i] = 0;
   __syncthreads();
   if (tid == 0) {
     mbar_arrive_expect_tx(s_bar, (uint32_t)nbox * (uint32_t)box_bytes);
@@ -150,9 +151,55 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
   // the dependency wait.
   const float gamma_w = p.gamma != nullptr ? __ldg(p.gamma) : 0.0f;
   pdl_launch_dependents();
-  // 2. Tokens and outputs are ordered after the previous kernel. One warp
-  //    waits for the prior grid; the others wait at the CTA barrier, so a CTA
-  //    launched early spends no issue slots while its predecessor runs.
+
+  // Contraction mapping (see step 5): thread t < RH·CG owns rows ra = t mod RH
+  // and rb = ra + RH (RH = ⌈R/2⌉) and chunk group cg = t / RH, i.e. the
+  // 64-weight chunks cg, cg + CG, ... of both rows.
+  const int RH = (R + 1) >> 1;
+  const int CG = gemv_chunk_groups(RH, K);
+  const int nchunks = (int)(K / 64);
+  const bool active = tid < RH * CG;
+  const int ra = active ? tid % RH : 0;
+  const int cg = active ? tid / RH : 0;
+  const bool has_b = ra + RH < R;
+  const int rb = has_b ? ra + RH : ra;
+  const uint8_t* wa = s_w + (size_t)ra * 128;
+  const uint8_t* wb = s_w + (size_t)rb * 128;
+  const int swa = ra & 7, swb = rb & 7;
+  auto wload = [&](const uint8_t* w, int sw, int c) {
+    // chunk c: box c/8, 16-byte slot (c mod 8) XOR (row mod 8)
+    return *reinterpret_cast<const uint4*>(w + (size_t)(c >> 3) * box_bytes + (((c & 7) ^ sw) << 4));
+  };
+
+  // 2. The weights do not depend on the previous kernel either: wait for
+  //    them and move this thread's first kRegChunks chunks into registers
+  //    before the dependency wait, so the contraction after it starts from
+  //    registers.
+  //    One thread waits (bounded) and the outcome is made CTA-uniform, so a
+  //    give-up returns every thread together and no barrier is left waiting.
+  __shared__ int s_wok;
+  if (tid == 0) s_wok = mbar_wait(s_bar, 0) ? 1 : 0;
+  __syncthreads();
+  if (!s_wok) {
+    // Gave up: the error flag is raised and this CTA's outputs stay
+    // untouched. The wait that gave up was the wait for its own copies.
+    return;
+  }
+  mbar_wait(s_bar, 0);  // phase complete: acquires the copies for this thread
+  constexpr int kRegChunks = MT <= 2 ? 2 : 0;
+  uint4 rwa[kRegChunks > 0 ? kRegChunks : 1], rwb[kRegChunks > 0 ? kRegChunks : 1];
+#pragma unroll
+  for (int i = 0; i < kRegChunks; ++i) {
+    const int c = cg + i * CG;
+    if (active && c < nchunks) {
+      rwa[i] = wload(wa, swa, c);
+      rwb[i] = wload(wb, swb, c);
+    }
+  }
+
+  // Tokens and outputs are ordered after the previous kernel. One warp
+  // waits for the prior grid; the others wait at the CTA barrier, so a CTA
+  // launched early spends no issue slots while its predecessor runs.
   if (warp == 0) pdl_wait_prior_grid();
   __syncthreads();
 
@@ -218,16 +265,18 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
         const float s = __fdiv_rn(127.0f, __fadd_rn(g, p.eps));
         const uint4* src = row_ptr(m);
         auto emit = [&](const uint4& u, int64_t v) {
-          int8_t q[VEC];
+          uint32_t b[VEC], w[VEC / 4];
 #pragma unroll
-          for (int i = 0; i < VEC; ++i) {
-            q[i] = quant_i8(value(u, i, m), s);
-            tsum += q[i];
+          for (int i = 0; i < VEC; ++i) b[i] = quant_i8_bits(value(u, i, m), s);
+#pragma unroll
+          for (int i = 0; i < VEC / 4; ++i) {
+            w[i] = pack4_low_bytes(b[4 * i], b[4 * i + 1], b[4 * i + 2], b[4 * i + 3]);
+            tsum = dp4a(w[i], 0x01010101u, tsum);  // Σ of the four int8 values
           }
           if constexpr (VEC == 8)
-            *reinterpret_cast<uint2*>(s_a + m * K + v * VEC) = *reinterpret_cast<uint2*>(q);
+            *reinterpret_cast<uint2*>(s_a + m * K + v * VEC) = make_uint2(w[0], w[1]);
           else
-            *reinterpret_cast<uint32_t*>(s_a + m * K + v * VEC) = *reinterpret_cast<uint32_t*>(q);
+            *reinterpret_cast<uint32_t*>(s_a + m * K + v * VEC) = w[0];
         };
 #pragma unroll
         for (int r = 0; r < RV; ++r) {
@@ -270,27 +319,10 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
   }
   __syncthreads();
 
-  // 4. Weights must have landed: every thread observes the completed phase.
-  if (!mbar_wait(s_bar, 0)) {
-    // Gave up: the error flag is raised and this CTA's outputs stay
-    // untouched. The wait that gave up was the wait for its own copies.
-    return;
-  }
-
-  // 5. Contraction. Thread t < RH·CG owns rows r = t mod RH and r + RH
-  //    (RH = ⌈R/2⌉) and the chunk group cg = t / RH: the 64-weight chunks
-  //    cg, cg + CG, ... of both rows. The two rows share every token load and
-  //    keep 8 independent accumulators per token. Consecutive lanes take
+  // 5. Contraction (mapping above). The two rows share every token load
+  //    and keep 8 independent accumulators per token. Consecutive lanes take
   //    consecutive rows at the same chunk: the swizzle keeps their weight
   //    loads conflict-free and the token loads are broadcasts.
-  const int RH = (R + 1) >> 1;
-  const int CG = gemv_chunk_groups(RH, K);
-  const int nchunks = (int)(K / 64);
-  const bool active = tid < RH * CG;
-  const int ra = active ? tid % RH : 0;
-  const int cg = active ? tid / RH : 0;
-  const bool has_b = ra + RH < R;
-  const int rb = has_b ? ra + RH : ra;
   int acc[2][MT][4];
 #pragma unroll
   for (int h = 0; h < 2; ++h)
@@ -298,66 +330,56 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
     for (int m = 0; m < MT; ++m)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[h][m][j] = 0;
-  if (active) {
-    const uint8_t* wa = s_w + (size_t)ra * 128;
-    const uint8_t* wb = s_w + (size_t)rb * 128;
-    const int swa = ra & 7, swb = rb & 7;
-#pragma unroll 2
-    for (int c = cg; c < nchunks; c += CG) {
-      // chunk c: box c/8, 16-byte slot (c mod 8) XOR (row mod 8)
-      const size_t box = (size_t)(c >> 3) * box_bytes;
-      const uint4 va = *reinterpret_cast<const uint4*>(wa + box + (((c & 7) ^ swa) << 4));
-      const uint4 vb = *reinterpret_cast<const uint4*>(wb + box + (((c & 7) ^ swb) << 4));
-      const uint32_t xa[4] = {va.x, va.y, va.z, va.w};
-      const uint32_t xb[4] = {vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        if (m < M) {
-          const uint4* ap = reinterpret_cast<const uint4*>(s_a + m * K + c * 64);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 a = ap[q];  // token words 16c+4q .. 16c+4q+3
-            acc[0][m][0] = dp4a_us(xa[q] & 0x03030303u, a.x, acc[0][m][0]);
-            acc[1][m][0] = dp4a_us(xb[q] & 0x03030303u, a.x, acc[1][m][0]);
-            acc[0][m][1] = dp4a_us(xa[q] & 0x0C0C0C0Cu, a.y, acc[0][m][1]);
-            acc[1][m][1] = dp4a_us(xb[q] & 0x0C0C0C0Cu, a.y, acc[1][m][1]);
-            acc[0][m][2] = dp4a_us(xa[q] & 0x30303030u, a.z, acc[0][m][2]);
-            acc[1][m][2] = dp4a_us(xb[q] & 0x30303030u, a.z, acc[1][m][2]);
-            acc[0][m][3] = dp4a_us(xa[q] & 0xC0C0C0C0u, a.w, acc[0][m][3]);
-            acc[1][m][3] = dp4a_us(xb[q] & 0xC0C0C0C0u, a.w, acc[1][m][3]);
-          }
-        }
-      }
-    }
-    // Σ c·a over this thread's chunks; acc[j] is a multiple of 4^j, so the
-    // arithmetic shifts are exact.
+  auto contract = [&](const uint4& va, const uint4& vb, int c) {
+    const uint32_t xa[4] = {va.x, va.y, va.z, va.w};
+    const uint32_t xb[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
       if (m < M) {
-        int* part = s_part + (m * CG + cg) * R;
-        part[ra] = acc[0][m][0] + (acc[0][m][1] >> 2) + (acc[0][m][2] >> 4) + (acc[0][m][3] >> 6);
+        const uint4* ap = reinterpret_cast<const uint4*>(s_a + m * K + c * 64);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 a = ap[q];  // token words 16c+4q .. 16c+4q+3
+          acc[0][m][0] = dp4a_us(xa[q] & 0x03030303u, a.x, acc[0][m][0]);
+          acc[1][m][0] = dp4a_us(xb[q] & 0x03030303u, a.x, acc[1][m][0]);
+          acc[0][m][1] = dp4a_us(xa[q] & 0x0C0C0C0Cu, a.y, acc[0][m][1]);
+          acc[1][m][1] = dp4a_us(xb[q] & 0x0C0C0C0Cu, a.y, acc[1][m][1]);
+          acc[0][m][2] = dp4a_us(xa[q] & 0x30303030u, a.z, acc[0][m][2]);
+          acc[1][m][2] = dp4a_us(xb[q] & 0x30303030u, a.z, acc[1][m][2]);
+          acc[0][m][3] = dp4a_us(xa[q] & 0xC0C0C0C0u, a.w, acc[0][m][3]);
+          acc[1][m][3] = dp4a_us(xb[q] & 0xC0C0C0C0u, a.w, acc[1][m][3]);
+        }
+      }
+    }
+  };
+  if (active) {
+#pragma unroll
+    for (int i = 0; i < kRegChunks; ++i) {
+      const int c = cg + i * CG;
+      if (c < nchunks) contract(rwa[i], rwb[i], c);
+    }
+#pragma unroll 2
+    for (int c = cg + kRegChunks * CG; c < nchunks; c += CG)
+      contract(wload(wa, swa, c), wload(wb, swb, c), c);
+    // Σ c·a over this thread's chunks (acc[j] is a multiple of 4^j, so the
+    // arithmetic shifts are exact), accumulated per row in shared memory.
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      if (m < M) {
+        atomicAdd(&s_part[m * R + ra],
+                  acc[0][m][0] + (acc[0][m][1] >> 2) + (acc[0][m][2] >> 4) + (acc[0][m][3] >> 6));
         if (has_b)
-          part[rb] = acc[1][m][0] + (acc[1][m][1] >> 2) + (acc[1][m][2] >> 4) + (acc[1][m][3] >> 6);
+          atomicAdd(&s_part[m * R + rb],
+                    acc[1][m][0] + (acc[1][m][1] >> 2) + (acc[1][m][2] >> 4) + (acc[1][m][3] >> 6));
       }
     }
   }
   __syncthreads();
 
-  // 6. Epilogue: combine the chunk groups, undo the code offset, scale.
+  // 6. Epilogue: undo the code offset, scale.
   for (int e = tid; e < M * R; e += kGemvThreads) {
     const int m = e / R, r = e - m * R;
-    // Four independent partial sums keep the shared loads in flight together.
-    const int* pp = s_part + m * CG * R + r;
-    int d0 = 0, d1 = 0, d2 = 0, d3 = 0;
-    int k = 0;
-    for (; k + 4 <= CG; k += 4) {
-      d0 += pp[(k + 0) * R];
-      d1 += pp[(k + 1) * R];
-      d2 += pp[(k + 2) * R];
-      d3 += pp[(k + 3) * R];
-    }
-    for (; k < CG; ++k) d0 += pp[k * R];
-    const int v = (d0 + d1) + (d2 + d3) - s_sum[m];
+    const int v = s_part[m * R + r] - s_sum[m];
     const int64_t o = (int64_t)m * p.N + r0 + r;
     if constexpr (OUT == kOutRawI32) {
       reinterpret_cast<int32_t*>(p.Y)[o] = v;

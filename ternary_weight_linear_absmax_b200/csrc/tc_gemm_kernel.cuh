@@ -14,12 +14,13 @@
 //               weight tile into one shared-memory stage.
 //  * warp 1   : allocates TMEM, issues tcgen05.mma (one elected thread) and
 //               commits completion to the stage barriers.
-//  * warps 2-5: expansion, then epilogue. Each thread owns one weight row
-//               (one TMEM lane): it turns 32 packed bytes (128 codes) into
-//               32 words of int8 codes {0,1,2} — two ALU ops per 4 weights —
-//               and stores them with tcgen05.st straight into TMEM, where
-//               the MMA reads its A operand. Nothing expanded goes through
-//               shared memory.
+//  * warps 2-9: expansion, then epilogue. Two warps share each TMEM lane
+//               quarter; a thread owns one weight row (one TMEM lane) and
+//               half of each K block: it turns 16 packed bytes (64 codes)
+//               into 16 words of int8 codes {0,1,2} — two ALU ops per 4
+//               weights — and stores them with tcgen05.st straight into
+//               TMEM, where the MMA reads its A operand. Nothing expanded
+//               goes through shared memory.
 //  * The accumulator D[weight row, token] lives in TMEM (int32). The
 //    epilogue reads it with tcgen05.ld, subtracts the token's Σ A_q (codes
 //    are w+1), scales by (γ_A·γ)/127 (optionally ReLU²) and stores.
@@ -31,7 +32,10 @@
 
 namespace bl {
 
-constexpr int kTcThreads = 192;
+// Warps: 0 TMA producer, 1 MMA issuer, 2..9 expansion + epilogue (two per
+// TMEM lane quarter).
+constexpr int kTcThreads = 320;
+constexpr int kTcMathThreads = 256;
 constexpr int kTcBK = 128;  // int8 K elements per stage (one 128-byte swizzle row)
 
 enum TcOut : int { kTcDequant = 0, kTcRawI32 = 1 };
@@ -72,7 +76,7 @@ struct TcConfig {
   static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
                                    : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
   static constexpr int kRingBytes = kSStages * kBStage + kWStages * kWStage;
-  static constexpr int kBarBytes = (2 * kSStages + 2 * kWStages + 2 * kTStages + 2) * 8;
+  static constexpr int kBarBytes = (2 * kSStages + 2 * kWStages + 2 * kTStages + 3) * 8;
   static constexpr int kParamBytes = BN * 8;
   // 1 KiB slack for aligning the dynamic buffer to 1024 bytes. At least
   // 116 KiB are requested so that only one CTA is resident per SM: every CTA
@@ -163,25 +167,22 @@ __device__ __forceinline__ void tc_epilogue_chunk(const uint32_t (&d)[CW], int c
 // (summing the kAcc accumulators), with the next chunk's load issued before
 // the current chunk is processed.
 template <int BN, int OUT, bool RELU, bool BF16, bool STAGE>
-__device__ __forceinline__ void tc_epilogue(uint32_t t_lane, int row, const float* s_sc,
+__device__ __forceinline__ void tc_epilogue(uint32_t t_lane, int row, int half, const float* s_sc,
                                             const int* s_rs, uint8_t* stage, const TcParams& p,
                                             int64_t m0, int64_t n) {
   using C = TcConfig<BN>;
-  constexpr int CW = BN >= 32 ? 32 : 16;
+  // 16-column chunks, alternating between the two warps of a lane quarter.
+  constexpr int CW = 16;
+  const int c_begin = half * CW;
+  if (c_begin >= BN) return;
   auto load = [&](int c0, uint32_t (&d)[CW]) {
-    if constexpr (CW == 32)
-      tmem_ld_32x32b_x32(t_lane + c0, d);
-    else
-      tmem_ld_32x32b_x16(t_lane + c0, d);
+    tmem_ld_32x32b_x16(t_lane + c0, d);
     if constexpr (C::kAcc > 1) {
       tmem_wait_ld();
 #pragma unroll
       for (int a = 1; a < C::kAcc; ++a) {
         uint32_t e[CW];
-        if constexpr (CW == 32)
-          tmem_ld_32x32b_x32(t_lane + a * C::kDCols + c0, e);
-        else
-          tmem_ld_32x32b_x16(t_lane + a * C::kDCols + c0, e);
+        tmem_ld_32x32b_x16(t_lane + a * C::kDCols + c0, e);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < CW; ++j) d[j] = (uint32_t)((int)d[j] + (int)e[j]);
@@ -189,12 +190,12 @@ __device__ __forceinline__ void tc_epilogue(uint32_t t_lane, int row, const floa
     }
   };
   uint32_t cur[CW], nxt[CW];
-  load(0, cur);
+  load(c_begin, cur);
   tmem_wait_ld();
 #pragma unroll 1
-  for (int c0 = 0; c0 < BN; c0 += CW) {
-    const bool more = c0 + CW < BN;
-    if (more) load(c0 + CW, nxt);  // in flight while this chunk is processed
+  for (int c0 = c_begin; c0 < BN; c0 += 2 * CW) {
+    const bool more = c0 + 2 * CW < BN;
+    if (more) load(c0 + 2 * CW, nxt);  // in flight while this chunk is processed
     tc_epilogue_chunk<CW, OUT, RELU, BF16, STAGE>(cur, c0, row, s_sc, s_rs, stage, p, m0, n);
     if (more) {
       tmem_wait_ld();
@@ -224,7 +225,8 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
   uint64_t* afull = bars + 2 * SS + 2 * WS;         // [TS] A operand in TMEM ready
   uint64_t* aempty = afull + TS;                    // [TS] MMA done with A stage
   uint64_t* done = aempty + TS;                     // accumulator complete
-  uint64_t* staged = done + 1;                      // output tile staged (128 arrivals)
+  uint64_t* staged = done + 1;                      // output tile staged (math threads)
+  uint64_t* pready = done + 2;                      // epilogue parameters in shared memory
   float* s_sc = reinterpret_cast<float*>(smem + C::kRingBytes + C::kBarBytes);
   int* s_rs = reinterpret_cast<int*>(s_sc + BN);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_rs + BN);
@@ -236,17 +238,6 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
   const int64_t m0 = (int64_t)blockIdx.y * BN;
   const int KB = (int)((p.K + kTcBK - 1) / kTcBK);
 
-  // Per-token epilogue parameters.
-  {
-    // γ and γ_A are absent for raw INT32 output.
-    const float g = p.gamma != nullptr ? *p.gamma : 0.0f;
-    for (int j = tid; j < BN; j += kTcThreads) {
-      const int64_t m = m0 + j;
-      s_sc[j] = (m < p.M && p.gammaA != nullptr) ? __fdiv_rn(__fmul_rn(p.gammaA[m], g), 127.0f)
-                                                  : 0.0f;
-      s_rs[j] = m < p.M ? p.rowsum[m] : 0;
-    }
-  }
   if (tid == 0) {
     for (int s = 0; s < SS; ++s) {
       mbar_init(&full[s], 1);
@@ -254,14 +245,15 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
     }
     for (int v = 0; v < WS; ++v) {
       mbar_init(&wfull[v], 1);
-      mbar_init(&wempty[v], 128);
+      mbar_init(&wempty[v], kTcMathThreads);
     }
     for (int t = 0; t < TS; ++t) {
-      mbar_init(&afull[t], 128);
+      mbar_init(&afull[t], kTcMathThreads);
       mbar_init(&aempty[t], 1);
     }
     mbar_init(done, 1);
-    mbar_init(staged, 128);
+    mbar_init(staged, kTcMathThreads);
+    mbar_init(pready, kTcMathThreads);
     *s_abort = 0;
     fence_barrier_init();
     prefetch_tensormap(&tm_act);
@@ -328,10 +320,29 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
     }
     mma_commit_warp(done);  // also on abort: tracks every MMA issued
   } else {
-    // ---------------- expansion (warps 2..5) ----------------
+    // ---------------- expansion (warps 2..9) ----------------
     const int q = warp & 3;         // TMEM lane quarter this warp may access
+    const int hw = (warp - 2) >> 2; // which half of each K block (and of the epilogue columns)
     const int row = 32 * q + lane;  // weight row within the tile
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
+    const int mtid = tid - 64;      // 0 .. 255 among the math warps
+    // Per-token epilogue parameters, loaded now and parked in registers; they
+    // are written to shared memory after the main loop (only the epilogue
+    // reads them), so their memory latency overlaps the main loop.
+    constexpr int kPar = (BN + kTcMathThreads - 1) / kTcMathThreads;
+    float par_sc[kPar];
+    int par_rs[kPar];
+    {
+      const float g = p.gamma != nullptr ? __ldg(p.gamma) : 0.0f;  // absent for raw INT32 output
+#pragma unroll
+      for (int i = 0; i < kPar; ++i) {
+        const int j = mtid + i * kTcMathThreads;
+        const int64_t m = m0 + j;
+        const bool in = j < BN && m < p.M;
+        par_sc[i] = (in && p.gammaA != nullptr) ? __fdiv_rn(__fmul_rn(__ldg(p.gammaA + m), g), 127.0f) : 0.0f;
+        par_rs[i] = in ? __ldg(p.rowsum + m) : 0;
+      }
+    }
     for (int kb = 0; kb < KB; ++kb) {
       const int t = kb % TS, ws = kb >> 2, v = ws % WS, sub = kb & 3;
       // tcgen05.st is warp-collective: the whole warp continues or stops.
@@ -340,22 +351,32 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       // This K block is 16-byte chunks 2·sub and 2·sub+1 of the row's 128-byte
-      // line; the 128-byte swizzle stores chunk j at slot j ^ (row mod 8).
+      // line (this warp takes chunk 2·sub + hw); the 128-byte swizzle stores
+      // chunk j at slot j ^ (row mod 8).
       const uint8_t* line = s_w + v * C::kWStage + row * 128;
-      const uint4 u0 = *reinterpret_cast<const uint4*>(line + (((2 * sub) ^ (row & 7)) << 4));
-      const uint4 u1 = *reinterpret_cast<const uint4*>(line + (((2 * sub + 1) ^ (row & 7)) << 4));
+      const uint4 u = *reinterpret_cast<const uint4*>(line + (((2 * sub + hw) ^ (row & 7)) << 4));
       if (sub == 3 || kb == KB - 1) mbar_arrive(&wempty[v]);  // done reading this stage
-      const uint32_t x[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-      uint32_t vv[32];
+      const uint32_t x[4] = {u.x, u.y, u.z, u.w};
+      uint32_t vv[16];
 #pragma unroll
-      for (int g = 0; g < 8; ++g) expand_word(x[g], vv[4 * g], vv[4 * g + 1], vv[4 * g + 2], vv[4 * g + 3]);
-      tmem_st_32x32b_x32(tmem + lane_addr + C::kACol + t * 32, vv);
+      for (int g = 0; g < 4; ++g) expand_word(x[g], vv[4 * g], vv[4 * g + 1], vv[4 * g + 2], vv[4 * g + 3]);
+      tmem_st_32x32b_x16(tmem + lane_addr + C::kACol + t * 32 + hw * 16, vv);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&afull[t]);
     }
+#pragma unroll
+    for (int i = 0; i < kPar; ++i) {
+      const int j = mtid + i * kTcMathThreads;
+      if (j < BN) {
+        s_sc[j] = par_sc[i];
+        s_rs[j] = par_rs[i];
+      }
+    }
+    mbar_arrive(pready);  // parameters visible to all math warps
     // ---------------- epilogue ----------------
     bool ok = wait_or_abort(done, 0, s_abort);
+    if (ok) ok = wait_or_abort(pready, 0, s_abort);
     ok = __all_sync(0xffffffffu, ok && !*s_abort);  // tcgen05.ld is warp-collective
     if (ok) {
       tc_fence_after();
@@ -365,20 +386,20 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
       const uint32_t t_lane = tmem + lane_addr;
       if constexpr (OUT == kTcRawI32) {
         if (p.tma_store)
-          tc_epilogue<BN, OUT, false, false, true>(t_lane, row, s_sc, s_rs, smem, p, m0, n);
+          tc_epilogue<BN, OUT, false, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n);
         else
-          tc_epilogue<BN, OUT, false, false, false>(t_lane, row, s_sc, s_rs, smem, p, m0, n);
+          tc_epilogue<BN, OUT, false, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n);
       } else {
         const int sel = (p.tma_store ? 4 : 0) | (p.y_bf16 ? 2 : 0) | (p.relu2 ? 1 : 0);
         switch (sel) {
-          case 0: tc_epilogue<BN, OUT, false, false, false>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
-          case 1: tc_epilogue<BN, OUT, true, false, false>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
-          case 2: tc_epilogue<BN, OUT, false, true, false>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
-          case 3: tc_epilogue<BN, OUT, true, true, false>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
-          case 4: tc_epilogue<BN, OUT, false, false, true>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
-          case 5: tc_epilogue<BN, OUT, true, false, true>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
-          case 6: tc_epilogue<BN, OUT, false, true, true>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
-          default: tc_epilogue<BN, OUT, true, true, true>(t_lane, row, s_sc, s_rs, smem, p, m0, n); break;
+          case 0: tc_epilogue<BN, OUT, false, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
+          case 1: tc_epilogue<BN, OUT, true, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
+          case 2: tc_epilogue<BN, OUT, false, true, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
+          case 3: tc_epilogue<BN, OUT, true, true, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
+          case 4: tc_epilogue<BN, OUT, false, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
+          case 5: tc_epilogue<BN, OUT, true, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
+          case 6: tc_epilogue<BN, OUT, false, true, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
+          default: tc_epilogue<BN, OUT, true, true, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
         }
       }
       if (p.tma_store) fence_proxy_async_smem();  // staged writes -> visible to the tensor store
