@@ -12,6 +12,7 @@
 #include "bl_device.cuh"
 #include "gemv_kernel.cuh"
 #include "quant_kernels.cuh"
+#include "skinny_kernel.cuh"
 #include "tc_gemm_kernel.cuh"
 
 namespace bl {
@@ -349,6 +350,146 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
                            : launch_tc_bn<kTcRawI32>(bn, ta, tw, ty, p, dev, st);
 }
 
+// --------------------------------------------------------------------------
+// Skinny launches (5 ≤ M ≤ 64 tokens, mma.sync over all SMs).
+template <int MTT, int NTW, int KPS>
+bl_status launch_skinny_t(const CUtensorMap& tw, const CUtensorMap& ta, const SkinnyParams& p,
+                          int grid, size_t smem, bool pdl, int dev, cudaStream_t st) {
+  auto* k = skinny_ternary_kernel<MTT, NTW, KPS>;
+  BL_TRY(ensure_smem(k, dev, smem));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kSkThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  BL_CUDA(cudaLaunchKernelEx(&cfg, k, tw, ta, p));
+  return BL_OK;
+}
+
+// Instantiated warp splits (NTW n-tiles per warp, KPS 32-K steps per warp
+// and stage). With 16 warps, KPS n-tile groups cover KPS·NTW n-tiles.
+struct SkinnySplit {
+  int ntw, kps;
+};
+constexpr SkinnySplit kSkSplits[] = {{1, 2}, {2, 2}, {3, 2}, {5, 2}, {2, 4}, {3, 4}, {4, 4}};
+
+template <int MTT>
+bl_status launch_skinny_split(SkinnySplit sp, const CUtensorMap& tw, const CUtensorMap& ta,
+                              const SkinnyParams& p, int grid, size_t smem, bool pdl, int dev,
+                              cudaStream_t st) {
+  if (sp.kps == 2) {
+    switch (sp.ntw) {
+      case 1: return launch_skinny_t<MTT, 1, 2>(tw, ta, p, grid, smem, pdl, dev, st);
+      case 2: return launch_skinny_t<MTT, 2, 2>(tw, ta, p, grid, smem, pdl, dev, st);
+      case 3: return launch_skinny_t<MTT, 3, 2>(tw, ta, p, grid, smem, pdl, dev, st);
+      default:
+        if constexpr (MTT <= 2) return launch_skinny_t<MTT, 5, 2>(tw, ta, p, grid, smem, pdl, dev, st);
+        return BL_ERR_SHAPE;
+    }
+  }
+  switch (sp.ntw) {
+    case 2: return launch_skinny_t<MTT, 2, 4>(tw, ta, p, grid, smem, pdl, dev, st);
+    case 3: return launch_skinny_t<MTT, 3, 4>(tw, ta, p, grid, smem, pdl, dev, st);
+    default: return launch_skinny_t<MTT, 4, 4>(tw, ta, p, grid, smem, pdl, dev, st);
+  }
+}
+
+inline int skinny_mtt(int64_t M) { return M <= 16 ? 1 : (M <= 32 ? 2 : 4); }
+
+// Rows per CTA: one wave over the SMs (8..128 rows). The warp split
+// minimises a cycle estimate per CTA: per stage the larger of the mma.sync
+// time (≈2.2 SM cycles per m16n8k32, measured with the step loop unrolled)
+// and the shared-memory time (a 512-byte ldmatrix per token fragment, 64
+// bytes per weight fragment, 128 bytes per cycle), plus writing and reading
+// the K-lanes' partial sums once. The ring is as deep as shared memory
+// allows.
+bl_status skinny_plan(int64_t M, int64_t N, int64_t K, int sms, SkinnyParams* p,
+                      SkinnySplit* split, int* grid, size_t* smem) {
+  const int mtt = skinny_mtt(M);
+  int64_t r = (N + sms - 1) / sms;
+  if (r < 8) r = 8;
+  if (r > kSkMaxRowsPad) r = kSkMaxRowsPad;
+  const int nt = (int)((r + 7) / 8);
+  const int rp = nt * 8;
+  const int nchunk = skinny_chunks(K);
+  SkinnySplit best = {0, 0};
+  double best_cost = 1e30;
+  for (const SkinnySplit& sp : kSkSplits) {
+    if (sp.ntw * sp.kps < nt) continue;      // n-tiles not covered
+    if (sp.ntw * mtt > 16) continue;         // accumulator registers
+    if (mtt == 4 && sp.ntw > 4) continue;    // not instantiated
+    const double t_mma = (double)kSkWarps * sp.kps * sp.ntw * mtt * 2.2;
+    const double t_smem = (double)kSkWarps * sp.kps * (4.0 * mtt + sp.ntw / 2.0);
+    const double cost = nchunk * (t_mma > t_smem ? t_mma : t_smem) +
+                        2.0 * (double)skinny_red_bytes(sp.ntw, mtt) / 128.0;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = sp;
+    }
+  }
+  if (best.ntw == 0) return BL_ERR_SHAPE;
+  int stages = nchunk;
+  while (stages > 1 && skinny_smem_bytes(rp, mtt, stages, best.ntw) > kSkSmemCap) --stages;
+  if (skinny_smem_bytes(rp, mtt, stages, best.ntw) > kSkSmemCap) return BL_ERR_SHAPE;
+  if (stages < 2 && nchunk > 1) return BL_ERR_SHAPE;
+  p->rows_per_cta = (int)r;
+  p->rows_pad = rp;
+  p->stages = stages;
+  *split = best;
+  *grid = (int)((N + r - 1) / r);
+  *smem = skinny_smem_bytes(rp, mtt, stages, best.ntw);
+  return BL_OK;
+}
+
+// acc/Y[M,N] = epilogue(A_q[M,K] · W_q[N,K]ᵀ − rowsum) for 5 ≤ M ≤ 64.
+// pdl: the preceding kernel on the stream does not write W_packed or gamma.
+bl_status run_skinny(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,
+                     const float* gamma, const float* gammaA, const int32_t* rowsum, void* Y,
+                     int raw, int relu2, int y_bf16, bool pdl, int dev, int sms,
+                     cudaStream_t st) {
+  SkinnyParams p = {};
+  SkinnySplit split;
+  int grid;
+  size_t smem;
+  BL_TRY(skinny_plan(M, N, K, sms, &p, &split, &grid, &smem));
+  const int mtt = skinny_mtt(M);
+  CUtensorMap tw, ta;
+  BL_TRY(make_map_u8(&tw, Wp, (uint64_t)N, (uint64_t)(K / 4), 128, (uint32_t)p.rows_pad,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+  BL_TRY(make_map_u8(&ta, Aq, (uint64_t)M, (uint64_t)K, 128, (uint32_t)(16 * mtt),
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+  p.gamma = gamma;
+  p.gammaA = gammaA;
+  p.rowsum = rowsum;
+  p.Y = Y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.relu2 = relu2;
+  p.y_bf16 = y_bf16;
+  p.raw = raw;
+  if (mtt == 1) return launch_skinny_split<1>(split, tw, ta, p, grid, smem, pdl, dev, st);
+  if (mtt == 2) return launch_skinny_split<2>(split, tw, ta, p, grid, smem, pdl, dev, st);
+  return launch_skinny_split<4>(split, tw, ta, p, grid, smem, pdl, dev, st);
+}
+
+// Contraction of pre-quantised tokens: the skinny kernel up to 64 tokens,
+// tensor cores above. out: kTcDequant or kTcRawI32.
+bl_status run_contract(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,
+                       const float* gamma, const float* gammaA, const int32_t* rowsum, void* Y,
+                       int out, int relu2, int y_bf16, bool pdl, int dev, int sms,
+                       cudaStream_t st) {
+  if (M <= kSkMaxTokens)
+    return run_skinny(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out == kTcRawI32 ? 1 : 0, relu2,
+                      y_bf16, pdl, dev, sms, st);
+  return run_tc(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out, relu2, y_bf16, dev, st);
+}
+
 bl_status run_quant_acts(const void* A, bl_dtype dt, int64_t M, int64_t K, float eps, int8_t* Aq,
                          float* gA, int32_t* rs, cudaStream_t st) {
   if (M == 0) return BL_OK;
@@ -500,7 +641,8 @@ bl_status bl_zero_gemm(const int8_t* A_q, int64_t M, int64_t K, const uint8_t* W
   int32_t* rs = reinterpret_cast<int32_t*>(workspace);
   rowsum_i8_kernel<<<(unsigned)M, kQuantThreads, 0, st>>>(A_q, K, rs);
   BL_CUDA(cudaGetLastError());
-  return run_tc(A_q, W_packed, M, K, N, nullptr, nullptr, rs, acc, kTcRawI32, 0, 0, dev, st);
+  return run_contract(A_q, W_packed, M, K, N, nullptr, nullptr, rs, acc, kTcRawI32, 0, 0, true,
+                      dev, sms, st);
 }
 
 size_t bl_linear_q_workspace_bytes(int64_t M, int64_t K, int64_t N) {
@@ -556,8 +698,10 @@ bl_status bl_linear_q(const int8_t* A_q, const float* gamma_A, const int32_t* ro
     BL_CUDA(cudaGetLastError());
     rs = w;
   }
-  return run_tc(A_q, W_packed, M, K, N, gamma, gamma_A, rs, Y, kTcDequant, relu2 ? 1 : 0,
-                y_dtype == BL_BF16, dev, st);
+  // After this call's row-sum kernel the weights may stream early; without
+  // it the preceding kernel is the caller's, so no early start.
+  return run_contract(A_q, W_packed, M, K, N, gamma, gamma_A, rs, Y, kTcDequant, relu2 ? 1 : 0,
+                      y_dtype == BL_BF16, rowsum == nullptr, dev, sms, st);
 }
 
 size_t bl_linear_workspace_bytes(int64_t M, int64_t K, int64_t N) {
@@ -610,8 +754,8 @@ bl_status bl_linear_ex(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
   float* gA = reinterpret_cast<float*>(base + w.gamma);
   int32_t* rs = reinterpret_cast<int32_t*>(base + w.rowsum);
   BL_TRY(run_quant_acts(A, a_dtype, M, K, eps, Aq, gA, rs, st));
-  return run_tc(Aq, W_packed, M, K, N, gamma, gA, rs, Y, kTcDequant, relu2 ? 1 : 0,
-                y_dtype == BL_BF16, dev, st);
+  return run_contract(Aq, W_packed, M, K, N, gamma, gA, rs, Y, kTcDequant, relu2 ? 1 : 0,
+                      y_dtype == BL_BF16, true, dev, sms, st);
 }
 
 bl_status bl_linear(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
@@ -684,12 +828,15 @@ bl_status bl_ffn_relu2(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, in
   float* gR = reinterpret_cast<float*>(base + w.gamma_r);
   int32_t* rsR = reinterpret_cast<int32_t*>(base + w.rs_r);
   BL_TRY(run_quant_acts(X, x_dtype, M, K, eps, Xq, gX, rsX, st));
-  BL_TRY(run_tc(Xq, W_up, M, K, H, gamma_up, gX, rsX, acc_up, kTcRawI32, 0, 0, dev, st));
+  // Each contraction follows one of this call's own kernels, which write
+  // neither W_up nor W_down: the weights may stream early (PDL).
+  BL_TRY(run_contract(Xq, W_up, M, K, H, gamma_up, gX, rsX, acc_up, kTcRawI32, 0, 0, true, dev,
+                      sms, st));
   relu2_requant_kernel<<<(unsigned)M, kQuantThreads, 0, st>>>(acc_up, H, gX, gamma_up, eps, Rq, gR,
                                                               rsR);
   BL_CUDA(cudaGetLastError());
-  return run_tc(Rq, W_down, M, H, K, gamma_down, gR, rsR, Y, kTcDequant, 0, y_dtype == BL_BF16,
-                dev, st);
+  return run_contract(Rq, W_down, M, H, K, gamma_down, gR, rsR, Y, kTcDequant, 0,
+                      y_dtype == BL_BF16, true, dev, sms, st);
 }
 
 bl_status bl_check_device_error(bl_stream_t stream) {
@@ -785,8 +932,8 @@ extern "C" bl_status bl_linear_noalloc(const void* A, bl_dtype a_dtype, int64_t 
   float* gA = reinterpret_cast<float*>(base + w.gamma);
   int32_t* rs = reinterpret_cast<int32_t*>(base + w.rowsum);
   BL_TRY(run_quant_acts(A, a_dtype, M, K, eps, Aq, gA, rs, st));
-  return run_tc(Aq, W_packed, M, K, N, gamma, gA, rs, Y, kTcDequant, relu2 ? 1 : 0,
-                y_dtype == BL_BF16, dev, st);
+  return run_contract(Aq, W_packed, M, K, N, gamma, gA, rs, Y, kTcDequant, relu2 ? 1 : 0,
+                      y_dtype == BL_BF16, true, dev, sms, st);
 }
 
 namespace bl {

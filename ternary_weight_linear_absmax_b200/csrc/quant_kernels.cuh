@@ -110,6 +110,9 @@ template <typename T>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_acts_kernel(const T* __restrict__ A, int64_t K, float eps, int8_t* __restrict__ Aq,
                   float* __restrict__ gammaA, int32_t* __restrict__ rowsum) {
+  // A kernel launched after this one with programmatic dependent launch may
+  // start its own independent work now; it waits for this grid's results.
+  pdl_launch_dependents();
   const int64_t m = blockIdx.x;
   const T* row = A + m * K;
   constexpr int VEC = 16 / sizeof(T);
@@ -171,6 +174,7 @@ quant_acts_kernel(const T* __restrict__ A, int64_t K, float eps, int8_t* __restr
 // quantised activations without their sums.
 __global__ void __launch_bounds__(kQuantThreads)
 rowsum_i8_kernel(const int8_t* __restrict__ Aq, int64_t K, int32_t* __restrict__ rowsum) {
+  pdl_launch_dependents();
   const int64_t m = blockIdx.x;
   const uint4* r4 = reinterpret_cast<const uint4*>(Aq + m * K);
   int sum = 0;
@@ -203,6 +207,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 relu2_requant_kernel(const int32_t* __restrict__ acc, int64_t H, const float* __restrict__ gammaX,
                      const float* __restrict__ g_up, float eps, int8_t* __restrict__ Rq,
                      float* __restrict__ gammaR, int32_t* __restrict__ rowsum) {
+  pdl_launch_dependents();
   const int64_t m = blockIdx.x;
   const int4* a4 = reinterpret_cast<const int4*>(acc + m * H);
   const float sc = __fdiv_rn(__fmul_rn(gammaX[m], *g_up), 127.0f);

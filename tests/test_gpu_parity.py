@@ -188,8 +188,10 @@ def test_quant_acts_special_rows(bl):
 
 ZG_CASES = [
     (1, 64, 128), (2, 128, 200), (3, 192, 256), (4, 512, 256),      # GEMV path
-    (5, 128, 128), (16, 4096, 384), (17, 192, 200), (33, 512, 130),  # tensor-core path
-    (64, 1024, 256), (100, 320, 256), (128, 256, 128), (129, 640, 260),
+    (5, 128, 128), (16, 4096, 384), (17, 192, 200), (33, 512, 130),  # skinny path (5..64 tokens)
+    (64, 1024, 256), (8, 64, 1), (48, 3200, 1500), (20, 640, 9000),
+    (7, 64, 20000), (64, 4096, 4096), (32, 4096, 11008),
+    (65, 256, 200), (100, 320, 256), (128, 256, 128), (129, 640, 260),  # tensor-core path
     (256, 512, 384), (300, 384, 512), (520, 128, 136),
 ]
 
@@ -280,7 +282,7 @@ def test_linear_gemv_multi_token(bl, M):
 
 
 def test_linear_small_batch_full(bl):
-    """M=16, K=4096, N=11008 (tensor-core path), all outputs."""
+    """M=16, K=4096, N=11008 (skinny path), all outputs."""
     _linear_case(bl, 16, 4096, 11008, "bf16", "bf16", True, torch.bfloat16)
 
 
@@ -382,5 +384,28 @@ def test_pdl_chain_distinct_weights(bl):
     for p, g in Ws:
         outs.append(bl.bl_linear(At, p, g, EPS, pdl=True))
     torch.cuda.synchronize()
+    for y, r in zip(outs, refs):
+        assert_close(y.float().cpu().numpy(), r, torch.bfloat16)
+
+
+def test_skinny_chain_shared_workspace(bl):
+    """Back-to-back 16-token calls that share one workspace: each call's
+    contraction streams its weights before the quantiser of the same call has
+    finished (programmatic dependent launch) and must still read its own
+    call's tokens, not the next call's."""
+    M, K, N = 16, 1024, 2048
+    ws = torch.empty(bl.workspace_bytes("linear", M, K, N), dtype=torch.uint8, device=DEV)
+    cases, args = [], []
+    for i in range(6):
+        W = si.weights(N, K, seed=200 + i, dtype="bf16")
+        codes, g = oracle.quant_weights(W.f32, EPS)
+        A = si.activations(M, K, seed=300 + i, dtype="bf16", outliers=True)
+        cases.append((A, codes, g))
+        args.append((A.torch(DEV), to_dev(oracle.pack_ternary(codes)),
+                     to_dev(np.array([g], np.float32))))
+    torch.cuda.synchronize()
+    outs = [bl.bl_linear(a, p, g, EPS, workspace=ws) for a, p, g in args]  # back to back
+    torch.cuda.synchronize()
+    refs = [oracle.bitlinear(A.f32, codes, g, EPS)["Y"] for A, codes, g in cases]
     for y, r in zip(outs, refs):
         assert_close(y.float().cpu().numpy(), r, torch.bfloat16)
