@@ -414,6 +414,7 @@ bl_status skinny_plan(int64_t M, int64_t N, int64_t K, int sms, SkinnyParams* p,
   int64_t r = (N + sms - 1) / sms;
   if (r < 8) r = 8;
   if (r > kSkMaxRowsPad) r = kSkMaxRowsPad;
+  if ((N & 1) == 0 && (r & 1) != 0) ++r;  // even rows per CTA: paired output stores
   const int nt = (int)((r + 7) / 8);
   const int rp = nt * 8;
   const int nchunk = skinny_chunks(K);

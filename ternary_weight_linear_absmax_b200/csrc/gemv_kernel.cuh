@@ -99,6 +99,26 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
   return d;
 }
 
+// Combine the per-warp entries of one token (16 values, 16-byte aligned).
+__device__ __forceinline__ unsigned warp_slots_max(const unsigned (&v)[kGemvWarps]) {
+  unsigned r = 0u;
+#pragma unroll
+  for (int i = 0; i < kGemvWarps; i += 4) {
+    const uint4 q = *reinterpret_cast<const uint4*>(v + i);
+    r = max(r, max(max(q.x, q.y), max(q.z, q.w)));
+  }
+  return r;
+}
+__device__ __forceinline__ int warp_slots_sum(const int (&v)[kGemvWarps]) {
+  int r = 0;
+#pragma unroll
+  for (int i = 0; i < kGemvWarps; i += 4) {
+    const int4 q = *reinterpret_cast<const int4*>(v + i);
+    r += (q.x + q.y) + (q.z + q.w);
+  }
+  return r;
+}
+
 template <int MT, typename TA, int SRC, int OUT>
 __global__ void __launch_bounds__(kGemvThreads, 2)
 gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p) {
@@ -106,8 +126,10 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  __shared__ unsigned s_max[MT];  // per-token max as float bits (all values are ≥ 0)
-  __shared__ int s_sum[MT];       // per-token Σ A_q
+  // Per-warp partial results (no shared atomics): the max as float bits (all
+  // values are ≥ 0) and Σ A_q; every reader combines the 16 entries itself.
+  __shared__ __align__(16) unsigned s_wmax[MT][kGemvWarps];
+  __shared__ __align__(16) int s_wsum[MT][kGemvWarps];
   __shared__ float s_sc[MT];      // per-token dequant scale (γ_A·γ)/127
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -128,10 +150,6 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
   if (tid == 0) {
     mbar_init(s_bar, 1);
     fence_barrier_init();
-  }
-  if (tid < MT) {
-    s_max[tid] = 0u;
-    s_sum[tid] = 0;
   }
   for (int i = tid; i < M * p.rows_per_cta; i += kGemvThreads) s_part[i] = 0;
   __syncthreads();
@@ -254,14 +272,14 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
         }
       }
       const unsigned wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
-      if (lane == 0 && m < M) atomicMax(&s_max[m], wmax);
+      if (lane == 0) s_wmax[m][warp] = wmax;
     }
     __syncthreads();
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
       int tsum = 0;
       if (m < M) {
-        const float g = __uint_as_float(s_max[m]);  // γ_A (or γ_r)
+        const float g = __uint_as_float(warp_slots_max(s_wmax[m]));  // γ_A (or γ_r)
         const float s = __fdiv_rn(127.0f, __fadd_rn(g, p.eps));
         const uint4* src = row_ptr(m);
         auto emit = [&](const uint4& u, int64_t v) {
@@ -285,13 +303,15 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
         }
         for (int64_t v = tid + (int64_t)RV * kGemvThreads; v < nvec; v += kGemvThreads)
           emit(__ldg(src + v), v);
-        if (tid == 0) {
+        // The last thread has no token vector when K/VEC < 512: it makes the
+        // scale while the others quantise.
+        if (tid == kGemvThreads - 1) {
           s_sc[m] = __fdiv_rn(__fmul_rn(g, gamma_w), 127.0f);  // (γ_A·γ)/127
           if (p.gamma_out != nullptr && blockIdx.x == 0) p.gamma_out[m] = g;
         }
       }
       const int wsum = __reduce_add_sync(0xffffffffu, tsum);
-      if (lane == 0 && m < M) atomicAdd(&s_sum[m], wsum);
+      if (lane == 0) s_wsum[m][warp] = wsum;
     }
   } else {  // kSrcInt8
     const int8_t* A = reinterpret_cast<const int8_t*>(p.A);
@@ -308,13 +328,13 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
           tsum = dp4a(u.z, 0x01010101u, tsum);
           tsum = dp4a(u.w, 0x01010101u, tsum);
         }
-        if (tid == 0) {
+        if (tid == kGemvThreads - 1) {
           const float g = p.a_scale != nullptr ? p.a_scale[m] : 0.0f;
           s_sc[m] = __fdiv_rn(__fmul_rn(g, gamma_w), 127.0f);
         }
       }
       const int wsum = __reduce_add_sync(0xffffffffu, tsum);
-      if (lane == 0 && m < M) atomicAdd(&s_sum[m], wsum);
+      if (lane == 0) s_wsum[m][warp] = wsum;
     }
   }
   __syncthreads();
@@ -379,7 +399,7 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
   // 6. Epilogue: undo the code offset, scale.
   for (int e = tid; e < M * R; e += kGemvThreads) {
     const int m = e / R, r = e - m * R;
-    const int v = s_part[m * R + r] - s_sum[m];
+    const int v = s_part[m * R + r] - warp_slots_sum(s_wsum[m]);
     const int64_t o = (int64_t)m * p.N + r0 + r;
     if constexpr (OUT == kOutRawI32) {
       reinterpret_cast<int32_t*>(p.Y)[o] = v;

@@ -275,6 +275,9 @@ skinny_ternary_kernel(const __grid_constant__ CUtensorMap tm_w,
   //    undo the code offset (Σ A_q), scale, store. Fragment c0, c1: token
   //    16m+g, weight rows 8·tile+2t, +1; c2, c3: token 16m+g+8.
   const int Rv = (int)min((int64_t)p.rows_per_cta, p.N - r0);  // rows stored by this CTA
+  // Rows 8·tile+2t, +1 are adjacent outputs; with N and r0 even their offset
+  // is even, so the pair is one aligned vector store.
+  const bool pair_ok = ((p.N | r0) & 1) == 0;
   constexpr int kSlots = NG * NTW * MTT * 32;
   for (int sl = tid; sl < kSlots; sl += kSkThreads) {
     const int ln = sl & 31, m = (sl >> 5) % MTT, tile = (sl >> 5) / MTT;  // tile = ng·NTW + j
@@ -289,26 +292,50 @@ skinny_ternary_kernel(const __grid_constant__ CUtensorMap tm_w,
       v.w += u.w;
     }
     const int gg = ln >> 2, tt = ln & 3;
-    const int row = tile * 8 + 2 * tt;
+    const int row = tile * 8 + 2 * tt;  // even
     const int vals[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int tok = 16 * m + gg + ((e >> 1) << 3), rr = row + (e & 1);
-      if (tok >= M || rr >= Rv) continue;
-      const int acc_v = vals[e] - s_rs[tok];
-      const int64_t o = (int64_t)tok * p.N + r0 + rr;
+    for (int h = 0; h < 2; ++h) {  // token 16m+g, then 16m+g+8
+      const int tok = 16 * m + gg + 8 * h;
+      if (tok >= M || row >= Rv) continue;
+      const int rs = s_rs[tok];
+      const int a0 = vals[2 * h] - rs, a1 = vals[2 * h + 1] - rs;
+      const bool two = row + 1 < Rv;
+      const int64_t o = (int64_t)tok * p.N + r0 + row;
       if (p.raw) {
-        reinterpret_cast<int32_t*>(p.Y)[o] = acc_v;
-      } else {
-        float y = __fmul_rn((float)acc_v, s_sc[tok]);
-        if (p.relu2) {
-          y = fmaxf(y, 0.0f);
-          y = __fmul_rn(y, y);
+        int32_t* y = reinterpret_cast<int32_t*>(p.Y) + o;
+        if (two && pair_ok) {
+          *reinterpret_cast<int2*>(y) = make_int2(a0, a1);
+        } else {
+          y[0] = a0;
+          if (two) y[1] = a1;
         }
-        if (p.y_bf16)
-          reinterpret_cast<__nv_bfloat16*>(p.Y)[o] = __float2bfloat16_rn(y);
-        else
-          reinterpret_cast<float*>(p.Y)[o] = y;
+      } else {
+        const float sc = s_sc[tok];
+        float y0 = __fmul_rn((float)a0, sc), y1 = __fmul_rn((float)a1, sc);
+        if (p.relu2) {
+          y0 = fmaxf(y0, 0.0f);
+          y0 = __fmul_rn(y0, y0);
+          y1 = fmaxf(y1, 0.0f);
+          y1 = __fmul_rn(y1, y1);
+        }
+        if (p.y_bf16) {
+          __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(p.Y) + o;
+          if (two && pair_ok) {
+            *reinterpret_cast<__nv_bfloat162*>(y) = __floats2bfloat162_rn(y0, y1);
+          } else {
+            y[0] = __float2bfloat16_rn(y0);
+            if (two) y[1] = __float2bfloat16_rn(y1);
+          }
+        } else {
+          float* y = reinterpret_cast<float*>(p.Y) + o;
+          if (two && pair_ok) {
+            *reinterpret_cast<float2*>(y) = make_float2(y0, y1);
+          } else {
+            y[0] = y0;
+            if (two) y[1] = y1;
+          }
+        }
       }
     }
   }
