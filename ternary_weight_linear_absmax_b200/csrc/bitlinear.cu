@@ -278,9 +278,19 @@ bl_status launch_tc_t(const CUtensorMap& ta, const CUtensorMap& tw, const CUtens
   auto* k = tc_ternary_gemm_kernel<BN, OUT>;
   constexpr size_t smem = TcConfig<BN>::kSmemBytes;
   BL_TRY(ensure_smem(k, dev, smem));
-  dim3 grid((unsigned)((p.N + 127) / 128), (unsigned)((p.M + BN - 1) / BN));
-  k<<<grid, kTcThreads, smem, st>>>(ta, tw, ty, p);
-  BL_CUDA(cudaGetLastError());
+  // Always with programmatic dependent launch: the kernel waits for the
+  // previous grid before it touches global memory.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((p.N + 127) / 128), (unsigned)((p.M + BN - 1) / BN));
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  BL_CUDA(cudaLaunchKernelEx(&cfg, k, ta, tw, ty, p));
   return BL_OK;
 }
 
@@ -326,7 +336,7 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
     if (!enc) return BL_ERR_CUDA;
     cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
     cuuint64_t strides[1] = {(cuuint64_t)N * esz};
-    cuuint32_t box[2] = {128, (cuuint32_t)bn};
+    cuuint32_t box[2] = {128, (cuuint32_t)(bn < 32 ? bn : 32)};  // stored 32 tokens at a time
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&ty, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32,
                      2, Y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,

@@ -48,8 +48,9 @@ struct TcParams {
   int64_t M, N, K;
   int relu2;
   int y_bf16;
-  int tma_store;  // 1: the epilogue stages the tile in shared memory and writes it with one
-                  //    tensor store through tm_y (needs N·element bytes % 16 == 0)
+  int tma_store;  // 1: the epilogue stages the tile in shared memory and the producer warp
+                  //    writes it with tensor stores of 32 tokens through tm_y (needs
+                  //    N·element bytes % 16 == 0)
 };
 
 template <int BN>
@@ -76,7 +77,10 @@ struct TcConfig {
   static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
                                    : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
   static constexpr int kRingBytes = kSStages * kBStage + kWStages * kWStage;
-  static constexpr int kBarBytes = (2 * kSStages + 2 * kWStages + 2 * kTStages + 3) * 8;
+  // The staged output tile is stored in chunks of 32 tokens, each with its
+  // own barrier, so the stores overlap the rest of the epilogue.
+  static constexpr int kStoreChunks = (BN + 31) / 32;
+  static constexpr int kBarBytes = (2 * kSStages + 2 * kWStages + 2 * kTStages + 2 + kStoreChunks) * 8;
   static constexpr int kParamBytes = BN * 8;
   // 1 KiB slack for aligning the dynamic buffer to 1024 bytes. At least
   // 116 KiB are requested so that only one CTA is resident per SM: every CTA
@@ -169,7 +173,7 @@ __device__ __forceinline__ void tc_epilogue_chunk(const uint32_t (&d)[CW], int c
 template <int BN, int OUT, bool RELU, bool BF16, bool STAGE>
 __device__ __forceinline__ void tc_epilogue(uint32_t t_lane, int row, int half, const float* s_sc,
                                             const int* s_rs, uint8_t* stage, const TcParams& p,
-                                            int64_t m0, int64_t n) {
+                                            int64_t m0, int64_t n, uint64_t* staged) {
   using C = TcConfig<BN>;
   // 16-column chunks, alternating between the two warps of a lane quarter.
   constexpr int CW = 16;
@@ -197,6 +201,12 @@ __device__ __forceinline__ void tc_epilogue(uint32_t t_lane, int row, int half, 
     const bool more = c0 + 2 * CW < BN;
     if (more) load(c0 + 2 * CW, nxt);  // in flight while this chunk is processed
     tc_epilogue_chunk<CW, OUT, RELU, BF16, STAGE>(cur, c0, row, s_sc, s_rs, stage, p, m0, n);
+    if constexpr (STAGE) {
+      // This thread's part of tokens [32·(c0/32), +32) is staged: make it
+      // visible to the tensor store and report it.
+      fence_proxy_async_smem();
+      mbar_arrive(&staged[c0 >> 5]);
+    }
     if (more) {
       tmem_wait_ld();
 #pragma unroll
@@ -225,8 +235,8 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
   uint64_t* afull = bars + 2 * SS + 2 * WS;         // [TS] A operand in TMEM ready
   uint64_t* aempty = afull + TS;                    // [TS] MMA done with A stage
   uint64_t* done = aempty + TS;                     // accumulator complete
-  uint64_t* staged = done + 1;                      // output tile staged (math threads)
-  uint64_t* pready = done + 2;                      // epilogue parameters in shared memory
+  uint64_t* pready = done + 1;                      // epilogue parameters in shared memory
+  uint64_t* staged = done + 2;                      // [kStoreChunks] 32 output tokens staged
   float* s_sc = reinterpret_cast<float*>(smem + C::kRingBytes + C::kBarBytes);
   int* s_rs = reinterpret_cast<int*>(s_sc + BN);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_rs + BN);
@@ -252,8 +262,8 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
       mbar_init(&aempty[t], 1);
     }
     mbar_init(done, 1);
-    mbar_init(staged, kTcMathThreads);
     mbar_init(pready, kTcMathThreads);
+    for (int i = 0; i < C::kStoreChunks; ++i) mbar_init(&staged[i], kTcMathThreads);
     *s_abort = 0;
     fence_barrier_init();
     prefetch_tensormap(&tm_act);
@@ -267,6 +277,11 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
+  // Launched with programmatic dependent launch: the set-up above overlaps
+  // the previous kernel's tail; global memory is touched only after it has
+  // completed. The next kernel may start its own set-up from here on.
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();
 
   if (warp == 0) {
     // ---------------- TMA producer (whole warp, one elected lane issues) ---
@@ -294,6 +309,20 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
         mbar_wait_for(&full[d % SS], (d / SS) & 1, 100000000ull);
       for (int d = max(0, wissued - WS); d < wissued; ++d)
         mbar_wait_for(&wfull[d % WS], (d / WS) & 1, 100000000ull);
+    }
+    // Output: store each 32-token chunk of the staged tile as soon as the
+    // math warps have written it (the tile reuses the ring, whose loads have
+    // all landed once the math warps observed `done`).
+    if (p.tma_store && lane == 0 && !*s_abort) {
+      const int esz = (OUT == kTcRawI32 || !p.y_bf16) ? 4 : 2;
+      int issued = 0;
+      for (int i = 0; i < C::kStoreChunks && m0 + 32 * i < p.M; ++i) {  // chunks past M: nothing
+        if (!mbar_wait(&staged[i], 0) || *s_abort) break;
+        tma_store_2d(&tm_y, (int32_t)n0, (int32_t)(m0 + 32 * i), smem + (size_t)i * 32 * 128 * esz);
+        bulk_commit_group();
+        ++issued;
+      }
+      if (issued) bulk_wait_group_read0();  // shared source read before the CTA may exit
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer (whole warp, one elected lane issues) -----
@@ -386,35 +415,30 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
       const uint32_t t_lane = tmem + lane_addr;
       if constexpr (OUT == kTcRawI32) {
         if (p.tma_store)
-          tc_epilogue<BN, OUT, false, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n);
+          tc_epilogue<BN, OUT, false, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, staged);
         else
-          tc_epilogue<BN, OUT, false, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n);
+          tc_epilogue<BN, OUT, false, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, staged);
       } else {
         const int sel = (p.tma_store ? 4 : 0) | (p.y_bf16 ? 2 : 0) | (p.relu2 ? 1 : 0);
         switch (sel) {
-          case 0: tc_epilogue<BN, OUT, false, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
-          case 1: tc_epilogue<BN, OUT, true, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
-          case 2: tc_epilogue<BN, OUT, false, true, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
-          case 3: tc_epilogue<BN, OUT, true, true, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
-          case 4: tc_epilogue<BN, OUT, false, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
-          case 5: tc_epilogue<BN, OUT, true, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
-          case 6: tc_epilogue<BN, OUT, false, true, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
-          default: tc_epilogue<BN, OUT, true, true, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n); break;
+          case 0: tc_epilogue<BN, OUT, false, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, staged); break;
+          case 1: tc_epilogue<BN, OUT, true, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, staged); break;
+          case 2: tc_epilogue<BN, OUT, false, true, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, staged); break;
+          case 3: tc_epilogue<BN, OUT, true, true, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, staged); break;
+          case 4: tc_epilogue<BN, OUT, false, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, staged); break;
+          case 5: tc_epilogue<BN, OUT, true, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, staged); break;
+          case 6: tc_epilogue<BN, OUT, false, true, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, staged); break;
+          default: tc_epilogue<BN, OUT, true, true, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, staged); break;
         }
       }
-      if (p.tma_store) fence_proxy_async_smem();  // staged writes -> visible to the tensor store
     }
-    // Every epilogue thread arrives (also when it skipped the epilogue), so
-    // the storing thread's bounded wait can only time out on a failed CTA.
+    // Every epilogue thread arrives on every chunk barrier exactly once: the
+    // epilogue arrives per chunk it staged; the rest (a skipped epilogue, or
+    // the second half of a 16-token tile) arrive here, so the storing
+    // thread's bounded waits can only time out on a failed CTA.
     if (p.tma_store) {
-      mbar_arrive(staged);
-      if (warp == 2 && lane == 0 && ok) {
-        if (mbar_wait(staged, 0) && !*s_abort) {
-          tma_store_2d(&tm_y, (int32_t)n0, (int32_t)m0, smem);
-          bulk_commit_group();
-          bulk_wait_group_read0();  // shared source read before the CTA may exit
-        }
-      }
+      const int first = (ok && hw * 16 < BN) ? (BN - hw * 16 + 31) / 32 : 0;
+      for (int i = first; i < C::kStoreChunks; ++i) mbar_arrive(&staged[i]);
     }
   }
 
