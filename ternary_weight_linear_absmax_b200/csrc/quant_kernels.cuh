@@ -105,7 +105,12 @@ ternary_pack_kernel(const T* __restrict__ W, int64_t nwords, double count, float
 
 // ---------------------------------------------------------------------------
 // AbsMax activation quantisation: one block per token row.
-// Writes int8 A_q, γ_A and (optionally) the row sum of A_q.
+// Writes int8 A_q, γ_A and (optionally) the row sum of A_q. The first
+// kQuantRegVecs 16-byte vectors of each thread stay in registers between the
+// max pass and the quantise pass (all of a row up to 8192 bf16 / 4096 fp32
+// values), so the row is read from memory once.
+constexpr int kQuantRegVecs = 4;
+
 template <typename T>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_acts_kernel(const T* __restrict__ A, int64_t K, float eps, int8_t* __restrict__ Aq,
@@ -122,9 +127,21 @@ quant_acts_kernel(const T* __restrict__ A, int64_t K, float eps, int8_t* __restr
   __shared__ int redi[kQuantThreads / 32];
   __shared__ float s_scale;
 
+  uint4 reg[kQuantRegVecs];
   float mx = 0.0f;
-  for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
-    uint4 u = __ldg(r4 + v);
+#pragma unroll
+  for (int r = 0; r < kQuantRegVecs; ++r) {
+    const int64_t v = threadIdx.x + (int64_t)r * kQuantThreads;
+    if (v < nvec) {
+      reg[r] = __ldg(r4 + v);
+      const T* e = reinterpret_cast<const T*>(&reg[r]);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) mx = fmaxf(mx, fabsf(to_f32<T>(e[i])));
+    }
+  }
+  for (int64_t v = threadIdx.x + (int64_t)kQuantRegVecs * kQuantThreads; v < nvec;
+       v += kQuantThreads) {
+    const uint4 u = __ldg(r4 + v);
     const T* e = reinterpret_cast<const T*>(&u);
 #pragma unroll
     for (int i = 0; i < VEC; ++i) mx = fmaxf(mx, fabsf(to_f32<T>(e[i])));
@@ -143,21 +160,30 @@ quant_acts_kernel(const T* __restrict__ A, int64_t K, float eps, int8_t* __restr
   __syncthreads();
   const float s = s_scale;
   int sum = 0;
-  for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
-    uint4 u = __ldg(r4 + v);
+  auto emit = [&](const uint4& u, int64_t v) {
     const T* e = reinterpret_cast<const T*>(&u);
-    int8_t q[VEC];
+    uint32_t w[VEC / 4];
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) {
-      q[i] = quant_i8(to_f32<T>(e[i]), s);
-      sum += q[i];
+    for (int i = 0; i < VEC / 4; ++i) {
+      w[i] = pack4_low_bytes(quant_i8_bits(to_f32<T>(e[4 * i]), s),
+                             quant_i8_bits(to_f32<T>(e[4 * i + 1]), s),
+                             quant_i8_bits(to_f32<T>(e[4 * i + 2]), s),
+                             quant_i8_bits(to_f32<T>(e[4 * i + 3]), s));
+      sum = dp4a(w[i], 0x01010101u, sum);  // Σ of the four int8 values
     }
-    if constexpr (VEC == 8) {
-      *reinterpret_cast<uint2*>(Aq + m * K + v * VEC) = *reinterpret_cast<uint2*>(q);
-    } else {
-      *reinterpret_cast<uint32_t*>(Aq + m * K + v * VEC) = *reinterpret_cast<uint32_t*>(q);
-    }
+    if constexpr (VEC == 8)
+      *reinterpret_cast<uint2*>(Aq + m * K + v * VEC) = make_uint2(w[0], w[1]);
+    else
+      *reinterpret_cast<uint32_t*>(Aq + m * K + v * VEC) = w[0];
+  };
+#pragma unroll
+  for (int r = 0; r < kQuantRegVecs; ++r) {
+    const int64_t v = threadIdx.x + (int64_t)r * kQuantThreads;
+    if (v < nvec) emit(reg[r], v);
   }
+  for (int64_t v = threadIdx.x + (int64_t)kQuantRegVecs * kQuantThreads; v < nvec;
+       v += kQuantThreads)
+    emit(__ldg(r4 + v), v);
   if (rowsum != nullptr) {
     sum = warp_sum_i(sum);
     if ((threadIdx.x & 31) == 0) redi[threadIdx.x >> 5] = sum;
