@@ -155,7 +155,12 @@ bl_status bl_linear_q(const int8_t* A_q, const float* gamma_A,
  * bl_quant_acts, bl_zero_gemm and the dequantisation of bl_linear_q in one
  * call. For M ≤ bl_gemv_max_tokens() it is a single fused GEMV launch (the
  * activation quantiser runs in the kernel prologue; no workspace needed);
- * above that, an activation-quantiser launch and a tensor-core launch.
+ * above that, an activation-quantiser launch and one contraction launch:
+ * warp-level int8 MMAs over all SMs for M ≤ 64, tensor-core (tcgen05) tiles
+ * above. The contraction launches with programmatic dependent launch; it
+ * reads no memory written by the kernel before it until that kernel has
+ * completed, except that after this call's own quantiser it streams W_packed
+ * early (the quantiser does not write it).
  *   A [M, K] fp32/bf16; W_packed [N, K/4]; gamma 1 fp32; Y [M, N] fp32/bf16.
  *   workspace ≥ bl_linear_workspace_bytes(M, K, N) (may be 0 → NULL ok).
  * bl_linear_ex adds `flags` (BL_FLAG_PDL; only honoured on the GEMV path).

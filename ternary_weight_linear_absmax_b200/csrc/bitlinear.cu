@@ -294,25 +294,16 @@ bl_status launch_tc_t(const CUtensorMap& ta, const CUtensorMap& tw, const CUtens
   return BL_OK;
 }
 
+// Token tiles of 128 or 256: the tensor-core path only sees M > 64 (fewer
+// tokens take the skinny kernel).
 template <int OUT>
 bl_status launch_tc_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tw,
                        const CUtensorMap& ty, const TcParams& p, int dev, cudaStream_t st) {
-  switch (bn) {
-    case 16: return launch_tc_t<16, OUT>(ta, tw, ty, p, dev, st);
-    case 32: return launch_tc_t<32, OUT>(ta, tw, ty, p, dev, st);
-    case 64: return launch_tc_t<64, OUT>(ta, tw, ty, p, dev, st);
-    case 128: return launch_tc_t<128, OUT>(ta, tw, ty, p, dev, st);
-    default: return launch_tc_t<256, OUT>(ta, tw, ty, p, dev, st);
-  }
+  if (bn == 128) return launch_tc_t<128, OUT>(ta, tw, ty, p, dev, st);
+  return launch_tc_t<256, OUT>(ta, tw, ty, p, dev, st);
 }
 
-int tc_pick_bn(int64_t M) {
-  if (M <= 16) return 16;
-  if (M <= 32) return 32;
-  if (M <= 64) return 64;
-  if (M <= 128) return 128;
-  return 256;
-}
+int tc_pick_bn(int64_t M) { return M <= 128 ? 128 : 256; }
 
 // acc/Y[M,N] = epilogue(A_q[M,K] · W_q[N,K]ᵀ − rowsum).
 bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,

@@ -1,5 +1,5 @@
 // Ternary × INT8 contraction on the 5th-generation tensor cores (tcgen05,
-// kind::i8) for more than a handful of tokens (prefill, small batches, FFN).
+// kind::i8) for more than 64 tokens (prefill, the FFN at larger batches).
 //
 // "BitNet b1.58 — quantização ternária, BitLinear, Zero-GEMM", section
 // "Como funciona a camada BitLinear ... (Zero-GEMM)?": acc = A_q·W_qᵀ in
@@ -7,11 +7,12 @@
 // integer arithmetic; an INT8 MMA with operands in {0,1,2} × [-127,127]
 // computes the same integers exactly.
 //
-// Orientation ("swap AB"): the MMA's M side is 128 weight rows (so small
-// token counts still fill the 128-row instruction), its N side is BN tokens.
+// Orientation ("swap AB"): the MMA's M side is 128 weight rows, its N side
+// is BN tokens.
 //  * warp 0   : TMA producer. Per 128-wide K block it loads the BN×128 int8
-//               token tile (128-byte swizzle) and the 128×32-byte packed
-//               weight tile into one shared-memory stage.
+//               token tile (128-byte swizzle); every four K blocks, a
+//               128×128-byte packed weight tile. After the main loop it
+//               writes the staged output tile with tensor stores.
 //  * warp 1   : allocates TMEM, issues tcgen05.mma (one elected thread) and
 //               commits completion to the stage barriers.
 //  * warps 2-9: expansion, then epilogue. Two warps share each TMEM lane
