@@ -81,7 +81,10 @@ struct TcConfig {
   // The staged output tile is stored in chunks of 32 tokens, each with its
   // own barrier, so the stores overlap the rest of the epilogue.
   static constexpr int kStoreChunks = (BN + 31) / 32;
-  static constexpr int kBarBytes = (2 * kSStages + 2 * kWStages + 2 * kTStages + 2 + kStoreChunks) * 8;
+  // Rounded to 16 bytes: the epilogue parameters after the barriers are read
+  // with 16-byte vector loads.
+  static constexpr int kBarBytes =
+      ((2 * kSStages + 2 * kWStages + 2 * kTStages + 2 + kStoreChunks) * 8 + 15) / 16 * 16;
   static constexpr int kParamBytes = BN * 8;
   // 1 KiB slack for aligning the dynamic buffer to 1024 bytes. At least
   // 116 KiB are requested so that only one CTA is resident per SM: every CTA
@@ -121,12 +124,21 @@ __device__ __forceinline__ void tc_epilogue_chunk(const uint32_t (&d)[CW], int c
                                                   int64_t n) {
   // Read all per-token scalars first: the stores below go to shared memory
   // too, and without this split they would order every following load.
+  // c0 is a multiple of 16: 16-byte vector loads (warp-wide broadcasts).
   float sc[CW];
   int rs[CW];
 #pragma unroll
-  for (int j = 0; j < CW; ++j) {
-    sc[j] = s_sc[c0 + j];
-    rs[j] = s_rs[c0 + j];
+  for (int j = 0; j < CW; j += 4) {
+    const float4 f = *reinterpret_cast<const float4*>(s_sc + c0 + j);
+    const int4 r = *reinterpret_cast<const int4*>(s_rs + c0 + j);
+    sc[j] = f.x;
+    sc[j + 1] = f.y;
+    sc[j + 2] = f.z;
+    sc[j + 3] = f.w;
+    rs[j] = r.x;
+    rs[j + 1] = r.y;
+    rs[j + 2] = r.z;
+    rs[j + 3] = r.w;
   }
   uint32_t bits[CW];
 #pragma unroll
