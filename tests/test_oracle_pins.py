@@ -312,6 +312,44 @@ def test_bitlinear_approximates_float_linear(orc):
     assert rel < 0.6
 
 
+def test_dequant_matches_real_identity(orc):
+    """[BLOG, Zero-GEMM section] y = Σ_k (γ·W_q)(γ_A·A_q/127). The oracle's
+    fp32 path rounds three times: γ_A·γ, ÷127, acc·sc. So it must agree with
+    the real value, computed from the integers in float64, to within
+    3·2⁻²⁴ relative."""
+    rng = np.random.default_rng(11)
+    M, N = 5, 64
+    acc = rng.integers(-(2 ** 20), 2 ** 20, size=(M, N)).astype(np.int32)
+    gA = rng.uniform(0.1, 30.0, size=M).astype(np.float32)
+    gamma = np.float32(0.0159)
+    Y = orc.dequant_f32(acc, gA, gamma)
+    exact = acc.astype(np.float64) * (gA.astype(np.float64)[:, None] * np.float64(gamma) / 127.0)
+    rel = np.abs(Y.astype(np.float64) - exact) / np.maximum(np.abs(exact), 1e-300)
+    assert rel.max() <= 3 * 2.0 ** -24
+    # the float64 dequant of the oracle is the same identity up to its own roundings
+    np.testing.assert_allclose(orc.dequant(acc, gA, gamma), exact, rtol=4 * 2.0 ** -53 * 8)
+
+
+def test_requant_gamma_is_image_of_max_accumulator(orc):
+    """ReLU² and fp32 rounding are monotone, so γ_r = max_n r equals r computed
+    from the largest accumulator: γ_r = fl(fl(max(acc,0)·s)²) with
+    s = fl(fl(γ_X·γ_up)/127). A row with no positive accumulator has γ_r = 0
+    and codes 0."""
+    rng = np.random.default_rng(12)
+    M, H = 6, 320
+    acc = rng.integers(-50000, 50000, size=(M, H)).astype(np.int32)
+    acc[2] = -np.abs(acc[2]) - 1  # no positive value
+    gX = rng.uniform(0.5, 40.0, size=M).astype(np.float32)
+    g_up = np.float32(0.0173)
+    q, g = orc.relu2_requant(acc, gX, g_up, 1e-5)
+    for m in range(M):
+        s = np.float32(np.float32(gX[m] * g_up) / np.float32(127.0))
+        h = np.float32(np.float32(max(int(acc[m].max()), 0)) * s)
+        assert g[m] == np.float32(h * h), m
+    assert g[2] == 0 and np.all(q[2] == 0)
+    assert np.all(np.abs(q.astype(np.int32)).max(axis=1)[[0, 1, 3, 4, 5]] == 127)
+
+
 def test_relu2_requant_hand_case(orc):
     """ReLU² then per-token AbsMax requant, values fixed by hand:
     h = [508, 254, 0, -254] → r = [258064, 64516, 0, 0] → γ_r = 258064;
