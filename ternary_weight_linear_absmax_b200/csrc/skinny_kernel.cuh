@@ -31,9 +31,11 @@
 //    same lines (integer sums do not depend on the order).
 //  * The 16 warps form NG n-tile groups × KS K-lanes (NG = KPS, KS = 16/KPS).
 //    Warp (ng, ks) owns n-tiles [ng·NTW, ng·NTW+NTW) for all MTT m-tiles and
-//    the KPS 32-K steps ks, ks+KS, … of each stage; KPS is a compile-time
-//    constant so the step loop unrolls and fragment loads run ahead of the
-//    mma.sync chain (a rolled loop measured ~2.7x slower). The K-lanes'
+//    the KPS consecutive 32-K steps ks·KPS … ks·KPS+KPS-1 of each stage (a
+//    pair of steps shares one 16-byte load of packed weights). KPS is a
+//    compile-time constant so the step loop unrolls and fragment loads run
+//    ahead of the mma.sync chain (a rolled loop measured ~2.7x slower). The
+//    K-lanes'
 //    partial sums are written in fragment order to shared memory
 //    (conflict-free 16-byte stores) and summed by the epilogue, which
 //    dequantises (or writes raw INT32) straight from fragment coordinates.
