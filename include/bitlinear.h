@@ -19,9 +19,13 @@
  *  * Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream) and makes no host synchronisation. Scales
  *    (γ, γ_A) are passed by device pointer for the same reason.
- *  * Pointers must be 16-byte aligned. K must be a positive multiple of 64;
+ *  * Pointers must be 16-byte aligned. K must be a positive multiple of 64
+ *    and at most BL_MAX_K (the same holds for the FFN hidden size H);
  *    M, N ≥ 0 (M == 0 or N == 0 is a no-op returning BL_OK). eps must be
  *    finite and > 0. NaN/Inf inputs are outside the contract (not checked).
+ *  * BL_MAX_K = 2^22 keeps every INT32 sum exact: |Σ_k A_q·W_q| ≤ 127·K
+ *    < 2^31, and so do the kernels' internal partial sums (the decode GEMV
+ *    keeps sums scaled by up to 64 per thread).
  *  * Errors are returned, never thrown or aborted: argument errors are found
  *    on the host before any launch (nothing is launched then); launch errors
  *    map to BL_ERR_CUDA. Device-side waits are bounded: a wait that gives up
@@ -63,6 +67,9 @@ typedef enum {
 } bl_status;
 
 typedef enum { BL_F32 = 0, BL_BF16 = 1 } bl_dtype;
+
+/* Largest K (and FFN hidden size H) any entry point accepts. */
+#define BL_MAX_K 4194304
 
 /* cudaStream_t-compatible handle (cudaStream_t is struct CUstream_st*). */
 typedef struct CUstream_st* bl_stream_t;
@@ -177,6 +184,43 @@ bl_status bl_linear_ex(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
                        bl_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Taps: the integers and scales the path decides on its way, written out
+ * besides the normal result so that each can be compared, element by element,
+ * with an independent implementation. Every pointer is a device buffer the
+ * caller owns (16-byte aligned), or NULL to skip that tap.
+ *   act_q      [M, K] int8  tokens the contraction used (AbsMax quantiser)
+ *   act_gamma  [M]    fp32  γ_A per token
+ *   act_rowsum [M]    int32 Σ_k A_q[m,k]
+ *   acc_up     [M, H] int32 FFN only: up-projection accumulators
+ *   req_q      [M, H] int8  FFN only: requantised ReLU² of the up-projection
+ *   req_gamma  [M]    fp32  FFN only: γ_r per token
+ *   req_rowsum [M]    int32 FFN only: Σ_n R_q[m,n]
+ *   cta        On the fused GEMV path (M ≤ bl_gemv_max_tokens()) every CTA
+ *              quantises the tokens for itself; the taps report the tokens
+ *              of CTA `cta` (-1 or any value past the last CTA: the last one).
+ * With more tokens the quantiser runs once in its own kernel and the taps are
+ * copies of its outputs. The taps add device-to-device copies and one branch;
+ * the computed results are those of the calls without taps. */
+typedef struct {
+  int8_t* act_q;
+  float* act_gamma;
+  int32_t* act_rowsum;
+  int32_t* acc_up;
+  int8_t* req_q;
+  float* req_gamma;
+  int32_t* req_rowsum;
+  int32_t cta;
+  int32_t reserved; /* must be 0 */
+} bl_taps;
+
+/* bl_linear_ex with taps (act_* only; the FFN taps must be NULL). */
+bl_status bl_linear_taps(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
+                         const uint8_t* W_packed, const float* gamma, int64_t N,
+                         float eps, int relu2, void* Y, bl_dtype y_dtype,
+                         void* workspace, size_t ws_bytes, unsigned flags,
+                         const bl_taps* taps, bl_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * bl_linear_noalloc — bl_linear for callers that cannot allocate device memory.
  * The pages have no counterpart: this is a deployment variant, not part of
  * the method.
@@ -194,8 +238,11 @@ bl_status bl_linear_ex(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
  *     4 MiB, e.g. M·K above about 4.1 million) are refused with
  *     BL_ERR_WORKSPACE before anything is launched; use bl_linear then.
  *   * The first call on a device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture.
+ *     that device current) and caches it together with the device's current
+ *     context; make that first call before any stream capture. A call that
+ *     finds a different context current (for example after
+ *     cudaDeviceReset) looks the address up again, so it too must not be the
+ *     first call inside a stream capture.
  *   * All calls on a device share the array, which keeps whatever the last
  *     call left in it. Nothing in it needs to start at zero (each call writes
  *     every byte it reads), but calls whose kernels overlap on the GPU (for
@@ -224,6 +271,16 @@ bl_status bl_ffn_relu2(const void* X, bl_dtype x_dtype, int64_t M, int64_t K,
                        const uint8_t* W_down, const float* gamma_down,
                        float eps, void* Y, bl_dtype y_dtype, void* workspace,
                        size_t ws_bytes, bl_stream_t stream);
+
+/* bl_ffn_relu2 with taps: act_* report the quantised block input X_q, acc_up
+ * the up-projection, req_* the requantised ReLU² tokens fed to the
+ * down-projection (see bl_taps). */
+bl_status bl_ffn_relu2_taps(const void* X, bl_dtype x_dtype, int64_t M,
+                            int64_t K, int64_t H, const uint8_t* W_up,
+                            const float* gamma_up, const uint8_t* W_down,
+                            const float* gamma_down, float eps, void* Y,
+                            bl_dtype y_dtype, void* workspace, size_t ws_bytes,
+                            const bl_taps* taps, bl_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Device error flag. Synchronises `stream`, then returns BL_ERR_TIMEOUT if

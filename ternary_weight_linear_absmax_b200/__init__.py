@@ -18,11 +18,11 @@ from __future__ import annotations
 import torch
 
 from . import _lib
-from ._lib import BL_BF16, BL_F32, BL_FLAG_PDL, BitLinearError, check, load
+from ._lib import BL_BF16, BL_F32, BL_FLAG_PDL, BitLinearError, BlTaps, check, load
 
 __all__ = [
     "bl_quant_weights", "bl_quant_acts", "bl_zero_gemm", "bl_linear_q", "bl_linear",
-    "bl_linear_noalloc", "bl_ffn_relu2", "bl_check_device_error", "bl_selftest_wait_timeout",
+    "bl_linear_noalloc", "bl_ffn_relu2", "bl_linear_taps", "bl_ffn_relu2_taps", "bl_check_device_error", "bl_selftest_wait_timeout",
     "bl_gemv_max_tokens", "workspace_bytes", "BitLinearError", "load", "BL_FLAG_PDL",
 ]
 
@@ -199,6 +199,62 @@ def bl_ffn_relu2(X, W_up, gamma_up, W_down, gamma_down, eps: float = 1e-5, *,
                          _dt(out, "out"), _ptr(workspace), _nbytes(workspace), _stream(stream)),
           "bl_ffn_relu2")
     return out
+
+
+def _taps(M, K, H, device, ffn: bool, cta: int):
+    """Allocate tap buffers (torch) and the matching bl_taps structure."""
+    t = {"act_q": torch.empty((M, K), dtype=torch.int8, device=device),
+         "act_gamma": torch.empty((M,), dtype=torch.float32, device=device),
+         "act_rowsum": torch.empty((M,), dtype=torch.int32, device=device)}
+    if ffn:
+        t.update({"acc_up": torch.empty((M, H), dtype=torch.int32, device=device),
+                  "req_q": torch.empty((M, H), dtype=torch.int8, device=device),
+                  "req_gamma": torch.empty((M,), dtype=torch.float32, device=device),
+                  "req_rowsum": torch.empty((M,), dtype=torch.int32, device=device)})
+    s = BlTaps(**{k: v.data_ptr() for k, v in t.items()}, cta=int(cta), reserved=0)
+    return t, s
+
+
+def bl_linear_taps(A, W_packed, gamma, eps: float = 1e-5, *, relu2=False,
+                   out_dtype=torch.bfloat16, pdl=False, cta: int = 0, stream=None):
+    """bl_linear that also returns the int8 tokens, γ_A and Σ A_q the
+    contraction used (for the fused GEMV path: those of CTA ``cta``; -1 =
+    the last CTA). Returns (Y, taps dict)."""
+    _cuda(A, "A")
+    _cuda(W_packed, "W_packed")
+    _cuda(gamma, "gamma")
+    M, K = A.shape
+    N = W_packed.shape[0]
+    out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    L = load()
+    ws = _ws(int(L.bl_linear_workspace_bytes(M, K, N)), A.device)
+    taps, s = _taps(M, K, 0, A.device, False, cta)
+    check(L.bl_linear_taps(A.data_ptr(), _dt(A, "A"), M, K, W_packed.data_ptr(), gamma.data_ptr(),
+                           N, float(eps), int(bool(relu2)), out.data_ptr(), _dt(out, "out"),
+                           _ptr(ws), _nbytes(ws), BL_FLAG_PDL if pdl else 0, s,
+                           _stream(stream)), "bl_linear_taps")
+    return out, taps
+
+
+def bl_ffn_relu2_taps(X, W_up, gamma_up, W_down, gamma_down, eps: float = 1e-5, *,
+                      out_dtype=torch.bfloat16, cta: int = 0, stream=None):
+    """bl_ffn_relu2 that also returns X_q, γ_X, Σ X_q, the up-projection
+    accumulators, the requantised ReLU² tokens R_q, γ_r and Σ R_q.
+    Returns (Y, taps dict)."""
+    for t, n in ((X, "X"), (W_up, "W_up"), (gamma_up, "gamma_up"), (W_down, "W_down"),
+                 (gamma_down, "gamma_down")):
+        _cuda(t, n)
+    M, K = X.shape
+    H = W_up.shape[0]
+    out = torch.empty((M, K), dtype=out_dtype, device=X.device)
+    L = load()
+    ws = _ws(int(L.bl_ffn_workspace_bytes(M, K, H)), X.device)
+    taps, s = _taps(M, K, H, X.device, True, cta)
+    check(L.bl_ffn_relu2_taps(X.data_ptr(), _dt(X, "X"), M, K, H, W_up.data_ptr(),
+                              gamma_up.data_ptr(), W_down.data_ptr(), gamma_down.data_ptr(),
+                              float(eps), out.data_ptr(), _dt(out, "out"), _ptr(ws), _nbytes(ws),
+                              s, _stream(stream)), "bl_ffn_relu2_taps")
+    return out, taps
 
 
 def bl_check_device_error(stream=None) -> int:

@@ -20,6 +20,15 @@ STATUS_NAMES = {
 BL_F32, BL_BF16 = 0, 1
 BL_FLAG_PDL = 1
 
+class BlTaps(ctypes.Structure):
+    """bl_taps of include/bitlinear.h: device pointers (0 = tap off)."""
+    _fields_ = [("act_q", ctypes.c_void_p), ("act_gamma", ctypes.c_void_p),
+                ("act_rowsum", ctypes.c_void_p), ("acc_up", ctypes.c_void_p),
+                ("req_q", ctypes.c_void_p), ("req_gamma", ctypes.c_void_p),
+                ("req_rowsum", ctypes.c_void_p), ("cta", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
 # Every symbol declared in include/bitlinear.h: name -> (restype, argtypes).
 _vp, _i64, _f32, _int, _uint, _sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_float,
                                      ctypes.c_int, ctypes.c_uint, ctypes.c_size_t)
@@ -40,11 +49,15 @@ SIGNATURES = {
                          _sz, _vp]),
     "bl_linear_ex": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _i64, _f32, _int, _vp, _int, _vp,
                             _sz, _uint, _vp]),
+    "bl_linear_taps": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _i64, _f32, _int, _vp, _int,
+                              _vp, _sz, _uint, ctypes.POINTER(BlTaps), _vp]),
     "bl_linear_noalloc": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _i64, _f32, _int, _vp, _int,
                                  _vp]),
     "bl_ffn_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_ffn_relu2": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _f32, _vp, _int,
                             _vp, _sz, _vp]),
+    "bl_ffn_relu2_taps": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _f32, _vp,
+                                 _int, _vp, _sz, ctypes.POINTER(BlTaps), _vp]),
     "bl_check_device_error": (_int, [_vp]),
     "bl_selftest_wait_timeout": (_int, [_i64, _vp]),
 }

@@ -133,9 +133,12 @@ bl_status make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_
 
 // --------------------------------------------------------------------------
 // Argument checks.
+// K (and the FFN hidden size) ≤ BL_MAX_K = 2^22: every INT32 sum stays exact
+// (127·K < 2^31), including the decode GEMV's per-thread sums scaled by up to
+// 64 (each thread covers at most K/512 of a row's weights there).
 bl_status check_k(int64_t K) {
   if (K <= 0 || K % 64 != 0) return BL_ERR_SHAPE;
-  if (K > ((int64_t)1 << 30)) return BL_ERR_SHAPE;
+  if (K > (int64_t)BL_MAX_K) return BL_ERR_SHAPE;
   return BL_OK;
 }
 bl_status check_rows(int64_t R) {
@@ -243,11 +246,14 @@ bl_status gemv_plan(int64_t N, int64_t K, int M, int sms, int* rows, int* grid, 
 }
 
 // src: kSrcFloat (a_dtype says f32/bf16), kSrcFfnRequant, kSrcInt8.
+// Taps in p (if any) report CTA p.tap_cta; a value past the last CTA (or
+// negative) means the last CTA.
 bl_status run_gemv(int src, int out, bl_dtype a_dtype, GemvParams p, bool pdl, int dev, int sms,
                    cudaStream_t st) {
   int rows, grid;
   size_t smem;
   BL_TRY(gemv_plan(p.N, p.K, p.M, sms, &rows, &grid, &smem));
+  if (p.tap_cta < 0 || p.tap_cta >= grid) p.tap_cta = grid - 1;
   p.rows_per_cta = rows;
   p.rows_pad = gemv_rows_pad(rows);
   CUtensorMap tw;
@@ -505,6 +511,34 @@ bl_status run_quant_acts(const void* A, bl_dtype dt, int64_t M, int64_t K, float
   return BL_OK;
 }
 
+// Taps: argument checks and device-to-device copies of workspace pieces.
+bl_status check_taps(const bl_taps* t, bool ffn) {
+  if (t == nullptr) return BL_OK;
+  if (t->reserved != 0) return BL_ERR_INVALID_ARG;
+  if (!ffn && (t->acc_up || t->req_q || t->req_gamma || t->req_rowsum)) return BL_ERR_INVALID_ARG;
+  const void* ptrs[] = {t->act_q, t->act_gamma, t->act_rowsum, t->acc_up,
+                        t->req_q, t->req_gamma, t->req_rowsum};
+  for (const void* q : ptrs)
+    if (q != nullptr && !aligned16(q)) return BL_ERR_ALIGN;
+  return BL_OK;
+}
+
+bl_status tap_copy(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+  if (dst == nullptr || bytes == 0) return BL_OK;
+  BL_CUDA(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st));
+  return BL_OK;
+}
+
+// Points the GEMV prologue taps of p at (q, gamma, rowsum) when all are set.
+void gemv_taps(GemvParams& p, int8_t* q, float* gamma, int32_t* rowsum, int cta) {
+  if (q != nullptr && gamma != nullptr && rowsum != nullptr) {
+    p.tap_q = q;
+    p.tap_gamma = gamma;
+    p.tap_rowsum = rowsum;
+    p.tap_cta = cta;
+  }
+}
+
 }  // namespace
 }  // namespace bl
 
@@ -712,16 +746,18 @@ size_t bl_linear_workspace_bytes(int64_t M, int64_t K, int64_t N) {
   return act_ws(M, K).total;
 }
 
-bl_status bl_linear_ex(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
-                       const uint8_t* W_packed, const float* gamma, int64_t N, float eps,
-                       int relu2, void* Y, bl_dtype y_dtype, void* workspace, size_t ws_bytes,
-                       unsigned flags, bl_stream_t stream) {
+static bl_status linear_impl(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
+                             const uint8_t* W_packed, const float* gamma, int64_t N, float eps,
+                             int relu2, void* Y, bl_dtype y_dtype, void* workspace,
+                             size_t ws_bytes, unsigned flags, const bl_taps* taps,
+                             cudaStream_t st) {
   BL_TRY(check_dtype(a_dtype));
   BL_TRY(check_dtype(y_dtype));
   BL_TRY(check_k(K));
   BL_TRY(check_rows(M));
   BL_TRY(check_rows(N));
   BL_TRY(check_eps(eps));
+  BL_TRY(check_taps(taps, false));
   if ((flags & ~(unsigned)BL_FLAG_PDL) != 0) return BL_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return BL_OK;
   BL_TRY(check_ptr(A));
@@ -735,7 +771,6 @@ bl_status bl_linear_ex(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
   }
   int dev, sms;
   BL_TRY(current_device(&dev, &sms));
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (M <= kGemvMaxTokens) {
     GemvParams p = {};
     p.A = A;
@@ -748,6 +783,7 @@ bl_status bl_linear_ex(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
     p.eps = eps;
     p.relu2 = relu2 ? 1 : 0;
     p.y_bf16 = y_dtype == BL_BF16;
+    if (taps) gemv_taps(p, taps->act_q, taps->act_gamma, taps->act_rowsum, taps->cta);
     return run_gemv(kSrcFloat, kOutDequant, a_dtype, p, (flags & BL_FLAG_PDL) != 0, dev, sms, st);
   }
   const ActWs w = act_ws(M, K);
@@ -756,8 +792,30 @@ bl_status bl_linear_ex(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
   float* gA = reinterpret_cast<float*>(base + w.gamma);
   int32_t* rs = reinterpret_cast<int32_t*>(base + w.rowsum);
   BL_TRY(run_quant_acts(A, a_dtype, M, K, eps, Aq, gA, rs, st));
-  return run_contract(Aq, W_packed, M, K, N, gamma, gA, rs, Y, kTcDequant, relu2 ? 1 : 0,
-                      y_dtype == BL_BF16, true, dev, sms, st);
+  BL_TRY(run_contract(Aq, W_packed, M, K, N, gamma, gA, rs, Y, kTcDequant, relu2 ? 1 : 0,
+                      y_dtype == BL_BF16, true, dev, sms, st));
+  if (taps) {
+    BL_TRY(tap_copy(taps->act_q, Aq, (size_t)M * K, st));
+    BL_TRY(tap_copy(taps->act_gamma, gA, (size_t)M * 4, st));
+    BL_TRY(tap_copy(taps->act_rowsum, rs, (size_t)M * 4, st));
+  }
+  return BL_OK;
+}
+
+bl_status bl_linear_ex(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
+                       const uint8_t* W_packed, const float* gamma, int64_t N, float eps,
+                       int relu2, void* Y, bl_dtype y_dtype, void* workspace, size_t ws_bytes,
+                       unsigned flags, bl_stream_t stream) {
+  return linear_impl(A, a_dtype, M, K, W_packed, gamma, N, eps, relu2, Y, y_dtype, workspace,
+                     ws_bytes, flags, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bl_status bl_linear_taps(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
+                         const uint8_t* W_packed, const float* gamma, int64_t N, float eps,
+                         int relu2, void* Y, bl_dtype y_dtype, void* workspace, size_t ws_bytes,
+                         unsigned flags, const bl_taps* taps, bl_stream_t stream) {
+  return linear_impl(A, a_dtype, M, K, W_packed, gamma, N, eps, relu2, Y, y_dtype, workspace,
+                     ws_bytes, flags, taps, reinterpret_cast<cudaStream_t>(stream));
 }
 
 bl_status bl_linear(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
@@ -770,16 +828,18 @@ bl_status bl_linear(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
 
 size_t bl_ffn_workspace_bytes(int64_t M, int64_t K, int64_t H) { return ffn_ws(M, K, H).total; }
 
-bl_status bl_ffn_relu2(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, int64_t H,
-                       const uint8_t* W_up, const float* gamma_up, const uint8_t* W_down,
-                       const float* gamma_down, float eps, void* Y, bl_dtype y_dtype,
-                       void* workspace, size_t ws_bytes, bl_stream_t stream) {
+static bl_status ffn_impl(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, int64_t H,
+                          const uint8_t* W_up, const float* gamma_up, const uint8_t* W_down,
+                          const float* gamma_down, float eps, void* Y, bl_dtype y_dtype,
+                          void* workspace, size_t ws_bytes, const bl_taps* taps,
+                          cudaStream_t st) {
   BL_TRY(check_dtype(x_dtype));
   BL_TRY(check_dtype(y_dtype));
   BL_TRY(check_k(K));
   BL_TRY(check_k(H));
   BL_TRY(check_rows(M));
   BL_TRY(check_eps(eps));
+  BL_TRY(check_taps(taps, true));
   if (M == 0) return BL_OK;
   BL_TRY(check_ptr(X));
   BL_TRY(check_ptr(W_up));
@@ -791,7 +851,6 @@ bl_status bl_ffn_relu2(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, in
   BL_TRY(check_ptr(workspace));
   int dev, sms;
   BL_TRY(current_device(&dev, &sms));
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
   int32_t* acc_up = reinterpret_cast<int32_t*>(base + w.acc_up);
   if (M <= kGemvMaxTokens) {
@@ -806,6 +865,7 @@ bl_status bl_ffn_relu2(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, in
     up.K = K;
     up.M = (int)M;
     up.eps = eps;
+    if (taps) gemv_taps(up, taps->act_q, taps->act_gamma, taps->act_rowsum, taps->cta);
     BL_TRY(run_gemv(kSrcFloat, kOutRawI32, x_dtype, up, false, dev, sms, st));
     GemvParams dn = {};
     dn.A = acc_up;
@@ -819,9 +879,12 @@ bl_status bl_ffn_relu2(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, in
     dn.M = (int)M;
     dn.eps = eps;
     dn.y_bf16 = y_dtype == BL_BF16;
+    if (taps) gemv_taps(dn, taps->req_q, taps->req_gamma, taps->req_rowsum, taps->cta);
     // The kernel before this one is the up-projection above, which does not
     // write W_down: the down-projection may stream its weights early (PDL).
-    return run_gemv(kSrcFfnRequant, kOutDequant, BL_F32, dn, true, dev, sms, st);
+    BL_TRY(run_gemv(kSrcFfnRequant, kOutDequant, BL_F32, dn, true, dev, sms, st));
+    if (taps) BL_TRY(tap_copy(taps->acc_up, acc_up, (size_t)M * H * 4, st));
+    return BL_OK;
   }
   int8_t* Xq = reinterpret_cast<int8_t*>(base + w.x.aq);
   float* gX = reinterpret_cast<float*>(base + w.x.gamma);
@@ -837,8 +900,35 @@ bl_status bl_ffn_relu2(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, in
   relu2_requant_kernel<<<(unsigned)M, kQuantThreads, 0, st>>>(acc_up, H, gX, gamma_up, eps, Rq, gR,
                                                               rsR);
   BL_CUDA(cudaGetLastError());
-  return run_contract(Rq, W_down, M, H, K, gamma_down, gR, rsR, Y, kTcDequant, 0,
-                      y_dtype == BL_BF16, true, dev, sms, st);
+  BL_TRY(run_contract(Rq, W_down, M, H, K, gamma_down, gR, rsR, Y, kTcDequant, 0,
+                      y_dtype == BL_BF16, true, dev, sms, st));
+  if (taps) {
+    BL_TRY(tap_copy(taps->act_q, Xq, (size_t)M * K, st));
+    BL_TRY(tap_copy(taps->act_gamma, gX, (size_t)M * 4, st));
+    BL_TRY(tap_copy(taps->act_rowsum, rsX, (size_t)M * 4, st));
+    BL_TRY(tap_copy(taps->acc_up, acc_up, (size_t)M * H * 4, st));
+    BL_TRY(tap_copy(taps->req_q, Rq, (size_t)M * H, st));
+    BL_TRY(tap_copy(taps->req_gamma, gR, (size_t)M * 4, st));
+    BL_TRY(tap_copy(taps->req_rowsum, rsR, (size_t)M * 4, st));
+  }
+  return BL_OK;
+}
+
+bl_status bl_ffn_relu2(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, int64_t H,
+                       const uint8_t* W_up, const float* gamma_up, const uint8_t* W_down,
+                       const float* gamma_down, float eps, void* Y, bl_dtype y_dtype,
+                       void* workspace, size_t ws_bytes, bl_stream_t stream) {
+  return ffn_impl(X, x_dtype, M, K, H, W_up, gamma_up, W_down, gamma_down, eps, Y, y_dtype,
+                  workspace, ws_bytes, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bl_status bl_ffn_relu2_taps(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, int64_t H,
+                            const uint8_t* W_up, const float* gamma_up, const uint8_t* W_down,
+                            const float* gamma_down, float eps, void* Y, bl_dtype y_dtype,
+                            void* workspace, size_t ws_bytes, const bl_taps* taps,
+                            bl_stream_t stream) {
+  return ffn_impl(X, x_dtype, M, K, H, W_up, gamma_up, W_down, gamma_down, eps, Y, y_dtype,
+                  workspace, ws_bytes, taps, reinterpret_cast<cudaStream_t>(stream));
 }
 
 bl_status bl_check_device_error(bl_stream_t stream) {
@@ -871,20 +961,48 @@ constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;  // 4 MiB per device
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
-void* g_noalloc_ptr[bl::kMaxDevices] = {};
+struct NoAllocSlot {
+  void* ptr = nullptr;
+  CUcontext ctx = nullptr;  // context current when ptr was looked up
+};
+NoAllocSlot g_noalloc[bl::kMaxDevices];
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The current driver context, through the driver entry point (the library
+// does not link libcuda directly). Null if it cannot be queried.
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static int tried = 0;
+  if (!tried) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+    tried = 1;
+  }
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
 
 // Device address of the scratch array for the current device. In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// with the device current and cached; a call that finds another context
+// current (the device was reset since) looks it up again.
 bl_status noalloc_scratch(int dev, void** out) {
   std::lock_guard<std::mutex> lk(bl::g_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  const CUcontext ctx = current_context();
+  NoAllocSlot& slot = g_noalloc[dev];
+  if (slot.ptr == nullptr || slot.ctx != ctx) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
       return BL_ERR_CUDA;
-    g_noalloc_ptr[dev] = ptr;
+    slot.ptr = ptr;
+    slot.ctx = ctx;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = slot.ptr;
   return BL_OK;
 }
 }  // namespace

@@ -56,6 +56,12 @@ struct GemvParams {
   const float* gamma;       // γ of W (1 value); may be null for raw output
   void* Y;                  // kOutDequant: float/bf16 [M,N]; kOutRawI32: int32 [M,N]
   float* gamma_out;         // optional: per-token γ_A (or γ_r) written by CTA 0
+  // Optional taps (all null = off): the int8 tokens [M,K], their per-token
+  // scale γ and Σ of the int8 tokens, as the prologue of CTA tap_cta made them.
+  int8_t* tap_q;
+  float* tap_gamma;
+  int32_t* tap_rowsum;
+  int tap_cta;
   int64_t N;
   int64_t K;
   int rows_per_cta;
@@ -200,7 +206,11 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
   __syncthreads();
   if (!s_wok) {
     // Gave up: the error flag is raised and this CTA's outputs stay
-    // untouched. The wait that gave up was the wait for its own copies.
+    // untouched. The CTA still waits for the previous grid, so that a kernel
+    // launched after this one stays ordered after it, and gives its own
+    // copies a last bounded chance to land before shared memory is released.
+    if (warp == 0) pdl_wait_prior_grid();
+    if (tid == 0) mbar_wait_for(s_bar, 0, 100000000ull);
     return;
   }
   mbar_wait(s_bar, 0);  // phase complete: acquires the copies for this thread
@@ -338,6 +348,20 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
     }
   }
   __syncthreads();
+
+  // 4. Taps: CTA tap_cta reports its int8 tokens, scales and sums.
+  if (p.tap_q != nullptr && (int)blockIdx.x == p.tap_cta) {
+    const int64_t nv = (int64_t)M * K / 16;
+    for (int64_t v = tid; v < nv; v += kGemvThreads)
+      reinterpret_cast<uint4*>(p.tap_q)[v] = reinterpret_cast<const uint4*>(s_a)[v];
+    if (tid < M) {
+      if constexpr (SRC == kSrcInt8)
+        p.tap_gamma[tid] = p.a_scale != nullptr ? p.a_scale[tid] : 0.0f;
+      else
+        p.tap_gamma[tid] = __uint_as_float(warp_slots_max(s_wmax[tid]));
+      p.tap_rowsum[tid] = warp_slots_sum(s_wsum[tid]);
+    }
+  }
 
   // 5. Contraction (mapping above). The two rows share every token load
   //    and keep 8 independent accumulators per token. Consecutive lanes take

@@ -28,6 +28,24 @@ def pytest_collection_modifyitems(config, items):
             it.add_marker(skip)
 
 
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Report the rounding-boundary exemption count of every bit-exact check."""
+    try:
+        from parity_helpers import EXEMPTIONS
+    except ImportError:  # pragma: no cover
+        return
+    if not EXEMPTIONS:
+        return
+    tr = terminalreporter
+    tot_d = sum(d for _, d, _ in EXEMPTIONS)
+    tot_n = sum(n for _, _, n in EXEMPTIONS)
+    tr.write_sep("-", f"quantiser boundary exemptions: {tot_d} of {tot_n} elements "
+                      f"in {len(EXEMPTIONS)} bit-exact checks")
+    for what, d, n in EXEMPTIONS:
+        if d:
+            tr.write_line(f"  {what}: {d} of {n}")
+
+
 def read_golden(name):
     """Parse a ``key: values`` fixture; repeated keys collect into lists."""
     out = {}

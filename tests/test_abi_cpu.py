@@ -91,3 +91,28 @@ def test_argument_errors_on_host(lib):
     assert lib.bl_linear(p, 1, 0, 512, p, p, 256, 1e-5, 0, p, 1, None, 0, None) == 0
     assert lib.bl_quant_acts(p, 1, 0, 512, 1e-5, p, p, None, None) == 0
     assert lib.bl_selftest_wait_timeout(10, None) == BL_ERR_INVALID_ARG
+
+
+def test_k_bound_and_taps_checked_on_host(lib):
+    """K (and H) above 2^22 is refused (INT32 sums could no longer be exact);
+    tap structures are validated before any launch."""
+    from ternary_weight_linear_absmax_b200._lib import BlTaps
+    keep, p = _aligned_buf()
+    BL_ERR_INVALID_ARG, BL_ERR_SHAPE, BL_ERR_ALIGN = 1, 2, 3
+    kmax = 1 << 22
+    assert lib.bl_quant_acts(p, 1, 1, kmax + 64, 1e-5, p, p, None, None) == BL_ERR_SHAPE
+    assert lib.bl_ffn_relu2(p, 1, 1, 512, kmax + 64, p, p, p, p, 1e-5, p, 1, p, 1 << 20,
+                            None) == BL_ERR_SHAPE
+    # K = 2^22 itself passes the shape check (M = 0: no-op, no device touched)
+    assert lib.bl_quant_acts(p, 1, 0, kmax, 1e-5, p, p, None, None) == 0
+    bad = BlTaps(reserved=1)
+    assert lib.bl_linear_taps(p, 1, 4, 512, p, p, 256, 1e-5, 0, p, 1, None, 0, 0, bad,
+                              None) == BL_ERR_INVALID_ARG
+    ffn_only = BlTaps(acc_up=p)
+    assert lib.bl_linear_taps(p, 1, 4, 512, p, p, 256, 1e-5, 0, p, 1, None, 0, 0, ffn_only,
+                              None) == BL_ERR_INVALID_ARG
+    misaligned = BlTaps(act_q=p + 8, act_gamma=p, act_rowsum=p)
+    assert lib.bl_linear_taps(p, 1, 4, 512, p, p, 256, 1e-5, 0, p, 1, None, 0, 0, misaligned,
+                              None) == BL_ERR_ALIGN
+    assert lib.bl_ffn_relu2_taps(p, 1, 1, 512, 640, p, p, p, p, 1e-5, p, 1, p, 1 << 20,
+                                 misaligned, None) == BL_ERR_ALIGN

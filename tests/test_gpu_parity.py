@@ -17,6 +17,8 @@ import torch
 
 import oracle
 import synth_inputs as si
+from parity_helpers import EXEMPTIONS, assert_acts_match, near_half_boundary
+from parity_helpers import assert_close as _assert_close
 
 pytestmark = pytest.mark.gpu
 
@@ -38,13 +40,6 @@ def to_dev(x: np.ndarray):
     return torch.from_numpy(np.ascontiguousarray(x)).to(DEV)
 
 
-def near_half_boundary(x: np.ndarray) -> np.ndarray:
-    """|x| within one ulp of a k + 1/2 rounding boundary (fp32)."""
-    x = np.abs(x.astype(np.float32))
-    b = np.floor(x) + np.float32(0.5)
-    return np.abs(x - b) <= np.spacing(b)
-
-
 def assert_codes_match(packed_gpu, W32, gamma_gpu, K):
     codes_ref, g_ref = oracle.quant_weights(W32, EPS)
     gg = np.float32(gamma_gpu)
@@ -54,6 +49,7 @@ def assert_codes_match(packed_gpu, W32, gamma_gpu, K):
     assert bad == 0
     diff = codes_gpu != codes_ref
     nd = int(diff.sum())
+    EXEMPTIONS.append((f"weight codes {W32.shape[0]}x{K}", nd, int(W32.size)))
     if nd:
         x = (W32[diff] / np.float32(np.float32(g_ref) + np.float32(EPS))).astype(np.float32)
         assert np.all(near_half_boundary(x)), "code mismatch away from a rounding boundary"
@@ -61,27 +57,8 @@ def assert_codes_match(packed_gpu, W32, gamma_gpu, K):
     return codes_ref, g_ref, nd
 
 
-def assert_acts_match(Aq_gpu, gA_gpu, rs_gpu, A32):
-    Aq_ref, gA_ref = oracle.quant_acts(A32, EPS)
-    np.testing.assert_array_equal(gA_gpu, gA_ref)
-    diff = Aq_gpu != Aq_ref
-    nd = int(diff.sum())
-    if nd:
-        s = (np.float32(127.0) / (gA_ref + np.float32(EPS))).astype(np.float32)
-        x = (A32 * s[:, None]).astype(np.float32)[diff]
-        assert np.all(near_half_boundary(x))
-        assert nd <= 1e-6 * A32.size
-    if rs_gpu is not None:
-        np.testing.assert_array_equal(rs_gpu, Aq_gpu.astype(np.int64).sum(axis=1))
-    return Aq_ref, gA_ref, nd
-
-
 def assert_close(got, ref, out_dtype):
-    got = np.asarray(got, np.float64)
-    if out_dtype == torch.float32:
-        np.testing.assert_allclose(got, ref, rtol=1e-3, atol=1e-5)
-    else:
-        np.testing.assert_allclose(got, ref, rtol=1e-2, atol=0.0)
+    _assert_close(got, ref, out_dtype == torch.float32)
 
 
 def random_codes(N, K, seed):
@@ -166,7 +143,8 @@ QA_CASES = [(4, 512, "f32", False), (1, 2560, "bf16", True), (16, 4096, "bf16", 
 def test_quant_acts_parity(bl, M, K, dt, outl):
     A = si.activations(M, K, seed=0, outliers=outl, dtype=dt)
     Aq, gA, rs = bl.bl_quant_acts(A.torch(DEV), EPS)
-    assert_acts_match(Aq.cpu().numpy(), gA.cpu().numpy(), rs.cpu().numpy(), A.f32)
+    assert_acts_match(Aq.cpu().numpy(), gA.cpu().numpy(), rs.cpu().numpy(), A.f32,
+                      what=f"bl_quant_acts {M}x{K} {dt}")
 
 
 def test_quant_acts_special_rows(bl):

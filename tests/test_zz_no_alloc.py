@@ -6,8 +6,9 @@ inside the library instead of a caller-provided workspace.
 
 Checked through the C ABI against the ordinary bl_linear on two calls in a
 row (the second call reuses the array the first one left behind), within the
-bf16 tolerance of the parity tests; sizes whose scratch would not fit must be
-refused before anything runs. This file is collected last on purpose.
+bf16 tolerance of the parity tests, and against the CPU oracle as well; sizes
+whose scratch would not fit must be refused before anything runs. This file
+is collected last on purpose.
 """
 import ctypes
 
@@ -35,6 +36,11 @@ def _packed(K, N, seed):
     return bl.bl_quant_weights(W, EPS)
 
 
+def _oracle_codes(K, N, seed):
+    import oracle
+    return oracle.quant_weights(si.weights(N, K, seed=seed, dtype="bf16").f32, EPS)
+
+
 def _reference(lib, A, packed, gamma, relu2):
     """Output of the existing entry point, bl_linear, with a torch workspace."""
     M, K = A.shape
@@ -59,14 +65,20 @@ def _noalloc(lib, A, packed, gamma, relu2, Y):
 
 @pytest.mark.parametrize("M,K,N", [(64, 512, 384), (300, 2560, 640), (3, 4096, 512)])
 def test_noalloc_matches_bl_linear_two_calls(lib, M, K, N):
+    import oracle
     packed, gamma = _packed(K, N, seed=M)
+    codes, g = _oracle_codes(K, N, seed=M)
     for call, relu2 in enumerate((False, True)):  # two calls in a row
-        A = si.activations(M, K, seed=10 * M + call, dtype="bf16").torch("cuda")
+        Ah = si.activations(M, K, seed=10 * M + call, dtype="bf16")
+        A = Ah.torch("cuda")
         Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
         assert _noalloc(lib, A, packed, gamma, relu2, Y) == BL_OK
         ref = _reference(lib, A, packed, gamma, relu2)
         torch.cuda.synchronize()
-        np.testing.assert_allclose(Y.float().cpu().numpy(), ref.float().cpu().numpy(),
+        got = Y.float().cpu().numpy()
+        np.testing.assert_allclose(got, ref.float().cpu().numpy(), rtol=1e-2, atol=0.0)
+        # and against the independent CPU oracle on the same inputs
+        np.testing.assert_allclose(got, oracle.bitlinear(Ah.f32, codes, g, EPS, relu2=relu2)["Y"],
                                    rtol=1e-2, atol=0.0)
     assert lib.bl_check_device_error(torch.cuda.current_stream().cuda_stream) == BL_OK
 
