@@ -45,11 +45,12 @@ METRIC = "BitLinear tokens/s; decode % of HBM roofline, prefill % of INT8 TC pea
 UNIT = "tokens/s"
 EPS = 1e-5
 DECODE = dict(M=1, K=2560, N=6912)
+DECODE_WORKLOAD = "decode GEMV: 1 token, K=2560, N=6912, bf16 in/out, 1% x20 outlier channels"
 CALLS_PER_STEP = 1000
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense ratio (B200: 4.5 PFLOP/s fp8/int8, 2.25 bf16)
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "gemv_decode_k2560_n6912.md")
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "gemv_decode_k2560_n6912.json")
 GEMV_SOURCE = os.path.join(ROOT, "ternary_weight_linear_absmax_b200", "csrc", "gemv_kernel.cuh")
 
 
@@ -113,17 +114,14 @@ def sha256_file(path):
 
 def profiled_traffic():
     """DRAM bytes per launch of the decode GEMV from the committed ncu
-    summary, or None when missing or taken on a different kernel source."""
+    summary (profiles/*.json), or None when missing or taken on a different
+    kernel source."""
     try:
-        kv = {}
         with open(PROFILE_TRAFFIC) as f:
-            for line in f:
-                if ":" in line and line.startswith("- "):
-                    k, v = line[2:].split(":", 1)
-                    kv[k.strip()] = v.strip().strip("`")
-        if kv.get("kernel_source_sha256") != sha256_file(GEMV_SOURCE):
+            d = json.load(f)
+        if d.get("kernel_source_sha256") != sha256_file(GEMV_SOURCE):
             return None
-        return float(kv["dram_bytes_per_launch"])
+        return float(d["dram_bytes_per_launch"])
     except Exception:
         return None
 
@@ -477,6 +475,83 @@ def oracle_decode_rate(seconds: float = 12.0, max_calls: int | None = None):
     return n * M / el, n, oracle.max_threads()
 
 
+# The five workloads, each timed on a bounded sample of its tokens (the
+# oracle treats tokens independently, so tokens/s scales from the sample).
+CPU_CONFIGS = [
+    # name, kind, M (full), K, N (or H), tokens timed, dtype
+    ("single_layer_4x512_256_f32", "linear", 4, 512, 256, 4, "f32"),
+    ("decode_1x2560_6912", "linear", 1, 2560, 6912, 1, "bf16"),
+    ("small_batch_16x4096_11008", "linear", 16, 4096, 11008, 2, "bf16"),
+    ("prefill_2048x4096_4096", "linear", 2048, 4096, 4096, 2, "bf16"),
+    ("ffn_4096_11008_M1", "ffn", 1, 4096, 11008, 1, "bf16"),
+    ("ffn_4096_11008_M64", "ffn", 64, 4096, 11008, 1, "bf16"),
+    ("ffn_4096_11008_M512", "ffn", 512, 4096, 11008, 1, "bf16"),
+]
+
+
+def oracle_per_config(min_seconds: float = 0.2):
+    """Wall time of the oracle on every workload, single-threaded and on all
+    host cores (OpenMP over output rows), on the same seeded inputs as the
+    GPU. Returns {name: {...}} in tokens/s."""
+    import oracle
+    cores = oracle.max_threads()
+    out, cache = {}, {}
+
+    def codes_of(N, K, seed, dt):  # the three FFN workloads share their matrices
+        if (N, K, seed, dt) not in cache:
+            cache[(N, K, seed, dt)] = oracle.quant_weights(si.weights(N, K, seed=seed, dtype=dt).f32, EPS)
+        return cache[(N, K, seed, dt)]
+
+    for name, kind, M, K, N, T, dt in CPU_CONFIGS:
+        X = si.activations(T, K, seed=0, outliers=(name != "single_layer_4x512_256_f32"),
+                           dtype=dt).f32
+        if kind == "linear":
+            codes, g = codes_of(N, K, 0, dt)
+            call = lambda: oracle.bitlinear(X, codes, g, EPS)  # noqa: E731
+        else:
+            cu, gu = codes_of(N, K, 1, dt)
+            cd, gd = codes_of(K, N, 2, dt)
+            call = lambda: oracle.ffn_relu2(X, cu, gu, cd, gd, EPS)  # noqa: E731
+        row = {"tokens_timed": T, "tokens_full": M}
+        for label, th in (("threads_1", 1), (f"threads_{cores}", cores)):
+            oracle.set_threads(th)
+            reps, t0 = 0, time.perf_counter()
+            while True:
+                call()
+                reps += 1
+                el = time.perf_counter() - t0
+                if el >= min_seconds or reps >= 50:
+                    break
+            row[label] = {"tokens_per_s": reps * T / el, "s_per_call_full": el / reps * M / T,
+                          "reps": reps}
+        oracle.set_threads(cores)
+        out[name] = row
+    return out, cores
+
+
+def lut_decode_rate(min_seconds: float = 1.0):
+    """The host table-lookup BitLinear (libbitlinear_lut_cpu.so) on the decode
+    workload, 1 thread and all cores. Returns {label: tokens/s} and the ISA."""
+    import oracle
+    from ternary_weight_linear_absmax_b200 import build as _b
+    from ternary_weight_linear_absmax_b200 import lut_cpu
+    _b.build_cpu()
+    M, K, N = DECODE["M"], DECODE["K"], DECODE["N"]
+    codes, g = oracle.quant_weights(si.weights(N, K, seed=0, dtype="bf16").f32, EPS)
+    idx = lut_cpu.index_from_packed(oracle.pack_ternary(codes), K)
+    tok = si.activations(64, K, seed=0, outliers=True, dtype="bf16").f32
+    cores = oracle.max_threads()
+    out = {}
+    for th in (1, cores):
+        lut_cpu.bitlinear_lut(tok[:1], idx, g, N, EPS, threads=th)
+        n, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < min_seconds:
+            lut_cpu.bitlinear_lut(tok[n % 64:n % 64 + 1], idx, g, N, EPS, threads=th)
+            n += 1
+        out[f"threads_{th}"] = n * M / (time.perf_counter() - t0)
+    return out, lut_cpu.ISA_NAMES[lut_cpu.best_isa()]
+
+
 def run_reference(args):
     ws, rank, local = dist_env()
     if rank != 0:
@@ -492,7 +567,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 / rate, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8xternary->int32, fp32 scales", "data": "synthetic",
-        "config": {"workload": "decode GEMV: 1 token, K=2560, N=6912, bf16 in/out",
+        "config": {"workload": DECODE_WORKLOAD,
                    "step": "one BitLinear call (1 token) of the CPU oracle"},
         "cpu_baseline": {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"{n} decode calls (1 token each) after {args.warmup} warm-up calls"},
@@ -544,6 +619,16 @@ def main(argv=None):
         rate, n, cores = oracle_decode_rate(seconds=args.cpu_seconds)
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{n} decode calls (1 token, K=2560, N=6912) in ~{args.cpu_seconds:g} s"}
+        if not args.no_extra:
+            rates, isa = lut_decode_rate()
+            cpu["lut_simd"] = {"unit": UNIT, "kind": "host table-lookup BitLinear (81 entries per "
+                                                     "4 activations), not the oracle",
+                               "isa": isa, **rates,
+                               "sample": "decode calls (1 token, K=2560, N=6912) for 1 s each"}
+            cpu["per_config"], _ = oracle_per_config()
+            cpu["per_config_sample"] = ("each workload timed for >= 0.2 s on 'tokens_timed' of its "
+                                        "tokens, 1 thread and all cores; s_per_call_full scales "
+                                        "to the workload's full token count")
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -555,7 +640,7 @@ def main(argv=None):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dec["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8 x ternary -> int32 (bf16 in/out, fp32 scales)", "data": "synthetic",
-        "config": {"workload": "decode GEMV: 1 token, K=2560, N=6912, bf16 in/out, 1% x20 outlier channels",
+        "config": {"workload": DECODE_WORKLOAD,
                    "calls_per_step": CALLS_PER_STEP, "launch": "CUDA graph, programmatic dependent launch",
                    "l2": f"no flush: rotating pool of {dec['pool']['matrices']} packed matrices "
                          f"({dec['pool']['bytes'] / 1e6:.0f} MB) > 3x L2",
