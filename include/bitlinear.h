@@ -283,6 +283,44 @@ bl_status bl_ffn_relu2_taps(const void* X, bl_dtype x_dtype, int64_t M,
                             const bl_taps* taps, bl_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Tensor-parallel FFN block: the per-rank steps of bl_ffn_relu2 when the
+ * hidden dimension H is split over g ranks. The pages give no multi-GPU
+ * design; this is the composition of the same formulas over a sharded H:
+ * rank r holds rows [h0, h1) of W_up (column-parallel up-projection) and
+ * columns [h0, h1) of W_down (row-parallel down-projection), with
+ * H_r = h1 - h0 a positive multiple of 64 (W_down_r is then the contiguous
+ * copy of bytes [h0/4, h1/4) of every packed row).
+ *   1. bl_ffn_tp_up: AbsMax quantisation of X (identical on every rank),
+ *      the shard's INT32 up-projection acc_up [M, H_r], γ_X [M], and
+ *      rmax[m] = max over the shard of r = max(h, 0)² (fp32).
+ *   2. the caller all-reduces rmax with MAX over the ranks: the result is
+ *      γ_r of the unsharded block, bit for bit (a maximum is exact).
+ *   3. bl_ffn_tp_down: requantisation of the shard's r with that γ_r and
+ *      the shard's partial down-projection acc_down [M, K_out] (INT32).
+ *   4. the caller all-reduces acc_down with SUM (INT32: exact, any order).
+ *   5. bl_dequant_i32(acc_down, γ_r, γ_down) gives the block output, equal
+ *      to bl_ffn_relu2's output bit for bit.
+ * Workspaces come from the matching *_workspace_bytes(). */
+size_t bl_ffn_tp_up_workspace_bytes(int64_t M, int64_t K);
+bl_status bl_ffn_tp_up(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, int64_t H_r,
+                       const uint8_t* W_up_r, const float* gamma_up, float eps,
+                       int32_t* acc_up, float* gamma_x, float* rmax, void* workspace,
+                       size_t ws_bytes, bl_stream_t stream);
+size_t bl_ffn_tp_down_workspace_bytes(int64_t M, int64_t H_r);
+bl_status bl_ffn_tp_down(const int32_t* acc_up, const float* gamma_x, const float* gamma_up,
+                         const float* gamma_r, int64_t M, int64_t H_r,
+                         const uint8_t* W_down_r, int64_t K_out, float eps,
+                         int32_t* acc_down, void* workspace, size_t ws_bytes,
+                         bl_stream_t stream);
+
+/* Y [M, N] = acc · ((γ_A[m]·γ)/127) in fp32 (relu2 != 0: max(Y, 0)²),
+ * stored as fp32 or bf16 (round to nearest even): BLOG, Zero-GEMM section,
+ * last paragraph, for INT32 accumulators computed elsewhere. */
+bl_status bl_dequant_i32(const int32_t* acc, const float* gamma_A, const float* gamma,
+                         int64_t M, int64_t N, int relu2, void* Y, bl_dtype y_dtype,
+                         bl_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Device error flag. Synchronises `stream`, then returns BL_ERR_TIMEOUT if
  * any kernel of this library on the current device gave up a bounded wait
  * since the last check (and clears the flag), BL_ERR_CUDA if the stream

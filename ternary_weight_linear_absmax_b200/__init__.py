@@ -22,7 +22,8 @@ from ._lib import BL_BF16, BL_F32, BL_FLAG_PDL, BitLinearError, BlTaps, check, l
 
 __all__ = [
     "bl_quant_weights", "bl_quant_acts", "bl_zero_gemm", "bl_linear_q", "bl_linear",
-    "bl_linear_noalloc", "bl_ffn_relu2", "bl_linear_taps", "bl_ffn_relu2_taps", "bl_check_device_error", "bl_selftest_wait_timeout",
+    "bl_linear_noalloc", "bl_ffn_relu2", "bl_linear_taps", "bl_ffn_relu2_taps",
+    "bl_ffn_tp_up", "bl_ffn_tp_down", "bl_dequant_i32", "bl_check_device_error", "bl_selftest_wait_timeout",
     "bl_gemv_max_tokens", "workspace_bytes", "BitLinearError", "load", "BL_FLAG_PDL",
 ]
 
@@ -255,6 +256,59 @@ def bl_ffn_relu2_taps(X, W_up, gamma_up, W_down, gamma_down, eps: float = 1e-5, 
                               float(eps), out.data_ptr(), _dt(out, "out"), _ptr(ws), _nbytes(ws),
                               s, _stream(stream)), "bl_ffn_relu2_taps")
     return out, taps
+
+
+def bl_ffn_tp_up(X, W_up_r, gamma_up, eps: float = 1e-5, *, stream=None):
+    """Tensor-parallel FFN, step 1 on this rank's shard of H: returns
+    (acc_up int32 [M, H_r], γ_X fp32 [M], rmax fp32 [M] = shard max of r)."""
+    _cuda(X, "X")
+    _cuda(W_up_r, "W_up_r")
+    _cuda(gamma_up, "gamma_up")
+    M, K = X.shape
+    H_r = W_up_r.shape[0]
+    if W_up_r.shape[1] * 4 != K:
+        raise ValueError("W_up_r must be [H_r, K/4]")
+    acc = torch.empty((M, H_r), dtype=torch.int32, device=X.device)
+    gX = torch.empty((M,), dtype=torch.float32, device=X.device)
+    rmax = torch.empty((M,), dtype=torch.float32, device=X.device)
+    L = load()
+    ws = _ws(int(L.bl_ffn_tp_up_workspace_bytes(M, K)), X.device)
+    check(L.bl_ffn_tp_up(X.data_ptr(), _dt(X, "X"), M, K, H_r, W_up_r.data_ptr(),
+                         gamma_up.data_ptr(), float(eps), acc.data_ptr(), gX.data_ptr(),
+                         rmax.data_ptr(), _ptr(ws), _nbytes(ws), _stream(stream)), "bl_ffn_tp_up")
+    return acc, gX, rmax
+
+
+def bl_ffn_tp_down(acc_up, gamma_x, gamma_up, gamma_r, W_down_r, eps: float = 1e-5, *,
+                   stream=None):
+    """Tensor-parallel FFN, step 3: requantise this shard with the all-ranks
+    γ_r and return its partial down-projection (int32 [M, K_out])."""
+    for t, n in ((acc_up, "acc_up"), (gamma_x, "gamma_x"), (gamma_up, "gamma_up"),
+                 (gamma_r, "gamma_r"), (W_down_r, "W_down_r")):
+        _cuda(t, n)
+    M, H_r = acc_up.shape
+    K_out = W_down_r.shape[0]
+    if W_down_r.shape[1] * 4 != H_r:
+        raise ValueError("W_down_r must be [K_out, H_r/4]")
+    out = torch.empty((M, K_out), dtype=torch.int32, device=acc_up.device)
+    L = load()
+    ws = _ws(int(L.bl_ffn_tp_down_workspace_bytes(M, H_r)), acc_up.device)
+    check(L.bl_ffn_tp_down(acc_up.data_ptr(), gamma_x.data_ptr(), gamma_up.data_ptr(),
+                           gamma_r.data_ptr(), M, H_r, W_down_r.data_ptr(), K_out, float(eps),
+                           out.data_ptr(), _ptr(ws), _nbytes(ws), _stream(stream)), "bl_ffn_tp_down")
+    return out
+
+
+def bl_dequant_i32(acc, gamma_A, gamma, *, relu2=False, out_dtype=torch.bfloat16, stream=None):
+    """Y = acc · ((γ_A·γ)/127) (ReLU² optional) from INT32 accumulators."""
+    for t, n in ((acc, "acc"), (gamma_A, "gamma_A"), (gamma, "gamma")):
+        _cuda(t, n)
+    M, N = acc.shape
+    out = torch.empty((M, N), dtype=out_dtype, device=acc.device)
+    check(load().bl_dequant_i32(acc.data_ptr(), gamma_A.data_ptr(), gamma.data_ptr(), M, N,
+                                int(bool(relu2)), out.data_ptr(), _dt(out, "out"),
+                                _stream(stream)), "bl_dequant_i32")
+    return out
 
 
 def bl_check_device_error(stream=None) -> int:

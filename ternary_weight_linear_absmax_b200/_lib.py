@@ -58,6 +58,13 @@ SIGNATURES = {
                             _vp, _sz, _vp]),
     "bl_ffn_relu2_taps": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _f32, _vp,
                                  _int, _vp, _sz, ctypes.POINTER(BlTaps), _vp]),
+    "bl_ffn_tp_up_workspace_bytes": (_sz, [_i64, _i64]),
+    "bl_ffn_tp_up": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _sz,
+                            _vp]),
+    "bl_ffn_tp_down_workspace_bytes": (_sz, [_i64, _i64]),
+    "bl_ffn_tp_down": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _vp, _i64, _f32, _vp, _vp, _sz,
+                              _vp]),
+    "bl_dequant_i32": (_int, [_vp, _vp, _vp, _i64, _i64, _int, _vp, _int, _vp]),
     "bl_check_device_error": (_int, [_vp]),
     "bl_selftest_wait_timeout": (_int, [_i64, _vp]),
 }

@@ -931,6 +931,130 @@ bl_status bl_ffn_relu2_taps(const void* X, bl_dtype x_dtype, int64_t M, int64_t 
                   workspace, ws_bytes, taps, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-parallel FFN steps (one rank's shard of the hidden dimension).
+
+size_t bl_ffn_tp_up_workspace_bytes(int64_t M, int64_t K) {
+  if (M <= kGemvMaxTokens) return 0;
+  return align_up((size_t)M * K) + align_up((size_t)M * 4);
+}
+
+bl_status bl_ffn_tp_up(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, int64_t H_r,
+                       const uint8_t* W_up_r, const float* gamma_up, float eps, int32_t* acc_up,
+                       float* gamma_x, float* rmax, void* workspace, size_t ws_bytes,
+                       bl_stream_t stream) {
+  BL_TRY(check_dtype(x_dtype));
+  BL_TRY(check_k(K));
+  BL_TRY(check_k(H_r));
+  BL_TRY(check_rows(M));
+  BL_TRY(check_eps(eps));
+  if (M == 0) return BL_OK;
+  BL_TRY(check_ptr(X));
+  BL_TRY(check_ptr(W_up_r));
+  if (gamma_up == nullptr) return BL_ERR_INVALID_ARG;
+  BL_TRY(check_ptr(acc_up));
+  BL_TRY(check_ptr(gamma_x));
+  BL_TRY(check_ptr(rmax));
+  const size_t need = bl_ffn_tp_up_workspace_bytes(M, K);
+  if (need > 0) {
+    if (workspace == nullptr || ws_bytes < need) return BL_ERR_WORKSPACE;
+    BL_TRY(check_ptr(workspace));
+  }
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (M <= kGemvMaxTokens) {
+    GemvParams up = {};
+    up.A = X;
+    up.W = W_up_r;
+    up.gamma = gamma_up;
+    up.Y = acc_up;
+    up.gamma_out = gamma_x;
+    up.N = H_r;
+    up.K = K;
+    up.M = (int)M;
+    up.eps = eps;
+    BL_TRY(run_gemv(kSrcFloat, kOutRawI32, x_dtype, up, false, dev, sms, st));
+  } else {
+    uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
+    int8_t* Xq = reinterpret_cast<int8_t*>(base);
+    int32_t* rs = reinterpret_cast<int32_t*>(base + align_up((size_t)M * K));
+    BL_TRY(run_quant_acts(X, x_dtype, M, K, eps, Xq, gamma_x, rs, st));
+    BL_TRY(run_contract(Xq, W_up_r, M, K, H_r, gamma_up, gamma_x, rs, acc_up, kTcRawI32, 0, 0,
+                        true, dev, sms, st));
+  }
+  relu2_rowmax_kernel<<<(unsigned)M, kQuantThreads, 0, st>>>(acc_up, H_r, gamma_x, gamma_up, rmax);
+  BL_CUDA(cudaGetLastError());
+  return BL_OK;
+}
+
+size_t bl_ffn_tp_down_workspace_bytes(int64_t M, int64_t H_r) {
+  return align_up((size_t)M * H_r) + align_up((size_t)M * 4);
+}
+
+bl_status bl_ffn_tp_down(const int32_t* acc_up, const float* gamma_x, const float* gamma_up,
+                         const float* gamma_r, int64_t M, int64_t H_r, const uint8_t* W_down_r,
+                         int64_t K_out, float eps, int32_t* acc_down, void* workspace,
+                         size_t ws_bytes, bl_stream_t stream) {
+  BL_TRY(check_k(H_r));
+  BL_TRY(check_rows(M));
+  BL_TRY(check_rows(K_out));
+  BL_TRY(check_eps(eps));
+  if (M == 0 || K_out == 0) return BL_OK;
+  BL_TRY(check_ptr(acc_up));
+  BL_TRY(check_ptr(gamma_x));
+  BL_TRY(check_ptr(gamma_r));
+  if (gamma_up == nullptr) return BL_ERR_INVALID_ARG;
+  BL_TRY(check_ptr(W_down_r));
+  BL_TRY(check_ptr(acc_down));
+  const size_t need = bl_ffn_tp_down_workspace_bytes(M, H_r);
+  if (workspace == nullptr || ws_bytes < need) return BL_ERR_WORKSPACE;
+  BL_TRY(check_ptr(workspace));
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
+  int8_t* Rq = reinterpret_cast<int8_t*>(base);
+  int32_t* rs = reinterpret_cast<int32_t*>(base + align_up((size_t)M * H_r));
+  relu2_requant_given_kernel<<<(unsigned)M, kQuantThreads, 0, st>>>(acc_up, H_r, gamma_x, gamma_up,
+                                                                    gamma_r, eps, Rq, rs);
+  BL_CUDA(cudaGetLastError());
+  if (M <= kGemvMaxTokens) {
+    GemvParams p = {};
+    p.A = Rq;
+    p.W = W_down_r;
+    p.Y = acc_down;
+    p.N = K_out;
+    p.K = H_r;
+    p.M = (int)M;
+    p.eps = 1.0f;
+    return run_gemv(kSrcInt8, kOutRawI32, BL_F32, p, false, dev, sms, st);
+  }
+  return run_contract(Rq, W_down_r, M, H_r, K_out, nullptr, nullptr, rs, acc_down, kTcRawI32, 0, 0,
+                      true, dev, sms, st);
+}
+
+bl_status bl_dequant_i32(const int32_t* acc, const float* gamma_A, const float* gamma, int64_t M,
+                         int64_t N, int relu2, void* Y, bl_dtype y_dtype, bl_stream_t stream) {
+  BL_TRY(check_dtype(y_dtype));
+  BL_TRY(check_rows(M));
+  BL_TRY(check_rows(N));
+  if (M == 0 || N == 0) return BL_OK;
+  BL_TRY(check_ptr(acc));
+  BL_TRY(check_ptr(gamma_A));
+  if (gamma == nullptr) return BL_ERR_INVALID_ARG;
+  BL_TRY(check_ptr(Y));
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  const int64_t total = M * N;
+  int64_t blocks = (total + kQuantThreads - 1) / kQuantThreads;
+  if (blocks > 16 * (int64_t)sms) blocks = 16 * (int64_t)sms;
+  dequant_i32_kernel<<<(unsigned)blocks, kQuantThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      acc, gamma_A, gamma, M, N, relu2 ? 1 : 0, Y, y_dtype == BL_BF16);
+  BL_CUDA(cudaGetLastError());
+  return BL_OK;
+}
+
 bl_status bl_check_device_error(bl_stream_t stream) {
   int dev, sms;
   BL_TRY(current_device(&dev, &sms));

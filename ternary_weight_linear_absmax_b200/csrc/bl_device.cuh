@@ -340,10 +340,6 @@ __device__ __forceinline__ uint32_t quant_i8_bits(float a, float s) {
   return __float_as_uint(__fadd_rn(v, 12582912.0f));
 }
 
-__device__ __forceinline__ int8_t quant_i8(float a, float s) {
-  return (int8_t)(quant_i8_bits(a, s) & 0xFFu);
-}
-
 // Packs the low bytes of four words into one word (byte i from word i).
 __device__ __forceinline__ uint32_t pack4_low_bytes(uint32_t b0, uint32_t b1, uint32_t b2,
                                                     uint32_t b3) {

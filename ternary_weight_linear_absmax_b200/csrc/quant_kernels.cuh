@@ -228,7 +228,64 @@ rowsum_i8_kernel(const int8_t* __restrict__ Aq, int64_t K, int32_t* __restrict__
 //   γ_r = max_n r,  q = Clip(Round(r · 127/(γ_r+ε)), -128, 127),  Σq.
 // ReLU² is monotone in acc and fp32 rounding is monotone, so γ_r is also
 // the image of the largest accumulator; computing it from r keeps the
-// kernel a literal restatement.
+// kernel a literal restatement. The two passes are also launched apart for
+// the tensor-parallel block, where γ_r is the maximum over every rank's
+// shard of H.
+
+__device__ __forceinline__ float relu2_of(int acc, float sc) {
+  const float h = __fmul_rn((float)acc, sc);
+  const float p = fmaxf(h, 0.0f);
+  return __fmul_rn(p, p);
+}
+
+// Pass 1: block-wide max of r over one token's row (returned to all threads).
+__device__ __forceinline__ float relu2_row_max(const int4* __restrict__ a4, int64_t H, float sc) {
+  __shared__ float redf[kQuantThreads / 32];
+  __shared__ float total;
+  float mx = 0.0f;
+  for (int64_t v = threadIdx.x; v < H / 4; v += blockDim.x) {
+    const int4 u = __ldg(a4 + v);
+    mx = fmaxf(fmaxf(mx, fmaxf(relu2_of(u.x, sc), relu2_of(u.y, sc))),
+               fmaxf(relu2_of(u.z, sc), relu2_of(u.w, sc)));
+  }
+  mx = warp_max(mx);
+  if ((threadIdx.x & 31) == 0) redf[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float t = threadIdx.x < kQuantThreads / 32 ? redf[threadIdx.x] : 0.0f;
+    t = warp_max(t);
+    if (threadIdx.x == 0) total = t;
+  }
+  __syncthreads();
+  return total;
+}
+
+// Pass 2: quantise one token's row of r with γ_r, write q and Σq.
+__device__ __forceinline__ void relu2_row_quant(const int4* __restrict__ a4, int64_t H, float sc,
+                                                float gamma_r, float eps, int8_t* __restrict__ q_row,
+                                                int32_t* __restrict__ rowsum) {
+  __shared__ int redi[kQuantThreads / 32];
+  const float s = __fdiv_rn(127.0f, __fadd_rn(gamma_r, eps));
+  int sum = 0;
+  for (int64_t v = threadIdx.x; v < H / 4; v += blockDim.x) {
+    const int4 u = __ldg(a4 + v);
+    const uint32_t w = pack4_low_bytes(quant_i8_bits(relu2_of(u.x, sc), s),
+                                       quant_i8_bits(relu2_of(u.y, sc), s),
+                                       quant_i8_bits(relu2_of(u.z, sc), s),
+                                       quant_i8_bits(relu2_of(u.w, sc), s));
+    sum = dp4a(w, 0x01010101u, sum);
+    *reinterpret_cast<uint32_t*>(q_row + v * 4) = w;
+  }
+  sum = warp_sum_i(sum);
+  if ((threadIdx.x & 31) == 0) redi[threadIdx.x >> 5] = sum;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    int t = threadIdx.x < kQuantThreads / 32 ? redi[threadIdx.x] : 0;
+    t = warp_sum_i(t);
+    if (threadIdx.x == 0) *rowsum = t;
+  }
+}
+
 __global__ void __launch_bounds__(kQuantThreads)
 relu2_requant_kernel(const int32_t* __restrict__ acc, int64_t H, const float* __restrict__ gammaX,
                      const float* __restrict__ g_up, float eps, int8_t* __restrict__ Rq,
@@ -237,54 +294,57 @@ relu2_requant_kernel(const int32_t* __restrict__ acc, int64_t H, const float* __
   const int64_t m = blockIdx.x;
   const int4* a4 = reinterpret_cast<const int4*>(acc + m * H);
   const float sc = __fdiv_rn(__fmul_rn(gammaX[m], *g_up), 127.0f);
-  __shared__ float redf[kQuantThreads / 32];
-  __shared__ int redi[kQuantThreads / 32];
-  __shared__ float s_scale;
-  float mx = 0.0f;
-  for (int64_t v = threadIdx.x; v < H / 4; v += blockDim.x) {
-    int4 u = __ldg(a4 + v);
-    const int e[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float h = __fmul_rn((float)e[i], sc);
-      float p = fmaxf(h, 0.0f);
-      mx = fmaxf(mx, __fmul_rn(p, p));
+  const float g = relu2_row_max(a4, H, sc);
+  if (threadIdx.x == 0) gammaR[m] = g;
+  relu2_row_quant(a4, H, sc, g, eps, Rq + m * H, rowsum + m);
+}
+
+// Tensor-parallel FFN, pass 1 on one rank's shard: rmax[m] = max_n r.
+__global__ void __launch_bounds__(kQuantThreads)
+relu2_rowmax_kernel(const int32_t* __restrict__ acc, int64_t H, const float* __restrict__ gammaX,
+                    const float* __restrict__ g_up, float* __restrict__ rmax) {
+  pdl_launch_dependents();
+  const int64_t m = blockIdx.x;
+  const float sc = __fdiv_rn(__fmul_rn(gammaX[m], *g_up), 127.0f);
+  const float g = relu2_row_max(reinterpret_cast<const int4*>(acc + m * H), H, sc);
+  if (threadIdx.x == 0) rmax[m] = g;
+}
+
+// Tensor-parallel FFN, pass 2 on one rank's shard with the all-ranks γ_r.
+__global__ void __launch_bounds__(kQuantThreads)
+relu2_requant_given_kernel(const int32_t* __restrict__ acc, int64_t H,
+                           const float* __restrict__ gammaX, const float* __restrict__ g_up,
+                           const float* __restrict__ gammaR, float eps, int8_t* __restrict__ Rq,
+                           int32_t* __restrict__ rowsum) {
+  pdl_launch_dependents();
+  const int64_t m = blockIdx.x;
+  const float sc = __fdiv_rn(__fmul_rn(gammaX[m], *g_up), 127.0f);
+  relu2_row_quant(reinterpret_cast<const int4*>(acc + m * H), H, sc, gammaR[m], eps, Rq + m * H,
+                  rowsum + m);
+}
+
+// Dequantisation of INT32 accumulators: y = acc · ((γ_A·γ)/127) in fp32
+// (optionally ReLU²), the same arithmetic as the contraction epilogues.
+// One thread per 4 outputs (N % 4 == 0 is not required; row tails handled).
+__global__ void __launch_bounds__(kQuantThreads)
+dequant_i32_kernel(const int32_t* __restrict__ acc, const float* __restrict__ gammaA,
+                   const float* __restrict__ gamma, int64_t M, int64_t N, int relu2, void* Y,
+                   int y_bf16) {
+  const float g = __ldg(gamma);
+  const int64_t total = M * N;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t m = i / N;
+    const float sc = __fdiv_rn(__fmul_rn(__ldg(gammaA + m), g), 127.0f);
+    float y = __fmul_rn((float)__ldg(acc + i), sc);
+    if (relu2) {
+      y = fmaxf(y, 0.0f);
+      y = __fmul_rn(y, y);
     }
-  }
-  mx = warp_max(mx);
-  if ((threadIdx.x & 31) == 0) redf[threadIdx.x >> 5] = mx;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float t = threadIdx.x < kQuantThreads / 32 ? redf[threadIdx.x] : 0.0f;
-    t = warp_max(t);
-    if (threadIdx.x == 0) {
-      gammaR[m] = t;
-      s_scale = __fdiv_rn(127.0f, __fadd_rn(t, eps));
-    }
-  }
-  __syncthreads();
-  const float s = s_scale;
-  int sum = 0;
-  for (int64_t v = threadIdx.x; v < H / 4; v += blockDim.x) {
-    int4 u = __ldg(a4 + v);
-    const int e[4] = {u.x, u.y, u.z, u.w};
-    int8_t q[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float h = __fmul_rn((float)e[i], sc);
-      float p = fmaxf(h, 0.0f);
-      q[i] = quant_i8(__fmul_rn(p, p), s);
-      sum += q[i];
-    }
-    *reinterpret_cast<uint32_t*>(Rq + m * H + v * 4) = *reinterpret_cast<uint32_t*>(q);
-  }
-  sum = warp_sum_i(sum);
-  if ((threadIdx.x & 31) == 0) redi[threadIdx.x >> 5] = sum;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    int t = threadIdx.x < kQuantThreads / 32 ? redi[threadIdx.x] : 0;
-    t = warp_sum_i(t);
-    if (threadIdx.x == 0) rowsum[m] = t;
+    if (y_bf16)
+      reinterpret_cast<__nv_bfloat16*>(Y)[i] = __float2bfloat16_rn(y);
+    else
+      reinterpret_cast<float*>(Y)[i] = y;
   }
 }
 
