@@ -65,6 +65,12 @@ def lib():
         L.orc_dequant_f32.argtypes = [P(ctypes.c_int32), P(ctypes.c_float), f32, i64, i64, P(ctypes.c_float)]
         L.orc_relu2_requant.argtypes = [P(ctypes.c_int32), P(ctypes.c_float), f32, i64, i64, f32,
                                         P(ctypes.c_int8), P(ctypes.c_float)]
+        L.orc_ste_grad_input.argtypes = [P(ctypes.c_float), i64, i64, P(ctypes.c_int8), i64, f32,
+                                         P(ctypes.c_double)]
+        L.orc_ste_weight_mask.argtypes = [P(ctypes.c_float), i64, i64, f32, f32, P(ctypes.c_uint8)]
+        L.orc_ste_grad_weight.argtypes = [P(ctypes.c_float), i64, i64, P(ctypes.c_int8),
+                                          P(ctypes.c_float), i64, P(ctypes.c_float), f32, f32,
+                                          P(ctypes.c_double)]
         L.orc_max_threads.restype = i32
         L.orc_set_threads.argtypes = [i32]
         _lib = L
@@ -218,3 +224,39 @@ def ffn_relu2(X, Wup, g_up, Wdown, g_down, eps):
     Y = dequant(acc_dn, gR, g_down, False)
     return {"Xq": Xq, "gammaX": gX, "acc_up": acc_up, "Rq": Rq, "gammaR": gR,
             "acc_down": acc_dn, "Y": Y}
+
+
+def ste_grad_input(dY, Wq, gamma):
+    """STE backward, activation gradient: dA = dY·Ŵ with Ŵ = γ·W_q (float64)."""
+    dY, Wq = _f32(dY), _i8(Wq)
+    M, N = dY.shape
+    K = Wq.shape[1]
+    assert Wq.shape[0] == N
+    dA = np.empty((M, K), np.float64)
+    lib().orc_ste_grad_input(_p(dY, ctypes.c_float), M, N, _p(Wq, ctypes.c_int8), K,
+                             float(np.float32(gamma)), _p(dA, ctypes.c_double))
+    return dA
+
+
+def ste_weight_mask(W, gamma, eps):
+    """1 where -1 <= fp32(W / (γ+ε)) <= 1 (the clip was not active)."""
+    W = _f32(W)
+    N, K = W.shape
+    mask = np.empty((N, K), np.uint8)
+    lib().orc_ste_weight_mask(_p(W, ctypes.c_float), N, K, float(np.float32(gamma)),
+                              float(np.float32(eps)), _p(mask, ctypes.c_uint8))
+    return mask
+
+
+def ste_grad_weight(dY, Aq, gammaA, W, gamma, eps):
+    """STE backward, weight gradient: dW = mask ⊙ (dYᵀ·Â), Â = (γ_A/127)·A_q."""
+    dY, Aq, gA, W = _f32(dY), _i8(Aq), _f32(gammaA), _f32(W)
+    M, N = dY.shape
+    K = Aq.shape[1]
+    assert W.shape == (N, K) and gA.shape == (M,)
+    dW = np.empty((N, K), np.float64)
+    lib().orc_ste_grad_weight(_p(dY, ctypes.c_float), M, N, _p(Aq, ctypes.c_int8),
+                              _p(gA, ctypes.c_float), K, _p(W, ctypes.c_float),
+                              float(np.float32(gamma)), float(np.float32(eps)),
+                              _p(dW, ctypes.c_double))
+    return dW

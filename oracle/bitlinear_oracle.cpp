@@ -334,4 +334,65 @@ void orc_ffn_relu2(const float* X, int64_t M, int64_t K, int64_t H,
   orc_dequant(acc_down, gammaR, g_down, M, Nout, 0, Y);
 }
 
+// ---------------------------------------------------------------------------
+// [BLOG] §Zero-GEMM, paragraph after the worked example: training uses the
+// Straight-Through Estimator; in the backward pass the gradient of the
+// quantisation is taken as the identity (∂W_q ÷ ∂W = 1) for values inside
+// the valid range. Reading (the page states no more): the forward is
+// Y = Â·Ŵᵀ with Ŵ = γ·W_q and Â = (γ_A ÷ 127)·A_q; the backward passes the
+// output gradient dY through both quantisers as if they were the identity,
+// except that the weight gradient is zero where the Clip of W ÷ (γ+ε) to
+// [-1, 1] was active. Sums in double.
+//   dA[m,k] = Σ_n dY[m,n]·Ŵ[n,k] = γ·(Σ_{W_q=+1} dY[m,n] − Σ_{W_q=−1} dY[m,n])
+//   dW[n,k] = 1[−1 ≤ W ÷ (γ+ε) ≤ 1] · Σ_m dY[m,n]·Â[m,k]
+// The range test uses the same fp32 quotient the forward rounds.
+void orc_ste_grad_input(const float* dY, int64_t M, int64_t N, const int8_t* Wq,
+                        int64_t K, float gamma, double* dA) {
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t k = 0; k < K; ++k) {
+      double s = 0.0;
+      for (int64_t n = 0; n < N; ++n) {
+        const int8_t w = Wq[n * K + k];
+        if (w == 1) {
+          s += (double)dY[m * N + n];
+        } else if (w == -1) {
+          s -= (double)dY[m * N + n];
+        }
+      }
+      dA[m * K + k] = (double)gamma * s;
+    }
+  }
+}
+
+// 1 where the forward's Clip(W ÷ (γ+ε), -1, 1) left the quotient unchanged.
+void orc_ste_weight_mask(const float* W, int64_t N, int64_t K, float gamma,
+                         float eps, uint8_t* mask) {
+  const float g = gamma + eps;  // fp32 add, as in the forward
+  for (int64_t i = 0; i < N * K; ++i) {
+    const float x = W[i] / g;  // fp32 division, as in the forward
+    mask[i] = (x >= -1.0f && x <= 1.0f) ? 1 : 0;
+  }
+}
+
+void orc_ste_grad_weight(const float* dY, int64_t M, int64_t N, const int8_t* Aq,
+                         const float* gammaA, int64_t K, const float* W,
+                         float gamma, float eps, double* dW) {
+  std::vector<uint8_t> mask((size_t)N * K);
+  orc_ste_weight_mask(W, N, K, gamma, eps, mask.data());
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t k = 0; k < K; ++k) {
+      double s = 0.0;
+      if (mask[n * K + k]) {
+        for (int64_t m = 0; m < M; ++m) {
+          const double a_hat = (double)gammaA[m] / 127.0 * (double)Aq[m * K + k];
+          s += (double)dY[m * N + n] * a_hat;
+        }
+      }
+      dW[n * K + k] = s;
+    }
+  }
+}
+
 }  // extern "C"

@@ -379,3 +379,89 @@ def test_ffn_exact_special_case_equals_float_ffn(orc):
     ref = (np.maximum(h, 0) ** 2) @ Wdn.astype(np.float64).T
     np.testing.assert_array_equal(out["Y"], ref)
     assert set(np.unique(out["Rq"])) <= {0, 127}
+
+
+# ---------------------------------------------------------------------------
+# STE backward ([BLOG] §Zero-GEMM, Straight-Through Estimator paragraph)
+
+def _ste_problem(orc, M=5, N=7, K=48, seed=11):
+    W = si.weights(N, K, seed=seed).f32
+    codes, g = orc.quant_weights(W, 1e-5)
+    A = si.activations(M, K, seed=seed + 1, outliers=True).f32
+    Aq, gA = orc.quant_acts(A, 1e-5)
+    dY = si.activations(M, N, seed=seed + 2).f32
+    return W, codes, g, A, Aq, gA, dY
+
+
+def test_ste_grad_input_bilinear_identity(orc):
+    """⟨dA, Â⟩ = ⟨dY, Y⟩: the activation gradient is the adjoint of the
+    forward (Y from the forward oracle, Â = γ_A·A_q/127). A transposed
+    operand, a dropped γ or a sign error breaks the equality."""
+    W, codes, g, A, Aq, gA, dY = _ste_problem(orc)
+    dA = orc.ste_grad_input(dY, codes, g)
+    A_hat = gA.astype(np.float64)[:, None] / 127.0 * Aq
+    Y = orc.bitlinear(A, codes, g, 1e-5)["Y"]
+    lhs, rhs = float((dA * A_hat).sum()), float((dY.astype(np.float64) * Y).sum())
+    assert abs(lhs - rhs) <= 1e-12 * (abs(rhs) + 1.0)
+
+
+def test_ste_grad_weight_bilinear_identity(orc):
+    """⟨dW, Ŵ⊙mask⟩ = ⟨dY, Y'⟩ with Y' the forward of the masked codes:
+    the weight gradient is the adjoint of the forward within the clip range."""
+    W, codes, g, A, Aq, gA, dY = _ste_problem(orc, seed=21)
+    mask = orc.ste_weight_mask(W, g, 1e-5)
+    assert 0 < mask.mean() < 1  # some weights were clipped, some not
+    dW = orc.ste_grad_weight(dY, Aq, gA, W, g, 1e-5)
+    assert np.all(dW[mask == 0] == 0.0)
+    W_hat = float(g) * (codes * mask).astype(np.float64)
+    Yp = orc.dequant(orc.zero_gemm(Aq, (codes * mask).astype(np.int8)), gA, g)
+    lhs, rhs = float((dW * W_hat).sum()), float((dY.astype(np.float64) * Yp).sum())
+    assert abs(lhs - rhs) <= 1e-12 * (abs(rhs) + 1.0)
+
+
+def test_ste_identity_weights_pass_dY(orc):
+    """W = c·I (N = K): the codes are the identity (the diagonal clips to 1,
+    the rest rounds to 0) and γ = c/K, so dA = γ·dY exactly."""
+    K = 64
+    W = np.eye(K, dtype=np.float32) * np.float32(0.5)
+    codes, g = orc.quant_weights(W, 1e-5)
+    np.testing.assert_array_equal(codes, np.eye(K, dtype=np.int8))
+    assert g == np.float32(0.5 / K)
+    dY = si.activations(3, K, seed=4).f32
+    np.testing.assert_array_equal(orc.ste_grad_input(dY, codes, g),
+                                  dY.astype(np.float64) * np.float64(g))
+
+
+def test_ste_mask_boundary_ulps(orc):
+    """The range test is the forward's fp32 quotient: W = γ+ε gives exactly 1
+    (inside), the next float above gives a quotient above 1 (outside), for
+    either sign; values between are inside."""
+    W = si.weights(4, 64, seed=9).f32.copy()
+    g = orc.absmean_gamma(W)
+    for _ in range(20):  # crafted entries barely move γ; iterate to a fixed point
+        gg = np.float32(np.float32(g) + np.float32(1e-5))
+        W[0, :4] = [gg, -gg, np.nextafter(gg, np.float32(np.inf)),
+                    -np.nextafter(gg, np.float32(np.inf))]
+        W[0, 4] = np.nextafter(gg, np.float32(0))
+        g_new = orc.absmean_gamma(W)
+        if g_new == g:
+            break
+        g = g_new
+    assert np.float32(np.float32(g) + np.float32(1e-5)) == W[0, 0]
+    mask = orc.ste_weight_mask(W, g, 1e-5)
+    np.testing.assert_array_equal(mask[0, :5], [1, 1, 0, 0, 1])
+    x = W[0, :5] / (np.float32(g) + np.float32(1e-5))
+    assert x[0] == 1.0 and x[1] == -1.0 and x[2] > 1.0 and x[3] < -1.0
+
+
+def test_ste_grads_match_float64_matmul(orc):
+    """Special case reducing to library routines: dA = γ·(dY @ W_q) and
+    dW = mask ⊙ (dYᵀ @ Â) in float64."""
+    W, codes, g, A, Aq, gA, dY = _ste_problem(orc, M=9, N=13, K=64, seed=31)
+    dA = orc.ste_grad_input(dY, codes, g)
+    np.testing.assert_allclose(dA, float(g) * (dY.astype(np.float64) @ codes.astype(np.float64)),
+                               rtol=1e-12, atol=1e-12)
+    A_hat = gA.astype(np.float64)[:, None] / 127.0 * Aq
+    mask = orc.ste_weight_mask(W, g, 1e-5)
+    dW = orc.ste_grad_weight(dY, Aq, gA, W, g, 1e-5)
+    np.testing.assert_allclose(dW, mask * (dY.astype(np.float64).T @ A_hat), rtol=1e-12, atol=1e-12)
