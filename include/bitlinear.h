@@ -321,6 +321,31 @@ bl_status bl_dequant_i32(const int32_t* acc, const float* gamma_A, const float* 
                          bl_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * STE backward (training). BLOG, Zero-GEMM section, paragraph after the
+ * worked example: the gradient of the quantisation is taken as the identity
+ * (∂W_q/∂W = 1) inside the valid range. With the forward Y = Â·Ŵᵀ,
+ * Ŵ = γ·W_q and Â = (γ_A/127)·A_q:
+ *   bl_ste_grad_input:  dA [M, K] = dY·Ŵ = γ·(dY·W_q)
+ *   bl_ste_grad_weight: dW [N, K] = mask ⊙ (dYᵀ·Â), mask = 1 where the
+ *                       forward's fp32 quotient W ÷ (γ+ε) lies in [-1, 1]
+ *                       (W: the latent fp32/bf16 weights, [N, K]).
+ * Arguments: dY [M, N] fp32 or bf16 (N a multiple of 8); W_packed, γ as for
+ * bl_linear; A_q [M, K] int8 and γ_A [M] as bl_quant_acts returns them;
+ * outputs fp32. Both contractions run on the tensor cores in bf16 with fp32
+ * accumulation: dY (if fp32) and Â are rounded to bf16 once (W_q is exact),
+ * so each output is within about 2^-7 of Σ|terms| of the exact value.
+ * Workspaces (caller-owned) from the matching *_workspace_bytes(). */
+size_t bl_ste_grad_input_workspace_bytes(int64_t M, int64_t N, int64_t K);
+bl_status bl_ste_grad_input(const void* dY, bl_dtype dy_dtype, int64_t M, int64_t N,
+                            const uint8_t* W_packed, const float* gamma, int64_t K,
+                            float* dA, void* workspace, size_t ws_bytes, bl_stream_t stream);
+size_t bl_ste_grad_weight_workspace_bytes(int64_t M, int64_t N, int64_t K);
+bl_status bl_ste_grad_weight(const void* dY, bl_dtype dy_dtype, int64_t M, int64_t N,
+                             const int8_t* A_q, const float* gamma_A, int64_t K,
+                             const void* W, bl_dtype w_dtype, const float* gamma, float eps,
+                             float* dW, void* workspace, size_t ws_bytes, bl_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Device error flag. Synchronises `stream`, then returns BL_ERR_TIMEOUT if
  * any kernel of this library on the current device gave up a bounded wait
  * since the last check (and clears the flag), BL_ERR_CUDA if the stream

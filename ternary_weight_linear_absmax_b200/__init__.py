@@ -23,7 +23,7 @@ from ._lib import BL_BF16, BL_F32, BL_FLAG_PDL, BitLinearError, BlTaps, check, l
 __all__ = [
     "bl_quant_weights", "bl_quant_acts", "bl_zero_gemm", "bl_linear_q", "bl_linear",
     "bl_linear_noalloc", "bl_ffn_relu2", "bl_linear_taps", "bl_ffn_relu2_taps",
-    "bl_ffn_tp_up", "bl_ffn_tp_down", "bl_dequant_i32", "bl_check_device_error", "bl_selftest_wait_timeout",
+    "bl_ffn_tp_up", "bl_ffn_tp_down", "bl_dequant_i32", "bl_ste_grad_input", "bl_ste_grad_weight", "bl_check_device_error", "bl_selftest_wait_timeout",
     "bl_gemv_max_tokens", "workspace_bytes", "BitLinearError", "load", "BL_FLAG_PDL",
 ]
 
@@ -309,6 +309,43 @@ def bl_dequant_i32(acc, gamma_A, gamma, *, relu2=False, out_dtype=torch.bfloat16
                                 int(bool(relu2)), out.data_ptr(), _dt(out, "out"),
                                 _stream(stream)), "bl_dequant_i32")
     return out
+
+
+def bl_ste_grad_input(dY, W_packed, gamma, *, stream=None):
+    """STE backward, activation gradient dA [M, K] = γ·(dY·W_q) (fp32)."""
+    _cuda(dY, "dY")
+    _cuda(W_packed, "W_packed")
+    _cuda(gamma, "gamma")
+    M, N = dY.shape
+    if W_packed.shape[0] != N:
+        raise ValueError("W_packed must be [N, K/4] with N = dY.shape[1]")
+    K = W_packed.shape[1] * 4
+    dA = torch.empty((M, K), dtype=torch.float32, device=dY.device)
+    L = load()
+    ws = _ws(int(L.bl_ste_grad_input_workspace_bytes(M, N, K)), dY.device)
+    check(L.bl_ste_grad_input(dY.data_ptr(), _dt(dY, "dY"), M, N, W_packed.data_ptr(),
+                              gamma.data_ptr(), K, dA.data_ptr(), _ptr(ws), _nbytes(ws),
+                              _stream(stream)), "bl_ste_grad_input")
+    return dA
+
+
+def bl_ste_grad_weight(dY, A_q, gamma_A, W, gamma, eps: float = 1e-5, *, stream=None):
+    """STE backward, weight gradient dW [N, K] = mask ⊙ (dYᵀ·Â) (fp32); W are
+    the latent weights [N, K] whose clip range makes the mask."""
+    for t, n in ((dY, "dY"), (A_q, "A_q"), (gamma_A, "gamma_A"), (W, "W"), (gamma, "gamma")):
+        _cuda(t, n)
+    M, N = dY.shape
+    K = A_q.shape[1]
+    if A_q.shape[0] != M or tuple(W.shape) != (N, K):
+        raise ValueError("A_q must be [M, K] and W [N, K]")
+    dW = torch.empty((N, K), dtype=torch.float32, device=dY.device)
+    L = load()
+    ws = _ws(int(L.bl_ste_grad_weight_workspace_bytes(M, N, K)), dY.device)
+    check(L.bl_ste_grad_weight(dY.data_ptr(), _dt(dY, "dY"), M, N, A_q.data_ptr(),
+                               gamma_A.data_ptr(), K, W.data_ptr(), _dt(W, "W"), gamma.data_ptr(),
+                               float(eps), dW.data_ptr(), _ptr(ws), _nbytes(ws), _stream(stream)),
+          "bl_ste_grad_weight")
+    return dW
 
 
 def bl_check_device_error(stream=None) -> int:

@@ -13,6 +13,7 @@
 #include "gemv_kernel.cuh"
 #include "quant_kernels.cuh"
 #include "skinny_kernel.cuh"
+#include "ste_kernels.cuh"
 #include "tc_gemm_kernel.cuh"
 
 namespace bl {
@@ -510,6 +511,54 @@ bl_status run_quant_acts(const void* A, bl_dtype dt, int64_t M, int64_t K, float
   BL_CUDA(cudaGetLastError());
   return BL_OK;
 }
+
+// --------------------------------------------------------------------------
+// STE backward: bf16 GEMM launches and layouts.
+
+// 2-D bf16 tensor [rows, cols] with row stride ld elements (ld·2 a multiple
+// of 16 bytes), 64 × box_rows boxes, 128-byte swizzle.
+bl_status make_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                        uint64_t ld, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return BL_ERR_CUDA;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kGmBK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? BL_OK : BL_ERR_CUDA;
+}
+
+template <int BN, bool MASK>
+bl_status launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const GmParams& p, int dev,
+                        cudaStream_t st) {
+  auto* k = bf16_gemm_kernel<BN, MASK>;
+  constexpr size_t smem = GmConfig<BN>::kSmem;
+  BL_TRY(ensure_smem(k, dev, smem));
+  const dim3 grid((unsigned)((p.rows + kGmBM - 1) / kGmBM), (unsigned)((p.cols + BN - 1) / BN));
+  k<<<grid, kGmThreads, smem, st>>>(ta, tb, p);
+  BL_CUDA(cudaGetLastError());
+  return BL_OK;
+}
+
+// C[rows, cols] (fp32) = epilogue(A[rows, kdim] · B[cols, kdim]ᵀ); A, B bf16
+// with row strides lda, ldb elements.
+bl_status run_bf16_gemm(const void* A, int64_t lda, const void* B, int64_t ldb, GmParams p,
+                        int dev, cudaStream_t st) {
+  if (p.rows > (int64_t)65535 * kGmBM) return BL_ERR_SHAPE;
+  const bool wide = p.cols >= 256;
+  CUtensorMap ta, tb;
+  BL_TRY(make_map_bf16(&ta, A, (uint64_t)p.rows, (uint64_t)p.kdim, (uint64_t)lda, kGmBM));
+  BL_TRY(make_map_bf16(&tb, B, (uint64_t)p.cols, (uint64_t)p.kdim, (uint64_t)ldb, wide ? 256 : 128));
+  const bool mask = p.mask_w != nullptr;
+  if (wide)
+    return mask ? launch_gemm_t<256, true>(ta, tb, p, dev, st) : launch_gemm_t<256, false>(ta, tb, p, dev, st);
+  return mask ? launch_gemm_t<128, true>(ta, tb, p, dev, st) : launch_gemm_t<128, false>(ta, tb, p, dev, st);
+}
+
+inline int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
 
 // Taps: argument checks and device-to-device copies of workspace pieces.
 bl_status check_taps(const bl_taps* t, bool ffn) {
@@ -1053,6 +1102,121 @@ bl_status bl_dequant_i32(const int32_t* acc, const float* gamma_A, const float* 
       acc, gamma_A, gamma, M, N, relu2 ? 1 : 0, Y, y_dtype == BL_BF16);
   BL_CUDA(cudaGetLastError());
   return BL_OK;
+}
+
+// ---------------------------------------------------------------------------
+// STE backward.
+
+size_t bl_ste_grad_input_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  // W_qᵀ [K, N8] bf16, plus a bf16 copy of dY [M, N] when it is fp32
+  return align_up((size_t)K * round8(N) * 2) + align_up((size_t)M * N * 2);
+}
+
+bl_status bl_ste_grad_input(const void* dY, bl_dtype dy_dtype, int64_t M, int64_t N,
+                            const uint8_t* W_packed, const float* gamma, int64_t K, float* dA,
+                            void* workspace, size_t ws_bytes, bl_stream_t stream) {
+  BL_TRY(check_dtype(dy_dtype));
+  BL_TRY(check_k(K));
+  BL_TRY(check_rows(M));
+  BL_TRY(check_rows(N));
+  if (N % 8 != 0) return BL_ERR_SHAPE;
+  if (M == 0) return BL_OK;
+  if (N == 0) return BL_ERR_SHAPE;
+  BL_TRY(check_ptr(dY));
+  BL_TRY(check_ptr(W_packed));
+  if (gamma == nullptr) return BL_ERR_INVALID_ARG;
+  BL_TRY(check_ptr(dA));
+  if (workspace == nullptr || ws_bytes < bl_ste_grad_input_workspace_bytes(M, N, K))
+    return BL_ERR_WORKSPACE;
+  BL_TRY(check_ptr(workspace));
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
+  __nv_bfloat16* wqt = reinterpret_cast<__nv_bfloat16*>(base);
+  const int64_t Np = round8(N);
+  expand_wqt_kernel<<<dim3((unsigned)((Np + 31) / 32), (unsigned)((K + 31) / 32)), 256, 0, st>>>(
+      W_packed, N, K, Np, wqt);
+  BL_CUDA(cudaGetLastError());
+  const void* a = dY;
+  if (dy_dtype == BL_F32) {  // one bf16 rounding of dY
+    __nv_bfloat16* dyb = reinterpret_cast<__nv_bfloat16*>(base + align_up((size_t)K * Np * 2));
+    const int64_t n = M * N;
+    int64_t blocks = (n / 4 + 255) / 256;
+    if (blocks > 16 * (int64_t)sms) blocks = 16 * (int64_t)sms;
+    convert_bf16_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const float*>(dY), n, dyb);
+    BL_CUDA(cudaGetLastError());
+    a = dyb;
+  }
+  GmParams p = {};
+  p.rows = M;
+  p.cols = K;
+  p.kdim = N;
+  p.C = dA;
+  p.scale = gamma;
+  return run_bf16_gemm(a, N, wqt, Np, p, dev, st);
+}
+
+size_t bl_ste_grad_weight_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  const size_t Mp = (size_t)round8(M);
+  return align_up((size_t)N * Mp * 2) + align_up((size_t)K * Mp * 2);
+}
+
+bl_status bl_ste_grad_weight(const void* dY, bl_dtype dy_dtype, int64_t M, int64_t N,
+                             const int8_t* A_q, const float* gamma_A, int64_t K, const void* W,
+                             bl_dtype w_dtype, const float* gamma, float eps, float* dW,
+                             void* workspace, size_t ws_bytes, bl_stream_t stream) {
+  BL_TRY(check_dtype(dy_dtype));
+  BL_TRY(check_dtype(w_dtype));
+  BL_TRY(check_k(K));
+  BL_TRY(check_rows(M));
+  BL_TRY(check_rows(N));
+  BL_TRY(check_eps(eps));
+  if (N % 8 != 0) return BL_ERR_SHAPE;
+  if (N == 0) return BL_OK;
+  BL_TRY(check_ptr(dW));
+  if (M == 0) {
+    int dev, sms;
+    BL_TRY(current_device(&dev, &sms));
+    BL_CUDA(cudaMemsetAsync(dW, 0, (size_t)N * K * 4, reinterpret_cast<cudaStream_t>(stream)));
+    return BL_OK;
+  }
+  BL_TRY(check_ptr(dY));
+  BL_TRY(check_ptr(A_q));
+  BL_TRY(check_ptr(gamma_A));
+  BL_TRY(check_ptr(W));
+  if (gamma == nullptr) return BL_ERR_INVALID_ARG;
+  if (workspace == nullptr || ws_bytes < bl_ste_grad_weight_workspace_bytes(M, N, K))
+    return BL_ERR_WORKSPACE;
+  BL_TRY(check_ptr(workspace));
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t Mp = round8(M);
+  uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
+  __nv_bfloat16* dyt = reinterpret_cast<__nv_bfloat16*>(base);
+  __nv_bfloat16* aht = reinterpret_cast<__nv_bfloat16*>(base + align_up((size_t)N * Mp * 2));
+  const dim3 gt((unsigned)((N + 31) / 32), (unsigned)((Mp + 31) / 32));
+  if (dy_dtype == BL_BF16)
+    transpose_bf16_kernel<__nv_bfloat16><<<gt, 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(dY), M, N, Mp, dyt);
+  else
+    transpose_bf16_kernel<float><<<gt, 256, 0, st>>>(reinterpret_cast<const float*>(dY), M, N, Mp,
+                                                     dyt);
+  BL_CUDA(cudaGetLastError());
+  ahat_t_kernel<<<dim3((unsigned)((K + 31) / 32), (unsigned)((Mp + 31) / 32)), 256, 0, st>>>(
+      A_q, gamma_A, M, K, Mp, aht);
+  BL_CUDA(cudaGetLastError());
+  GmParams p = {};
+  p.rows = N;
+  p.cols = K;
+  p.kdim = Mp;
+  p.C = dW;
+  p.mask_w = W;
+  p.mask_bf16 = w_dtype == BL_BF16;
+  p.mask_gamma = gamma;
+  p.eps = eps;
+  return run_bf16_gemm(dyt, Mp, aht, Mp, p, dev, st);
 }
 
 bl_status bl_check_device_error(bl_stream_t stream) {
