@@ -71,6 +71,11 @@ def lib():
         L.orc_ste_grad_weight.argtypes = [P(ctypes.c_float), i64, i64, P(ctypes.c_int8),
                                           P(ctypes.c_float), i64, P(ctypes.c_float), f32, f32,
                                           P(ctypes.c_double)]
+        L.orc_radix3_row_bytes.restype = i64
+        L.orc_radix3_row_bytes.argtypes = [i64]
+        L.orc_pack_radix3.argtypes = [P(ctypes.c_int8), i64, i64, P(ctypes.c_uint8)]
+        L.orc_unpack_radix3.restype = i64
+        L.orc_unpack_radix3.argtypes = [P(ctypes.c_uint8), i64, i64, P(ctypes.c_int8)]
         L.orc_max_threads.restype = i32
         L.orc_set_threads.argtypes = [i32]
         _lib = L
@@ -260,3 +265,26 @@ def ste_grad_weight(dY, Aq, gammaA, W, gamma, eps):
                               float(np.float32(gamma)), float(np.float32(eps)),
                               _p(dW, ctypes.c_double))
     return dW
+
+
+def radix3_row_bytes(K: int) -> int:
+    return int(lib().orc_radix3_row_bytes(K))
+
+
+def pack_radix3(Wq):
+    """Radix-3 storage: 5 ternary weights per byte (first most significant),
+    byte = ceil(256·b/243); rows padded to 16 bytes."""
+    Wq = _i8(Wq)
+    N, K = Wq.shape
+    out = np.empty((N, radix3_row_bytes(K)), np.uint8)
+    lib().orc_pack_radix3(_p(Wq, ctypes.c_int8), N, K, _p(out, ctypes.c_uint8))
+    return out
+
+
+def unpack_radix3(packed, K):
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    N = packed.shape[0]
+    assert packed.shape[1] == radix3_row_bytes(K)
+    out = np.empty((N, K), np.int8)
+    bad = lib().orc_unpack_radix3(_p(packed, ctypes.c_uint8), N, K, _p(out, ctypes.c_int8))
+    return out, int(bad)

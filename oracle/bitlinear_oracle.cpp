@@ -335,6 +335,65 @@ void orc_ffn_relu2(const float* X, int64_t M, int64_t K, int64_t H,
 }
 
 // ---------------------------------------------------------------------------
+// Radix-3 storage ([BLOG] §"Como o ecossistema bitnet.cpp acelera ...": five
+// ternary weights in one byte, 3^5 = 243 ≤ 256, 1.60 bits per weight).
+// This library's layout of it:
+//   * a row of K weights is split into groups t of five consecutive weights
+//     k = 5t .. 5t+4 (weights past K count as 0);
+//   * the group's value is b = Σ_i d_i·3^(4-i) with d_i = w_{5t+i} + 1 (the
+//     first weight most significant, the digit order of the lookup-table
+//     figure), so b ∈ [0, 242];
+//   * the byte stored is q = ceil(256·b ÷ 243), b scaled to a fraction of
+//     256, which is what lets a decoder peel digits off with multiplies by 3;
+//     b = floor(243·q ÷ 256) recovers the group value;
+//   * a row takes ceil(K/5) bytes, padded with zero-valued groups (q of all
+//     weights 0) to a multiple of 16 bytes: row_bytes = 16·ceil(ceil(K/5)/16).
+int64_t orc_radix3_row_bytes(int64_t K) {
+  const int64_t groups = (K + 4) / 5;
+  return (groups + 15) / 16 * 16;
+}
+
+void orc_pack_radix3(const int8_t* Wq, int64_t N, int64_t K, uint8_t* out) {
+  const int64_t rb = orc_radix3_row_bytes(K);
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t t = 0; t < rb; ++t) {
+      int b = 0;
+      for (int i = 0; i < 5; ++i) {
+        const int64_t k = 5 * t + i;
+        const int d = (k < K) ? (int)Wq[n * K + k] + 1 : 1;
+        b = 3 * b + d;
+      }
+      out[n * rb + t] = (uint8_t)((256 * b + 242) / 243);  // ceil(256·b / 243)
+    }
+  }
+}
+
+// Inverse of orc_pack_radix3 (weights past K are dropped). Returns the
+// number of bytes that are not the image of a group value (never written
+// by the packer); those decode as their floor group value.
+int64_t orc_unpack_radix3(const uint8_t* in, int64_t N, int64_t K, int8_t* Wq) {
+  const int64_t rb = orc_radix3_row_bytes(K);
+  int64_t bad = 0;
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t t = 0; t < rb; ++t) {
+      const int q = in[n * rb + t];
+      const int b = (243 * q) / 256;  // floor
+      if ((256 * b + 242) / 243 != q) ++bad;
+      int rest = b;
+      for (int i = 0; i < 5; ++i) {
+        int p = 1;
+        for (int j = 0; j < 4 - i; ++j) p *= 3;
+        const int d = rest / p;
+        rest -= d * p;
+        const int64_t k = 5 * t + i;
+        if (k < K) Wq[n * K + k] = (int8_t)(d - 1);
+      }
+    }
+  }
+  return bad;
+}
+
+// ---------------------------------------------------------------------------
 // [BLOG] §Zero-GEMM, paragraph after the worked example: training uses the
 // Straight-Through Estimator; in the backward pass the gradient of the
 // quantisation is taken as the identity (∂W_q ÷ ∂W = 1) for values inside

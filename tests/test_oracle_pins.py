@@ -465,3 +465,46 @@ def test_ste_grads_match_float64_matmul(orc):
     mask = orc.ste_weight_mask(W, g, 1e-5)
     dW = orc.ste_grad_weight(dY, Aq, gA, W, g, 1e-5)
     np.testing.assert_allclose(dW, mask * (dY.astype(np.float64).T @ A_hat), rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Radix-3 storage ([BLOG] §bitnet.cpp: 5 trits per byte)
+
+def test_radix3_all_groups_round_trip(orc):
+    """Every one of the 3^5 = 243 five-weight groups packs into a distinct
+    byte and unpacks to itself; 243 of 256 byte states are used (94.9 %)."""
+    groups = np.array(list(itertools.product([-1, 0, 1], repeat=5)), np.int8).reshape(1, -1)
+    K = groups.shape[1]  # 1215 weights = 243 groups
+    packed = orc.pack_radix3(groups)
+    used = packed[0, :243]
+    assert len(set(used.tolist())) == 243
+    back, bad = orc.unpack_radix3(packed, K)
+    assert bad == 0
+    np.testing.assert_array_equal(back, groups)
+    g = read_golden("information_content.txt")
+    assert round(len(set(used.tolist())) / 256, 3) == g["radix3_state_fraction"][0]
+
+
+def test_radix3_hand_derived_bytes(orc):
+    """b = Σ d_i 3^(4-i), byte = ceil(256 b / 243): all -1 → b 0 → 0;
+    all 0 → b 121 → 128; all +1 → b 242 → 255; (+1,-1,-1,-1,-1) → b 162 → 171;
+    (-1,-1,-1,-1,+1) → b 2 → 3 (first weight most significant)."""
+    W = np.array([[-1] * 5 + [0] * 5 + [1] * 5 + [1, -1, -1, -1, -1] + [-1, -1, -1, -1, 1]], np.int8)
+    packed = orc.pack_radix3(W)
+    np.testing.assert_array_equal(packed[0, :5], [0, 128, 255, 171, 3])
+    assert np.all(packed[0, 5:] == 128)  # padding groups: all weights 0
+
+
+def test_radix3_density_and_ragged_rows(orc):
+    """1.60 bits per weight when K is a multiple of 80; ragged K pads the last
+    group with zeros and the row to 16 bytes; random rows round-trip."""
+    g = read_golden("information_content.txt")
+    assert orc.radix3_row_bytes(2560) == 512
+    assert round(8 * orc.radix3_row_bytes(2560) / 2560, 2) == g["radix3_bits_per_weight"][0]
+    assert orc.radix3_row_bytes(4096) == 832  # ceil(4096/5) = 820 → 832
+    rng = np.random.default_rng(12)
+    for K in (64, 4096, 11008, 77):
+        W = rng.integers(-1, 2, size=(7, K)).astype(np.int8)
+        back, bad = orc.unpack_radix3(orc.pack_radix3(W), K)
+        assert bad == 0
+        np.testing.assert_array_equal(back, W)
