@@ -82,7 +82,9 @@ enum {
    * buffer was NOT written by the kernel immediately preceding this call on
    * `stream` (true for a decode chain over static weights). Activations and
    * outputs are still ordered after the previous kernel. */
-  BL_FLAG_PDL = 1
+  BL_FLAG_PDL = 1,
+  /* bl_linear_radix3 only: Y is the raw INT32 accumulator [M, N]. */
+  BL_FLAG_RAW_I32 = 2
 };
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -281,6 +283,28 @@ bl_status bl_ffn_relu2_taps(const void* X, bl_dtype x_dtype, int64_t M,
                             const float* gamma_down, float eps, void* Y,
                             bl_dtype y_dtype, void* workspace, size_t ws_bytes,
                             const bl_taps* taps, bl_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Radix-3 weight storage for decode: five ternary weights per byte.
+ * BLOG, section "Como o ecossistema bitnet.cpp acelera inferência em CPUs e
+ * borda?": 3^5 = 243 ≤ 256 states, 1.60 bits per weight.
+ * Layout (this library's): each row is cut into groups of five consecutive
+ * weights, first weight most significant, b = Σ_i (w_i + 1)·3^(4-i) ∈
+ * [0, 242]; the byte stored is q = ceil(256·b / 243) (b = floor(243·q/256));
+ * weights past K count as 0; a row takes bl_radix3_row_bytes(K) =
+ * 16·ceil(ceil(K/5)/16) bytes (padding groups hold all-zero weights).
+ *   bl_pack_radix3: 2-bit packed [N, K/4] → radix-3 [N, row_bytes].
+ *   bl_linear_radix3: bl_linear for M ≤ bl_gemv_max_tokens() tokens on
+ *     radix-3 weights (one fused GEMV launch, same results as bl_linear);
+ *     flags: BL_FLAG_PDL as for bl_linear_ex, BL_FLAG_RAW_I32 to write the
+ *     INT32 accumulators instead (y_dtype ignored). M > 4: BL_ERR_SHAPE. */
+int64_t bl_radix3_row_bytes(int64_t K);
+bl_status bl_pack_radix3(const uint8_t* W_packed, int64_t N, int64_t K, uint8_t* W_r3,
+                         bl_stream_t stream);
+bl_status bl_linear_radix3(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
+                           const uint8_t* W_r3, const float* gamma, int64_t N, float eps,
+                           int relu2, void* Y, bl_dtype y_dtype, unsigned flags,
+                           bl_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Tensor-parallel FFN block: the per-rank steps of bl_ffn_relu2 when the

@@ -18,12 +18,13 @@ from __future__ import annotations
 import torch
 
 from . import _lib
-from ._lib import BL_BF16, BL_F32, BL_FLAG_PDL, BitLinearError, BlTaps, check, load
+from ._lib import BL_BF16, BL_F32, BL_FLAG_PDL, BL_FLAG_RAW_I32, BitLinearError, BlTaps, check, load
 
 __all__ = [
     "bl_quant_weights", "bl_quant_acts", "bl_zero_gemm", "bl_linear_q", "bl_linear",
     "bl_linear_noalloc", "bl_ffn_relu2", "bl_linear_taps", "bl_ffn_relu2_taps",
-    "bl_ffn_tp_up", "bl_ffn_tp_down", "bl_dequant_i32", "bl_ste_grad_input", "bl_ste_grad_weight", "bl_check_device_error", "bl_selftest_wait_timeout",
+    "bl_ffn_tp_up", "bl_ffn_tp_down", "bl_dequant_i32", "bl_ste_grad_input", "bl_ste_grad_weight",
+    "bl_pack_radix3", "bl_linear_radix3", "bl_check_device_error", "bl_selftest_wait_timeout",
     "bl_gemv_max_tokens", "workspace_bytes", "BitLinearError", "load", "BL_FLAG_PDL",
 ]
 
@@ -308,6 +309,37 @@ def bl_dequant_i32(acc, gamma_A, gamma, *, relu2=False, out_dtype=torch.bfloat16
     check(load().bl_dequant_i32(acc.data_ptr(), gamma_A.data_ptr(), gamma.data_ptr(), M, N,
                                 int(bool(relu2)), out.data_ptr(), _dt(out, "out"),
                                 _stream(stream)), "bl_dequant_i32")
+    return out
+
+
+def bl_pack_radix3(W_packed, K: int, *, out=None, stream=None):
+    """2-bit packed [N, K/4] → radix-3 storage [N, row_bytes] (5 weights/byte)."""
+    _cuda(W_packed, "W_packed")
+    N = W_packed.shape[0]
+    L = load()
+    rb = int(L.bl_radix3_row_bytes(K))
+    if out is None:
+        out = torch.empty((N, rb), dtype=torch.uint8, device=W_packed.device)
+    check(L.bl_pack_radix3(W_packed.data_ptr(), N, K, out.data_ptr(), _stream(stream)),
+          "bl_pack_radix3")
+    return out
+
+
+def bl_linear_radix3(A, W_r3, gamma, eps: float = 1e-5, *, relu2=False, out_dtype=torch.bfloat16,
+                     raw=False, out=None, pdl=False, stream=None):
+    """BitLinear for ≤ 4 tokens on radix-3 weights (raw=True: INT32 accumulators)."""
+    _cuda(A, "A")
+    _cuda(W_r3, "W_r3")
+    _cuda(gamma, "gamma")
+    M, K = A.shape
+    N = W_r3.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.int32 if raw else out_dtype, device=A.device)
+    flags = (BL_FLAG_PDL if pdl else 0) | (BL_FLAG_RAW_I32 if raw else 0)
+    ydt = BL_F32 if raw else _dt(out, "out")
+    check(load().bl_linear_radix3(A.data_ptr(), _dt(A, "A"), M, K, W_r3.data_ptr(), gamma.data_ptr(),
+                                  N, float(eps), int(bool(relu2)), out.data_ptr(), ydt, flags,
+                                  _stream(stream)), "bl_linear_radix3")
     return out
 
 

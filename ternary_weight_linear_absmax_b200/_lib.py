@@ -19,6 +19,7 @@ STATUS_NAMES = {
 }
 BL_F32, BL_BF16 = 0, 1
 BL_FLAG_PDL = 1
+BL_FLAG_RAW_I32 = 2
 
 class BlTaps(ctypes.Structure):
     """bl_taps of include/bitlinear.h: device pointers (0 = tap off)."""
@@ -58,6 +59,10 @@ SIGNATURES = {
                             _vp, _sz, _vp]),
     "bl_ffn_relu2_taps": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _f32, _vp,
                                  _int, _vp, _sz, ctypes.POINTER(BlTaps), _vp]),
+    "bl_radix3_row_bytes": (_i64, [_i64]),
+    "bl_pack_radix3": (_int, [_vp, _i64, _i64, _vp, _vp]),
+    "bl_linear_radix3": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _i64, _f32, _int, _vp, _int, _uint,
+                                _vp]),
     "bl_ffn_tp_up_workspace_bytes": (_sz, [_i64, _i64]),
     "bl_ffn_tp_up": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _sz,
                             _vp]),

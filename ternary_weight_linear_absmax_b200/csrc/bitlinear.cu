@@ -11,6 +11,7 @@
 #include "bitlinear.h"
 #include "bl_device.cuh"
 #include "gemv_kernel.cuh"
+#include "gemv_r3_kernel.cuh"
 #include "quant_kernels.cuh"
 #include "skinny_kernel.cuh"
 #include "ste_kernels.cuh"
@@ -510,6 +511,51 @@ bl_status run_quant_acts(const void* A, bl_dtype dt, int64_t M, int64_t K, float
         reinterpret_cast<const float*>(A), K, eps, Aq, gA, rs);
   BL_CUDA(cudaGetLastError());
   return BL_OK;
+}
+
+// --------------------------------------------------------------------------
+// Radix-3 decode GEMV launch.
+template <int MT, typename TA>
+bl_status launch_r3_t(const CUtensorMap& tw, const GemvR3Params& p, int grid, size_t smem, bool pdl,
+                      int dev, cudaStream_t st) {
+  auto* k = gemv_r3_kernel<MT, TA>;
+  BL_TRY(ensure_smem(k, dev, smem));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  BL_CUDA(cudaLaunchKernelEx(&cfg, k, tw, p));
+  return BL_OK;
+}
+
+bl_status run_r3(bl_dtype a_dtype, GemvR3Params p, bool pdl, int dev, int sms, cudaStream_t st) {
+  int64_t r = (p.N + sms - 1) / sms;
+  if (r < 1) r = 1;
+  if (r > kGemvMaxRows) r = kGemvMaxRows;
+  while (r > 1 && gemv_r3_smem_bytes(p.rb, (int)r, p.M) > kGemvSmemCap) r = (r + 1) / 2;
+  const size_t smem = gemv_r3_smem_bytes(p.rb, (int)r, p.M);
+  if (smem > kGemvSmemCap) return BL_ERR_SHAPE;
+  p.rows_per_cta = (int)r;
+  p.rows_pad = gemv_rows_pad((int)r);
+  const int grid = (int)((p.N + r - 1) / r);
+  CUtensorMap tw;
+  BL_TRY(make_map_u8(&tw, p.W, (uint64_t)p.N, (uint64_t)p.rb, 128, (uint32_t)p.rows_pad,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+  const bool bf = a_dtype == BL_BF16;
+  if (p.M == 1)
+    return bf ? launch_r3_t<1, __nv_bfloat16>(tw, p, grid, smem, pdl, dev, st)
+              : launch_r3_t<1, float>(tw, p, grid, smem, pdl, dev, st);
+  if (p.M == 2)
+    return bf ? launch_r3_t<2, __nv_bfloat16>(tw, p, grid, smem, pdl, dev, st)
+              : launch_r3_t<2, float>(tw, p, grid, smem, pdl, dev, st);
+  return bf ? launch_r3_t<4, __nv_bfloat16>(tw, p, grid, smem, pdl, dev, st)
+            : launch_r3_t<4, float>(tw, p, grid, smem, pdl, dev, st);
 }
 
 // --------------------------------------------------------------------------
@@ -1102,6 +1148,65 @@ bl_status bl_dequant_i32(const int32_t* acc, const float* gamma_A, const float* 
       acc, gamma_A, gamma, M, N, relu2 ? 1 : 0, Y, y_dtype == BL_BF16);
   BL_CUDA(cudaGetLastError());
   return BL_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Radix-3 storage and its decode GEMV.
+
+int64_t bl_radix3_row_bytes(int64_t K) { return K > 0 ? radix3_row_bytes(K) : 0; }
+
+bl_status bl_pack_radix3(const uint8_t* W_packed, int64_t N, int64_t K, uint8_t* W_r3,
+                         bl_stream_t stream) {
+  BL_TRY(check_k(K));
+  BL_TRY(check_rows(N));
+  if (N == 0) return BL_OK;
+  BL_TRY(check_ptr(W_packed));
+  BL_TRY(check_ptr(W_r3));
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  const int64_t total = N * radix3_row_bytes(K);
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 16 * (int64_t)sms) blocks = 16 * (int64_t)sms;
+  radix3_pack_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      W_packed, N, K, radix3_row_bytes(K), W_r3);
+  BL_CUDA(cudaGetLastError());
+  return BL_OK;
+}
+
+bl_status bl_linear_radix3(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
+                           const uint8_t* W_r3, const float* gamma, int64_t N, float eps,
+                           int relu2, void* Y, bl_dtype y_dtype, unsigned flags,
+                           bl_stream_t stream) {
+  BL_TRY(check_dtype(a_dtype));
+  BL_TRY(check_dtype(y_dtype));
+  BL_TRY(check_k(K));
+  BL_TRY(check_rows(M));
+  BL_TRY(check_rows(N));
+  BL_TRY(check_eps(eps));
+  if ((flags & ~(unsigned)(BL_FLAG_PDL | BL_FLAG_RAW_I32)) != 0) return BL_ERR_INVALID_ARG;
+  if (M > kGemvMaxTokens) return BL_ERR_SHAPE;
+  if (M == 0 || N == 0) return BL_OK;
+  BL_TRY(check_ptr(A));
+  BL_TRY(check_ptr(W_r3));
+  if (gamma == nullptr) return BL_ERR_INVALID_ARG;
+  BL_TRY(check_ptr(Y));
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  GemvR3Params p = {};
+  p.A = A;
+  p.W = W_r3;
+  p.gamma = gamma;
+  p.Y = Y;
+  p.N = N;
+  p.K = K;
+  p.rb = radix3_row_bytes(K);
+  p.M = (int)M;
+  p.eps = eps;
+  p.relu2 = relu2 ? 1 : 0;
+  p.y_bf16 = y_dtype == BL_BF16;
+  p.raw = (flags & BL_FLAG_RAW_I32) != 0;
+  return run_r3(a_dtype, p, (flags & BL_FLAG_PDL) != 0, dev, sms,
+                reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------

@@ -116,3 +116,15 @@ def test_k_bound_and_taps_checked_on_host(lib):
                               None) == BL_ERR_ALIGN
     assert lib.bl_ffn_relu2_taps(p, 1, 1, 512, 640, p, p, p, p, 1e-5, p, 1, p, 1 << 20,
                                  misaligned, None) == BL_ERR_ALIGN
+
+
+def test_radix3_host_checks(lib):
+    keep, p = _aligned_buf()
+    BL_ERR_INVALID_ARG, BL_ERR_SHAPE = 1, 2
+    assert lib.bl_radix3_row_bytes(2560) == 512
+    assert lib.bl_radix3_row_bytes(4096) == 832
+    # more than 4 tokens, bad flags, bad K: refused before any launch
+    assert lib.bl_linear_radix3(p, 1, 5, 512, p, p, 64, 1e-5, 0, p, 1, 0, None) == BL_ERR_SHAPE
+    assert lib.bl_linear_radix3(p, 1, 1, 512, p, p, 64, 1e-5, 0, p, 1, 4, None) == BL_ERR_INVALID_ARG
+    assert lib.bl_linear_radix3(p, 1, 1, 500, p, p, 64, 1e-5, 0, p, 1, 0, None) == BL_ERR_SHAPE
+    assert lib.bl_pack_radix3(p, 8, 100, p, None) == BL_ERR_SHAPE
