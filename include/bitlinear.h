@@ -83,7 +83,8 @@ enum {
    * `stream` (true for a decode chain over static weights). Activations and
    * outputs are still ordered after the previous kernel. */
   BL_FLAG_PDL = 1,
-  /* bl_linear_radix3 only: Y is the raw INT32 accumulator [M, N]. */
+  /* bl_linear_radix3 / bl_linear_lut only: Y is the raw INT32
+   * accumulator [M, N]. */
   BL_FLAG_RAW_I32 = 2
 };
 
@@ -305,6 +306,25 @@ bl_status bl_linear_radix3(const void* A, bl_dtype a_dtype, int64_t M, int64_t K
                            const uint8_t* W_r3, const float* gamma, int64_t N, float eps,
                            int relu2, void* Y, bl_dtype y_dtype, unsigned flags,
                            bl_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Lookup-table decode (one token). BLOG, section "Como o ecossistema
+ * bitnet.cpp acelera inferência em CPUs e borda?", figure "Fluxo de Execução
+ * com Lookup Table (LUT-GEMM)": per block of 4 int8 activations a table of
+ * the 81 signed sums of all ternary patterns; each group of 4 weights is one
+ * index (27·d0 + 9·d1 + 3·d2 + d3, d = w + 1, first weight most significant:
+ * 0 = all -1, 40 = all 0, 80 = all +1).
+ *   bl_pack_lut_index: 2-bit packed [N, K/4] → index bytes [N, K/4]
+ *     (byte g of a row indexes weights 4g .. 4g+3).
+ *   bl_linear_lut: bl_linear for M = 1 on index bytes (tables of the token
+ *     built in shared memory by every CTA; results equal bl_linear's);
+ *     flags BL_FLAG_PDL, BL_FLAG_RAW_I32 as for bl_linear_radix3.
+ *     M > 1, or K whose tables exceed shared memory: BL_ERR_SHAPE. */
+bl_status bl_pack_lut_index(const uint8_t* W_packed, int64_t N, int64_t K, uint8_t* W_idx,
+                            bl_stream_t stream);
+bl_status bl_linear_lut(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
+                        const uint8_t* W_idx, const float* gamma, int64_t N, float eps,
+                        void* Y, bl_dtype y_dtype, unsigned flags, bl_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Tensor-parallel FFN block: the per-rank steps of bl_ffn_relu2 when the

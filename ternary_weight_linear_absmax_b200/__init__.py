@@ -24,7 +24,7 @@ __all__ = [
     "bl_quant_weights", "bl_quant_acts", "bl_zero_gemm", "bl_linear_q", "bl_linear",
     "bl_linear_noalloc", "bl_ffn_relu2", "bl_linear_taps", "bl_ffn_relu2_taps",
     "bl_ffn_tp_up", "bl_ffn_tp_down", "bl_dequant_i32", "bl_ste_grad_input", "bl_ste_grad_weight",
-    "bl_pack_radix3", "bl_linear_radix3", "bl_check_device_error", "bl_selftest_wait_timeout",
+    "bl_pack_radix3", "bl_linear_radix3", "bl_pack_lut_index", "bl_linear_lut", "bl_check_device_error", "bl_selftest_wait_timeout",
     "bl_gemv_max_tokens", "workspace_bytes", "BitLinearError", "load", "BL_FLAG_PDL",
 ]
 
@@ -340,6 +340,34 @@ def bl_linear_radix3(A, W_r3, gamma, eps: float = 1e-5, *, relu2=False, out_dtyp
     check(load().bl_linear_radix3(A.data_ptr(), _dt(A, "A"), M, K, W_r3.data_ptr(), gamma.data_ptr(),
                                   N, float(eps), int(bool(relu2)), out.data_ptr(), ydt, flags,
                                   _stream(stream)), "bl_linear_radix3")
+    return out
+
+
+def bl_pack_lut_index(W_packed, *, out=None, stream=None):
+    """2-bit packed [N, K/4] → lookup-table index bytes [N, K/4]."""
+    _cuda(W_packed, "W_packed")
+    N, Kq = W_packed.shape
+    if out is None:
+        out = torch.empty((N, Kq), dtype=torch.uint8, device=W_packed.device)
+    check(load().bl_pack_lut_index(W_packed.data_ptr(), N, 4 * Kq, out.data_ptr(), _stream(stream)),
+          "bl_pack_lut_index")
+    return out
+
+
+def bl_linear_lut(A, W_idx, gamma, eps: float = 1e-5, *, out_dtype=torch.bfloat16, raw=False,
+                  out=None, pdl=False, stream=None):
+    """BitLinear for one token by table lookup (raw=True: INT32 accumulators)."""
+    _cuda(A, "A")
+    _cuda(W_idx, "W_idx")
+    _cuda(gamma, "gamma")
+    M, K = A.shape
+    N = W_idx.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.int32 if raw else out_dtype, device=A.device)
+    flags = (BL_FLAG_PDL if pdl else 0) | (BL_FLAG_RAW_I32 if raw else 0)
+    check(load().bl_linear_lut(A.data_ptr(), _dt(A, "A"), M, K, W_idx.data_ptr(), gamma.data_ptr(),
+                               N, float(eps), out.data_ptr(), BL_F32 if raw else _dt(out, "out"),
+                               flags, _stream(stream)), "bl_linear_lut")
     return out
 
 

@@ -63,6 +63,8 @@ SIGNATURES = {
     "bl_pack_radix3": (_int, [_vp, _i64, _i64, _vp, _vp]),
     "bl_linear_radix3": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _i64, _f32, _int, _vp, _int, _uint,
                                 _vp]),
+    "bl_pack_lut_index": (_int, [_vp, _i64, _i64, _vp, _vp]),
+    "bl_linear_lut": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _i64, _f32, _vp, _int, _uint, _vp]),
     "bl_ffn_tp_up_workspace_bytes": (_sz, [_i64, _i64]),
     "bl_ffn_tp_up": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _sz,
                             _vp]),

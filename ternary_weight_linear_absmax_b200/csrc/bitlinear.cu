@@ -11,6 +11,7 @@
 #include "bitlinear.h"
 #include "bl_device.cuh"
 #include "gemv_kernel.cuh"
+#include "gemv_lut_kernel.cuh"
 #include "gemv_r3_kernel.cuh"
 #include "quant_kernels.cuh"
 #include "skinny_kernel.cuh"
@@ -556,6 +557,27 @@ bl_status run_r3(bl_dtype a_dtype, GemvR3Params p, bool pdl, int dev, int sms, c
               : launch_r3_t<2, float>(tw, p, grid, smem, pdl, dev, st);
   return bf ? launch_r3_t<4, __nv_bfloat16>(tw, p, grid, smem, pdl, dev, st)
             : launch_r3_t<4, float>(tw, p, grid, smem, pdl, dev, st);
+}
+
+// --------------------------------------------------------------------------
+// Lookup-table decode GEMV launch (one token).
+template <typename TA>
+bl_status launch_lut_t(const CUtensorMap& tw, const GemvLutParams& p, int grid, size_t smem,
+                       bool pdl, int dev, cudaStream_t st) {
+  auto* k = gemv_lut_kernel<TA>;
+  BL_TRY(ensure_smem(k, dev, smem));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  BL_CUDA(cudaLaunchKernelEx(&cfg, k, tw, p));
+  return BL_OK;
 }
 
 // --------------------------------------------------------------------------
@@ -1207,6 +1229,73 @@ bl_status bl_linear_radix3(const void* A, bl_dtype a_dtype, int64_t M, int64_t K
   p.raw = (flags & BL_FLAG_RAW_I32) != 0;
   return run_r3(a_dtype, p, (flags & BL_FLAG_PDL) != 0, dev, sms,
                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// Lookup-table weights and their decode GEMV (one token).
+
+bl_status bl_pack_lut_index(const uint8_t* W_packed, int64_t N, int64_t K, uint8_t* W_idx,
+                            bl_stream_t stream) {
+  BL_TRY(check_k(K));
+  BL_TRY(check_rows(N));
+  if (N == 0) return BL_OK;
+  BL_TRY(check_ptr(W_packed));
+  BL_TRY(check_ptr(W_idx));
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  const int64_t total = N * (K / 4);
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 16 * (int64_t)sms) blocks = 16 * (int64_t)sms;
+  lut_index_pack_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      W_packed, total, W_idx);
+  BL_CUDA(cudaGetLastError());
+  return BL_OK;
+}
+
+bl_status bl_linear_lut(const void* A, bl_dtype a_dtype, int64_t M, int64_t K, const uint8_t* W_idx,
+                        const float* gamma, int64_t N, float eps, void* Y, bl_dtype y_dtype,
+                        unsigned flags, bl_stream_t stream) {
+  BL_TRY(check_dtype(a_dtype));
+  BL_TRY(check_dtype(y_dtype));
+  BL_TRY(check_k(K));
+  BL_TRY(check_rows(M));
+  BL_TRY(check_rows(N));
+  BL_TRY(check_eps(eps));
+  if ((flags & ~(unsigned)(BL_FLAG_PDL | BL_FLAG_RAW_I32)) != 0) return BL_ERR_INVALID_ARG;
+  if (M > 1) return BL_ERR_SHAPE;
+  if (M == 0 || N == 0) return BL_OK;
+  BL_TRY(check_ptr(A));
+  BL_TRY(check_ptr(W_idx));
+  if (gamma == nullptr) return BL_ERR_INVALID_ARG;
+  BL_TRY(check_ptr(Y));
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  int64_t r = (N + sms - 1) / sms;
+  if (r < 1) r = 1;
+  if (r > kGemvMaxRows) r = kGemvMaxRows;
+  while (r > 1 && gemv_lut_smem_bytes(K, (int)r) > kGemvSmemCap) r = (r + 1) / 2;
+  const size_t smem = gemv_lut_smem_bytes(K, (int)r);
+  if (smem > kSkSmemCap) return BL_ERR_SHAPE;  // tables of very long rows do not fit
+  GemvLutParams p = {};
+  p.A = A;
+  p.W = W_idx;
+  p.gamma = gamma;
+  p.Y = Y;
+  p.N = N;
+  p.K = K;
+  p.rows_per_cta = (int)r;
+  p.rows_pad = gemv_rows_pad((int)r);
+  p.eps = eps;
+  p.y_bf16 = y_dtype == BL_BF16;
+  p.raw = (flags & BL_FLAG_RAW_I32) != 0;
+  const int grid = (int)((N + r - 1) / r);
+  CUtensorMap tw;
+  BL_TRY(make_map_u8(&tw, W_idx, (uint64_t)N, (uint64_t)(K / 4), 128, (uint32_t)p.rows_pad,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool pdl = (flags & BL_FLAG_PDL) != 0;
+  return a_dtype == BL_BF16 ? launch_lut_t<__nv_bfloat16>(tw, p, grid, smem, pdl, dev, st)
+                            : launch_lut_t<float>(tw, p, grid, smem, pdl, dev, st);
 }
 
 // ---------------------------------------------------------------------------

@@ -27,6 +27,7 @@
 
 #include "bl_device.cuh"
 #include "gemv_kernel.cuh"
+#include "gemv_prologue.cuh"
 
 namespace bl {
 
@@ -101,7 +102,7 @@ gemv_r3_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvR3Params p) {
   __shared__ __align__(16) int s_wsum[MT][kGemvWarps];
   __shared__ float s_sc[MT];
   __shared__ int s_wok;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t K = p.K, rb = p.rb, Kp = 5 * rb;
   const int64_t r0 = (int64_t)blockIdx.x * p.rows_per_cta;
   const int R = (int)min((int64_t)p.rows_per_cta, p.N - r0);
@@ -146,48 +147,8 @@ gemv_r3_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvR3Params p) {
   __syncthreads();
 
   // 2. AbsMax per token → int8 tokens (positions K .. 5·rb-1 are zero), Σ A_q.
-  constexpr int VEC = 16 / (int)sizeof(TA);
-  const int64_t nvec = K / VEC;
-  for (int m = 0; m < MT; ++m) {
-    float mx = 0.0f;
-    if (m < M) {
-      const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const TA*>(p.A) + m * K);
-      for (int64_t v = tid; v < nvec; v += kGemvThreads) {
-        const uint4 u = __ldg(src + v);
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) mx = fmaxf(mx, fabsf(to_f32<TA>(reinterpret_cast<const TA*>(&u)[i])));
-      }
-    }
-    const unsigned wm = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
-    if (lane == 0) s_wmax[m][warp] = wm;
-  }
-  __syncthreads();
-  for (int m = 0; m < MT; ++m) {
-    int tsum = 0;
-    if (m < M) {
-      const float g = __uint_as_float(warp_slots_max(s_wmax[m]));
-      const float s = __fdiv_rn(127.0f, __fadd_rn(g, p.eps));
-      const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const TA*>(p.A) + m * K);
-      for (int64_t v = tid; v < nvec; v += kGemvThreads) {
-        const uint4 u = __ldg(src + v);
-        uint32_t w[VEC / 4];
-#pragma unroll
-        for (int i = 0; i < VEC / 4; ++i) {
-          const TA* e = reinterpret_cast<const TA*>(&u) + 4 * i;
-          w[i] = pack4_low_bytes(quant_i8_bits(to_f32<TA>(e[0]), s), quant_i8_bits(to_f32<TA>(e[1]), s),
-                                 quant_i8_bits(to_f32<TA>(e[2]), s), quant_i8_bits(to_f32<TA>(e[3]), s));
-          tsum = dp4a(w[i], 0x01010101u, tsum);
-          *reinterpret_cast<uint32_t*>(s_a + m * Kp + v * VEC + 4 * i) = w[i];
-        }
-      }
-      for (int64_t v = K / 4 + tid; v < Kp / 4; v += kGemvThreads)
-        *reinterpret_cast<uint32_t*>(s_a + m * Kp + 4 * v) = 0u;
-      if (tid == kGemvThreads - 1) s_sc[m] = __fdiv_rn(__fmul_rn(g, gamma_w), 127.0f);
-    }
-    const int ws = __reduce_add_sync(0xffffffffu, tsum);
-    if (lane == 0) s_wsum[m][warp] = ws;
-  }
-  __syncthreads();
+  gemv_absmax_prologue<MT, TA>(reinterpret_cast<const TA*>(p.A), M, K, Kp, p.eps, gamma_w, s_a,
+                               s_wmax, s_wsum, s_sc);
 
   // 3. Token coefficients: word u holds groups t = 4u + j (j = 0..3); for digit
   //    i = 1..5, β_i of the four groups as int16 pairs (j = 0, 1 | j = 2, 3).

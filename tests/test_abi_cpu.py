@@ -128,3 +128,11 @@ def test_radix3_host_checks(lib):
     assert lib.bl_linear_radix3(p, 1, 1, 512, p, p, 64, 1e-5, 0, p, 1, 4, None) == BL_ERR_INVALID_ARG
     assert lib.bl_linear_radix3(p, 1, 1, 500, p, p, 64, 1e-5, 0, p, 1, 0, None) == BL_ERR_SHAPE
     assert lib.bl_pack_radix3(p, 8, 100, p, None) == BL_ERR_SHAPE
+
+
+def test_lut_host_checks(lib):
+    keep, p = _aligned_buf()
+    BL_ERR_INVALID_ARG, BL_ERR_SHAPE = 1, 2
+    assert lib.bl_linear_lut(p, 1, 2, 512, p, p, 64, 1e-5, p, 1, 0, None) == BL_ERR_SHAPE
+    assert lib.bl_linear_lut(p, 1, 1, 512, p, p, 64, 1e-5, p, 1, 8, None) == BL_ERR_INVALID_ARG
+    assert lib.bl_pack_lut_index(p, 8, 100, p, None) == BL_ERR_SHAPE
