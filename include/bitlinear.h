@@ -16,6 +16,11 @@
  *    memory the caller owns. The library never allocates, frees or keeps
  *    pointers after the call returns. Scratch memory ("workspace") is passed
  *    in by the caller; its size comes from the matching *_workspace_bytes().
+ *    For bl_zero_gemm, bl_linear_q, bl_linear and bl_ffn_relu2 part of that
+ *    size is optional: with more than 64 tokens and too few output tiles to
+ *    fill the SMs, the tensor-core contraction splits K into up to 4 ranges
+ *    whose INT32 partials go there; a smaller workspace (down to the
+ *    quantised tokens and row sums) gives the same results unsplit.
  *  * Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream) and makes no host synchronisation. Scales
  *    (γ, γ_A) are passed by device pointer for the same reason.
@@ -319,7 +324,8 @@ bl_status bl_linear_radix3(const void* A, bl_dtype a_dtype, int64_t M, int64_t K
  *   bl_linear_lut: bl_linear for M = 1 on index bytes (tables of the token
  *     built in shared memory by every CTA; results equal bl_linear's);
  *     flags BL_FLAG_PDL, BL_FLAG_RAW_I32 as for bl_linear_radix3.
- *     M > 1, or K whose tables exceed shared memory: BL_ERR_SHAPE. */
+ *     M > 1, or K whose tables (K/4 · 41 int16) do not fit in a CTA's
+ *     shared memory beside its weights (K above about 10,000): BL_ERR_SHAPE. */
 bl_status bl_pack_lut_index(const uint8_t* W_packed, int64_t N, int64_t K, uint8_t* W_idx,
                             bl_stream_t stream);
 bl_status bl_linear_lut(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,

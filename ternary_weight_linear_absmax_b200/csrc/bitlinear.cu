@@ -314,6 +314,96 @@ bl_status launch_tc_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tw,
 
 int tc_pick_bn(int64_t M) { return M <= 128 ? 128 : 256; }
 
+// ---------------------------------------------------------------------------
+// Persistent tensor-core kernel: K ranges per tile when the tiles alone fill at
+// most half of the SMs (each range at least 8 K blocks, at most 4 ranges).
+constexpr int kTc2WsSms = 148;  // B200: the SM count workspaces are sized for
+
+int tc2_splits(int64_t M, int64_t N, int64_t K, int sms) {
+  const int64_t tiles = ((N + 127) / 128) * ((M + kTc2BN - 1) / kTc2BN);
+  const int64_t KB = (K + kTcBK - 1) / kTcBK;
+  if (tiles * 2 > sms) return 1;
+  int64_t sp = sms / tiles;
+  if (sp > 4) sp = 4;
+  int64_t most = KB / 8;
+  if (sp > most) sp = most;
+  return sp < 1 ? 1 : (int)sp;
+}
+
+size_t tc2_ws_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= kSkMaxTokens) return 0;
+  const int sp = tc2_splits(M, N, K, kTc2WsSms);
+  if (sp <= 1) return 0;
+  const int64_t tiles = ((N + 127) / 128) * ((M + kTc2BN - 1) / kTc2BN);
+  return align_up((size_t)sp * M * N * 4) + align_up((size_t)tiles * 4);
+}
+
+// pdl: launch with programmatic dependent launch (not after a memset).
+template <int OUT>
+bl_status launch_tc2_t(const CUtensorMap& ta, const CUtensorMap& tw, const Tc2Params& p, int grid,
+                       bool pdl, int dev, cudaStream_t st) {
+  auto* k = tc_persistent_kernel<OUT>;
+  constexpr size_t smem = Tc2::kSmem;
+  BL_TRY(ensure_smem(k, dev, smem));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kTc2Threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  BL_CUDA(cudaLaunchKernelEx(&cfg, k, ta, tw, p));
+  return BL_OK;
+}
+
+// acc/Y[M,N] = epilogue(A_q[M,K] · W_q[N,K]ᵀ − rowsum), persistent CTAs.
+// split_ws: optional scratch of tc2_ws_bytes(M, N, K) bytes for K ranges.
+bl_status run_tc2(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,
+                  const float* gamma, const float* gammaA, const int32_t* rowsum, void* Y, int out,
+                  int relu2, int y_bf16, void* split_ws, size_t split_ws_bytes, int dev, int sms,
+                  cudaStream_t st) {
+  if (M > 0x7FFFFFFF || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
+  CUtensorMap ta, tw;
+  BL_TRY(make_map_u8(&ta, Aq, (uint64_t)M, (uint64_t)K, kTcBK, (uint32_t)kTc2BN,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+  BL_TRY(make_map_u8(&tw, Wp, (uint64_t)N, (uint64_t)(K / 4), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B));
+  Tc2Params p = {};
+  p.gamma = gamma;
+  p.gammaA = gammaA;
+  p.rowsum = rowsum;
+  p.Y = Y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.relu2 = relu2;
+  p.y_bf16 = y_bf16;
+  p.tiles_n = (int)((N + 127) / 128);
+  p.tiles = p.tiles_n * (int)((M + kTc2BN - 1) / kTc2BN);
+  const int KB = (int)((K + kTcBK - 1) / kTcBK);
+  int sp = tc2_splits(M, N, K, sms);
+  const int sp_ws = tc2_splits(M, N, K, kTc2WsSms);
+  if (sp > sp_ws) sp = sp_ws;
+  if (sp > 1 && (split_ws == nullptr || split_ws_bytes < tc2_ws_bytes(M, N, K))) sp = 1;
+  p.splits = sp;
+  p.kb_per_split = ((KB + sp - 1) / sp + 3) / 4 * 4;
+  p.splits = (KB + p.kb_per_split - 1) / p.kb_per_split;  // no empty ranges
+  if (p.splits > 1) {
+    uint8_t* base = reinterpret_cast<uint8_t*>(split_ws);
+    p.part = reinterpret_cast<int32_t*>(base);
+    p.counter = reinterpret_cast<int32_t*>(base + align_up((size_t)p.splits * M * N * 4));
+    BL_CUDA(cudaMemsetAsync(p.counter, 0, (size_t)p.tiles * 4, st));
+  }
+  const int items = p.tiles * p.splits;
+  const int grid = items < sms ? items : sms;
+  // After the counters' memset the launch is ordered normally.
+  const bool pdl = p.splits == 1;
+  return out == kTcDequant ? launch_tc2_t<kTcDequant>(ta, tw, p, grid, pdl, dev, st)
+                           : launch_tc2_t<kTcRawI32>(ta, tw, p, grid, pdl, dev, st);
+}
+
 // acc/Y[M,N] = epilogue(A_q[M,K] · W_q[N,K]ᵀ − rowsum).
 bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,
                  const float* gamma, const float* gammaA, const int32_t* rowsum, void* Y,
@@ -490,15 +580,18 @@ bl_status run_skinny(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, 
 }
 
 // Contraction of pre-quantised tokens: the skinny kernel up to 64 tokens,
-// tensor cores above. out: kTcDequant or kTcRawI32.
+// persistent tensor-core CTAs above. out: kTcDequant or kTcRawI32.
+// split_ws: optional scratch (tc2_ws_bytes) that lets under-filled tensor-core
+// launches split K.
 bl_status run_contract(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,
                        const float* gamma, const float* gammaA, const int32_t* rowsum, void* Y,
                        int out, int relu2, int y_bf16, bool pdl, int dev, int sms,
-                       cudaStream_t st) {
+                       cudaStream_t st, void* split_ws = nullptr, size_t split_ws_bytes = 0) {
   if (M <= kSkMaxTokens)
     return run_skinny(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out == kTcRawI32 ? 1 : 0, relu2,
                       y_bf16, pdl, dev, sms, st);
-  return run_tc(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out, relu2, y_bf16, dev, st);
+  return run_tc2(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out, relu2, y_bf16, split_ws,
+                 split_ws_bytes, dev, sms, st);
 }
 
 bl_status run_quant_acts(const void* A, bl_dtype dt, int64_t M, int64_t K, float eps, int8_t* Aq,
@@ -536,12 +629,14 @@ bl_status launch_r3_t(const CUtensorMap& tw, const GemvR3Params& p, int grid, si
 }
 
 bl_status run_r3(bl_dtype a_dtype, GemvR3Params p, bool pdl, int dev, int sms, cudaStream_t st) {
+  // Two CTAs per SM when the token coefficients leave room, else one.
+  const size_t cap = gemv_r3_smem_bytes(p.rb, 8, p.M) <= kGemvSmemCap ? kGemvSmemCap : kSkSmemCap;
   int64_t r = (p.N + sms - 1) / sms;
   if (r < 1) r = 1;
   if (r > kGemvMaxRows) r = kGemvMaxRows;
-  while (r > 1 && gemv_r3_smem_bytes(p.rb, (int)r, p.M) > kGemvSmemCap) r = (r + 1) / 2;
+  while (r > 1 && gemv_r3_smem_bytes(p.rb, (int)r, p.M) > cap) r = (r + 1) / 2;
   const size_t smem = gemv_r3_smem_bytes(p.rb, (int)r, p.M);
-  if (smem > kGemvSmemCap) return BL_ERR_SHAPE;
+  if (smem > cap) return BL_ERR_SHAPE;
   p.rows_per_cta = (int)r;
   p.rows_pad = gemv_rows_pad((int)r);
   const int grid = (int)((p.N + r - 1) / r);
@@ -756,10 +851,8 @@ bl_status bl_quant_acts(const void* A, bl_dtype a_dtype, int64_t M, int64_t K, f
 }
 
 size_t bl_zero_gemm_workspace_bytes(int64_t M, int64_t K, int64_t N) {
-  (void)K;
-  (void)N;
   if (M <= kGemvMaxTokens) return 0;
-  return align_up((size_t)M * 4);
+  return align_up((size_t)M * 4) + tc2_ws_bytes(M, N, K);
 }
 
 bl_status bl_zero_gemm(const int8_t* A_q, int64_t M, int64_t K, const uint8_t* W_packed,
@@ -772,7 +865,9 @@ bl_status bl_zero_gemm(const int8_t* A_q, int64_t M, int64_t K, const uint8_t* W
   BL_TRY(check_ptr(A_q));
   BL_TRY(check_ptr(W_packed));
   BL_TRY(check_ptr(acc));
-  const size_t need = bl_zero_gemm_workspace_bytes(M, K, N);
+  // Required: the row sums; the rest of bl_zero_gemm_workspace_bytes (K
+  // ranges of under-filled tensor-core launches) is used when present.
+  const size_t need = M <= kGemvMaxTokens ? 0 : align_up((size_t)M * 4);
   if (need > 0) {
     if (workspace == nullptr || ws_bytes < need) return BL_ERR_WORKSPACE;
     BL_TRY(check_ptr(workspace));
@@ -795,14 +890,13 @@ bl_status bl_zero_gemm(const int8_t* A_q, int64_t M, int64_t K, const uint8_t* W
   rowsum_i8_kernel<<<(unsigned)M, kQuantThreads, 0, st>>>(A_q, K, rs);
   BL_CUDA(cudaGetLastError());
   return run_contract(A_q, W_packed, M, K, N, nullptr, nullptr, rs, acc, kTcRawI32, 0, 0, true,
-                      dev, sms, st);
+                      dev, sms, st, reinterpret_cast<uint8_t*>(workspace) + align_up((size_t)M * 4),
+                      ws_bytes - align_up((size_t)M * 4));
 }
 
 size_t bl_linear_q_workspace_bytes(int64_t M, int64_t K, int64_t N) {
-  (void)K;
-  (void)N;
   if (M <= kGemvMaxTokens) return 0;
-  return align_up((size_t)M * 4);
+  return align_up((size_t)M * 4) + tc2_ws_bytes(M, N, K);
 }
 
 bl_status bl_linear_q(const int8_t* A_q, const float* gamma_A, const int32_t* rowsum, int64_t M,
@@ -820,11 +914,11 @@ bl_status bl_linear_q(const int8_t* A_q, const float* gamma_A, const int32_t* ro
   BL_TRY(check_ptr(W_packed));
   if (gamma == nullptr) return BL_ERR_INVALID_ARG;
   BL_TRY(check_ptr(Y));
-  const size_t need = rowsum ? 0 : bl_linear_q_workspace_bytes(M, K, N);
-  if (need > 0) {
-    if (workspace == nullptr || ws_bytes < need) return BL_ERR_WORKSPACE;
-    BL_TRY(check_ptr(workspace));
-  }
+  // The row sums' part is needed only without rowsum; the rest (K ranges of
+  // under-filled tensor-core launches) is used when present.
+  const size_t need = (rowsum || M <= kGemvMaxTokens) ? 0 : align_up((size_t)M * 4);
+  if (need > 0 && (workspace == nullptr || ws_bytes < need)) return BL_ERR_WORKSPACE;
+  if (workspace != nullptr) BL_TRY(check_ptr(workspace));
   int dev, sms;
   BL_TRY(current_device(&dev, &sms));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -853,14 +947,17 @@ bl_status bl_linear_q(const int8_t* A_q, const float* gamma_A, const int32_t* ro
   }
   // After this call's row-sum kernel the weights may stream early; without
   // it the preceding kernel is the caller's, so no early start.
+  const size_t rs_part = align_up((size_t)M * 4);
+  void* split_ws = (workspace != nullptr && ws_bytes > rs_part)
+                       ? reinterpret_cast<uint8_t*>(workspace) + rs_part : nullptr;
   return run_contract(A_q, W_packed, M, K, N, gamma, gamma_A, rs, Y, kTcDequant, relu2 ? 1 : 0,
-                      y_dtype == BL_BF16, rowsum == nullptr, dev, sms, st);
+                      y_dtype == BL_BF16, rowsum == nullptr, dev, sms, st, split_ws,
+                      split_ws ? ws_bytes - rs_part : 0);
 }
 
 size_t bl_linear_workspace_bytes(int64_t M, int64_t K, int64_t N) {
-  (void)N;
   if (M <= kGemvMaxTokens) return 0;
-  return act_ws(M, K).total;
+  return act_ws(M, K).total + tc2_ws_bytes(M, N, K);
 }
 
 static bl_status linear_impl(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
@@ -881,7 +978,9 @@ static bl_status linear_impl(const void* A, bl_dtype a_dtype, int64_t M, int64_t
   BL_TRY(check_ptr(W_packed));
   if (gamma == nullptr) return BL_ERR_INVALID_ARG;
   BL_TRY(check_ptr(Y));
-  const size_t need = bl_linear_workspace_bytes(M, K, N);
+  // Required: the quantised tokens; the rest of bl_linear_workspace_bytes (K
+  // ranges of under-filled tensor-core launches) is used when present.
+  const size_t need = M <= kGemvMaxTokens ? 0 : act_ws(M, K).total;
   if (need > 0) {
     if (workspace == nullptr || ws_bytes < need) return BL_ERR_WORKSPACE;
     BL_TRY(check_ptr(workspace));
@@ -910,7 +1009,7 @@ static bl_status linear_impl(const void* A, bl_dtype a_dtype, int64_t M, int64_t
   int32_t* rs = reinterpret_cast<int32_t*>(base + w.rowsum);
   BL_TRY(run_quant_acts(A, a_dtype, M, K, eps, Aq, gA, rs, st));
   BL_TRY(run_contract(Aq, W_packed, M, K, N, gamma, gA, rs, Y, kTcDequant, relu2 ? 1 : 0,
-                      y_dtype == BL_BF16, true, dev, sms, st));
+                      y_dtype == BL_BF16, true, dev, sms, st, base + w.total, ws_bytes - w.total));
   if (taps) {
     BL_TRY(tap_copy(taps->act_q, Aq, (size_t)M * K, st));
     BL_TRY(tap_copy(taps->act_gamma, gA, (size_t)M * 4, st));
@@ -943,7 +1042,10 @@ bl_status bl_linear(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
                       ws_bytes, 0u, stream);
 }
 
-size_t bl_ffn_workspace_bytes(int64_t M, int64_t K, int64_t H) { return ffn_ws(M, K, H).total; }
+size_t bl_ffn_workspace_bytes(int64_t M, int64_t K, int64_t H) {
+  const size_t up = tc2_ws_bytes(M, H, K), down = tc2_ws_bytes(M, K, H);
+  return ffn_ws(M, K, H).total + (up > down ? up : down);
+}
 
 static bl_status ffn_impl(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, int64_t H,
                           const uint8_t* W_up, const float* gamma_up, const uint8_t* W_down,
@@ -1012,13 +1114,15 @@ static bl_status ffn_impl(const void* X, bl_dtype x_dtype, int64_t M, int64_t K,
   BL_TRY(run_quant_acts(X, x_dtype, M, K, eps, Xq, gX, rsX, st));
   // Each contraction follows one of this call's own kernels, which write
   // neither W_up nor W_down: the weights may stream early (PDL).
+  void* split_ws = base + w.total;
+  const size_t split_bytes = ws_bytes - w.total;
   BL_TRY(run_contract(Xq, W_up, M, K, H, gamma_up, gX, rsX, acc_up, kTcRawI32, 0, 0, true, dev,
-                      sms, st));
+                      sms, st, split_ws, split_bytes));
   relu2_requant_kernel<<<(unsigned)M, kQuantThreads, 0, st>>>(acc_up, H, gX, gamma_up, eps, Rq, gR,
                                                               rsR);
   BL_CUDA(cudaGetLastError());
   BL_TRY(run_contract(Rq, W_down, M, H, K, gamma_down, gR, rsR, Y, kTcDequant, 0,
-                      y_dtype == BL_BF16, true, dev, sms, st));
+                      y_dtype == BL_BF16, true, dev, sms, st, split_ws, split_bytes));
   if (taps) {
     BL_TRY(tap_copy(taps->act_q, Xq, (size_t)M * K, st));
     BL_TRY(tap_copy(taps->act_gamma, gX, (size_t)M * 4, st));
@@ -1505,7 +1609,7 @@ extern "C" bl_status bl_linear_noalloc(const void* A, bl_dtype a_dtype, int64_t 
   if (gamma == nullptr) return BL_ERR_INVALID_ARG;
   BL_TRY(check_ptr(Y));
   // Scratch this call needs; refuse what the fixed array cannot hold.
-  const size_t need = bl_linear_workspace_bytes(M, K, N);
+  const size_t need = M <= kGemvMaxTokens ? 0 : act_ws(M, K).total;
   if (need > kNoAllocScratchBytes) return BL_ERR_WORKSPACE;
   int dev, sms;
   BL_TRY(current_device(&dev, &sms));

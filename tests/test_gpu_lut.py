@@ -47,7 +47,7 @@ def test_index_bytes_follow_figure(bl):
 
 
 @pytest.mark.parametrize("K,N,dt", [(2560, 6912, "bf16"), (4096, 1000, "f32"), (64, 33, "bf16"),
-                                    (11008, 4096, "bf16")])
+                                    (8192, 4096, "bf16")])
 def test_linear_lut(bl, K, N, dt):
     W = si.weights(N, K, seed=K % 97, dtype="bf16")
     codes, g = oracle.quant_weights(W.f32, EPS)
@@ -64,3 +64,15 @@ def test_linear_lut(bl, K, N, dt):
         assert torch.equal(Yl, Y2)
         assert_close(Yl.float().cpu().numpy(), oracle.bitlinear(A.f32, codes, g, EPS)["Y"],
                      out == torch.float32)
+
+
+def test_linear_lut_refuses_tables_beyond_shared_memory(bl):
+    """K = 11008 needs 2752 · 41 int16 table entries (220 KB) per token: more
+    than a CTA's shared memory next to its weights, so the call is refused."""
+    K, N = 11008, 256
+    widx = torch.zeros((N, K // 4), dtype=torch.uint8, device=DEV)
+    A = torch.zeros((1, K), dtype=torch.bfloat16, device=DEV)
+    g = torch.ones((1,), dtype=torch.float32, device=DEV)
+    with pytest.raises(bl.BitLinearError) as e:
+        bl.bl_linear_lut(A, widx, g, EPS)
+    assert e.value.status == 2

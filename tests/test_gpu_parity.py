@@ -208,6 +208,27 @@ def test_zero_gemm_worked_example(bl):
         assert np.all(acc.cpu().numpy() == -149)
 
 
+@pytest.mark.parametrize("M,K,N", [(256, 4096, 2048), (130, 1024, 640)])
+def test_zero_gemm_split_k(bl, M, K, N):
+    """Few output tiles: the tensor-core launch splits K into ranges whose INT32
+    partials the last range to finish sums; results must stay exact."""
+    Aq = random_int8(M, K, seed=M + 11)
+    codes = random_codes(N, K, seed=N + 13)
+    acc = bl.bl_zero_gemm(to_dev(Aq), to_dev(oracle.pack_ternary(codes))).cpu().numpy()
+    np.testing.assert_array_equal(acc, oracle.zero_gemm(Aq, codes))
+    # twice in a row: the arrival counters must be ready for the next launch
+    acc2 = bl.bl_zero_gemm(to_dev(Aq), to_dev(oracle.pack_ternary(codes))).cpu().numpy()
+    np.testing.assert_array_equal(acc2, acc)
+
+
+def test_linear_split_k_down_projection_shape(bl):
+    """512 tokens, K = 11008 → N = 4096 (the FFN down-projection's shape: 64
+    tiles, so K is split); sampled tokens × rows against the oracle."""
+    M, K, N = 512, 11008, 4096
+    _linear_case(bl, M, K, N, "bf16", "bf16", True, torch.bfloat16, seed=2,
+                 tok=[0, 1, 255, 256, 511], rows=list(range(0, 130)) + list(range(3990, 4096)))
+
+
 def test_zero_gemm_prefill_sampled(bl):
     """Full prefill size (2048 × 4096 × 4096) in the launch the benchmark
     uses; sampled tokens × rows checked against the oracle."""
