@@ -18,9 +18,10 @@
  *    in by the caller; its size comes from the matching *_workspace_bytes().
  *    For bl_zero_gemm, bl_linear_q, bl_linear and bl_ffn_relu2 part of that
  *    size is optional: with more than 64 tokens and too few output tiles to
- *    fill the SMs, the tensor-core contraction splits K into up to 4 ranges
- *    whose INT32 partials go there; a smaller workspace (down to the
- *    quantised tokens and row sums) gives the same results unsplit.
+ *    fill half of the SMs, the tensor-core contraction splits K into up to 4
+ *    ranges whose INT32 partials go there before one summing pass; a smaller
+ *    workspace (down to the quantised tokens and row sums) gives the same
+ *    results unsplit.
  *  * Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream) and makes no host synchronisation. Scales
  *    (γ, γ_A) are passed by device pointer for the same reason.

@@ -283,14 +283,14 @@ bl_status run_gemv(int src, int out, bl_dtype a_dtype, GemvParams p, bool pdl, i
 // Tensor-core launches.
 template <int BN, int OUT>
 bl_status launch_tc_t(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
-                      const TcParams& p, int dev, cudaStream_t st) {
+                      const TcParams& p, int splits, int dev, cudaStream_t st) {
   auto* k = tc_ternary_gemm_kernel<BN, OUT>;
   constexpr size_t smem = TcConfig<BN>::kSmemBytes;
   BL_TRY(ensure_smem(k, dev, smem));
   // Always with programmatic dependent launch: the kernel waits for the
   // previous grid before it touches global memory.
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((p.N + 127) / 128), (unsigned)((p.M + BN - 1) / BN));
+  cfg.gridDim = dim3((unsigned)((p.N + 127) / 128), (unsigned)((p.M + BN - 1) / BN), (unsigned)splits);
   cfg.blockDim = dim3(kTcThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -307,129 +307,74 @@ bl_status launch_tc_t(const CUtensorMap& ta, const CUtensorMap& tw, const CUtens
 // tokens take the skinny kernel).
 template <int OUT>
 bl_status launch_tc_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tw,
-                       const CUtensorMap& ty, const TcParams& p, int dev, cudaStream_t st) {
-  if (bn == 128) return launch_tc_t<128, OUT>(ta, tw, ty, p, dev, st);
-  return launch_tc_t<256, OUT>(ta, tw, ty, p, dev, st);
+                       const CUtensorMap& ty, const TcParams& p, int splits, int dev,
+                       cudaStream_t st) {
+  if (bn == 128) return launch_tc_t<128, OUT>(ta, tw, ty, p, splits, dev, st);
+  return launch_tc_t<256, OUT>(ta, tw, ty, p, splits, dev, st);
 }
 
 int tc_pick_bn(int64_t M) { return M <= 128 ? 128 : 256; }
 
 // ---------------------------------------------------------------------------
-// Persistent tensor-core kernel: K ranges per tile when the tiles alone fill at
-// most half of the SMs (each range at least 8 K blocks, at most 4 ranges).
-constexpr int kTc2WsSms = 148;  // B200: the SM count workspaces are sized for
+// K ranges for tensor-core launches whose tiles fill at most half of the SMs
+// (each range at least 8 K blocks, at most 4 ranges). The ranges write raw
+// INT32 partials to an optional workspace part; splitk_reduce_kernel sums
+// them (exact) and applies the epilogue.
+constexpr int kSplitWsSms = 148;  // B200: the SM count workspaces are sized for
 
-int tc2_splits(int64_t M, int64_t N, int64_t K, int sms) {
-  const int64_t tiles = ((N + 127) / 128) * ((M + kTc2BN - 1) / kTc2BN);
+int tc_splits(int64_t M, int64_t N, int64_t K, int sms) {
+  const int64_t tiles = ((N + 127) / 128) * ((M + tc_pick_bn(M) - 1) / tc_pick_bn(M));
   const int64_t KB = (K + kTcBK - 1) / kTcBK;
   if (tiles * 2 > sms) return 1;
   int64_t sp = sms / tiles;
   if (sp > 4) sp = 4;
-  int64_t most = KB / 8;
+  const int64_t most = KB / 8;
   if (sp > most) sp = most;
   return sp < 1 ? 1 : (int)sp;
 }
 
-size_t tc2_ws_bytes(int64_t M, int64_t N, int64_t K) {
+size_t tc_split_ws_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= kSkMaxTokens) return 0;
-  const int sp = tc2_splits(M, N, K, kTc2WsSms);
-  if (sp <= 1) return 0;
-  const int64_t tiles = ((N + 127) / 128) * ((M + kTc2BN - 1) / kTc2BN);
-  return align_up((size_t)sp * M * N * 4) + align_up((size_t)tiles * 4);
-}
-
-// pdl: launch with programmatic dependent launch (not after a memset).
-template <int OUT>
-bl_status launch_tc2_t(const CUtensorMap& ta, const CUtensorMap& tw, const Tc2Params& p, int grid,
-                       bool pdl, int dev, cudaStream_t st) {
-  auto* k = tc_persistent_kernel<OUT>;
-  constexpr size_t smem = Tc2::kSmem;
-  BL_TRY(ensure_smem(k, dev, smem));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kTc2Threads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  BL_CUDA(cudaLaunchKernelEx(&cfg, k, ta, tw, p));
-  return BL_OK;
-}
-
-// acc/Y[M,N] = epilogue(A_q[M,K] · W_q[N,K]ᵀ − rowsum), persistent CTAs.
-// split_ws: optional scratch of tc2_ws_bytes(M, N, K) bytes for K ranges.
-bl_status run_tc2(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,
-                  const float* gamma, const float* gammaA, const int32_t* rowsum, void* Y, int out,
-                  int relu2, int y_bf16, void* split_ws, size_t split_ws_bytes, int dev, int sms,
-                  cudaStream_t st) {
-  if (M > 0x7FFFFFFF || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
-  CUtensorMap ta, tw;
-  BL_TRY(make_map_u8(&ta, Aq, (uint64_t)M, (uint64_t)K, kTcBK, (uint32_t)kTc2BN,
-                     CU_TENSOR_MAP_SWIZZLE_128B));
-  BL_TRY(make_map_u8(&tw, Wp, (uint64_t)N, (uint64_t)(K / 4), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B));
-  Tc2Params p = {};
-  p.gamma = gamma;
-  p.gammaA = gammaA;
-  p.rowsum = rowsum;
-  p.Y = Y;
-  p.M = M;
-  p.N = N;
-  p.K = K;
-  p.relu2 = relu2;
-  p.y_bf16 = y_bf16;
-  p.tiles_n = (int)((N + 127) / 128);
-  p.tiles = p.tiles_n * (int)((M + kTc2BN - 1) / kTc2BN);
-  const int KB = (int)((K + kTcBK - 1) / kTcBK);
-  int sp = tc2_splits(M, N, K, sms);
-  const int sp_ws = tc2_splits(M, N, K, kTc2WsSms);
-  if (sp > sp_ws) sp = sp_ws;
-  if (sp > 1 && (split_ws == nullptr || split_ws_bytes < tc2_ws_bytes(M, N, K))) sp = 1;
-  p.splits = sp;
-  p.kb_per_split = ((KB + sp - 1) / sp + 3) / 4 * 4;
-  p.splits = (KB + p.kb_per_split - 1) / p.kb_per_split;  // no empty ranges
-  if (p.splits > 1) {
-    uint8_t* base = reinterpret_cast<uint8_t*>(split_ws);
-    p.part = reinterpret_cast<int32_t*>(base);
-    p.counter = reinterpret_cast<int32_t*>(base + align_up((size_t)p.splits * M * N * 4));
-    BL_CUDA(cudaMemsetAsync(p.counter, 0, (size_t)p.tiles * 4, st));
-  }
-  const int items = p.tiles * p.splits;
-  const int grid = items < sms ? items : sms;
-  // After the counters' memset the launch is ordered normally.
-  const bool pdl = p.splits == 1;
-  return out == kTcDequant ? launch_tc2_t<kTcDequant>(ta, tw, p, grid, pdl, dev, st)
-                           : launch_tc2_t<kTcRawI32>(ta, tw, p, grid, pdl, dev, st);
+  const int sp = tc_splits(M, N, K, kSplitWsSms);
+  return sp > 1 ? align_up((size_t)sp * M * N * 4) : 0;
 }
 
 // acc/Y[M,N] = epilogue(A_q[M,K] · W_q[N,K]ᵀ − rowsum).
 bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,
                  const float* gamma, const float* gammaA, const int32_t* rowsum, void* Y,
-                 int out, int relu2, int y_bf16, int dev, cudaStream_t st) {
+                 int out, int relu2, int y_bf16, void* split_ws, size_t split_ws_bytes, int dev,
+                 int sms, cudaStream_t st) {
   if (M > 0x7FFFFFFF || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
   const int bn = tc_pick_bn(M);
+  const int KBall = (int)((K + kTcBK - 1) / kTcBK);
+  int sp = tc_splits(M, N, K, sms);
+  const int sp_ws = tc_splits(M, N, K, kSplitWsSms);
+  if (sp > sp_ws) sp = sp_ws;
+  if (sp > 1 && (split_ws == nullptr || split_ws_bytes < tc_split_ws_bytes(M, N, K))) sp = 1;
+  const int kbs = sp > 1 ? ((KBall + sp - 1) / sp + 3) / 4 * 4 : KBall;
+  if (sp > 1) sp = (KBall + kbs - 1) / kbs;  // no empty ranges
+  void* Yk = sp > 1 ? split_ws : Y;        // where the kernel writes
+  const int outk = sp > 1 ? kTcRawI32 : out;
   CUtensorMap ta, tw;
   BL_TRY(make_map_u8(&ta, Aq, (uint64_t)M, (uint64_t)K, kTcBK, (uint32_t)bn,
                      CU_TENSOR_MAP_SWIZZLE_128B));
   BL_TRY(make_map_u8(&tw, Wp, (uint64_t)N, (uint64_t)(K / 4), 128, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B));
   // Output tensor map for the staged tensor-store epilogue (rows of N
-  // elements must be a multiple of 16 bytes).
-  const int esz = (out == kTcRawI32 || !y_bf16) ? 4 : 2;
+  // elements must be a multiple of 16 bytes); split partials are [sp·M, N].
+  const int esz = (outk == kTcRawI32 || !y_bf16) ? 4 : 2;
   CUtensorMap ty;
   std::memset(&ty, 0, sizeof(ty));
   int tma_store = 0;
   if (((uint64_t)N * esz) % 16 == 0) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return BL_ERR_CUDA;
-    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M * (cuuint64_t)sp};
     cuuint64_t strides[1] = {(cuuint64_t)N * esz};
     cuuint32_t box[2] = {128, (cuuint32_t)(bn < 32 ? bn : 32)};  // stored 32 tokens at a time
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&ty, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32,
-                     2, Y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     2, Yk, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return BL_ERR_CUDA;
@@ -440,14 +385,25 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
   p.gamma = gamma;
   p.gammaA = gammaA;
   p.rowsum = rowsum;
-  p.Y = Y;
+  p.Y = Yk;
   p.M = M;
   p.N = N;
   p.K = K;
   p.relu2 = relu2;
   p.y_bf16 = y_bf16;
-  return out == kTcDequant ? launch_tc_bn<kTcDequant>(bn, ta, tw, ty, p, dev, st)
-                           : launch_tc_bn<kTcRawI32>(bn, ta, tw, ty, p, dev, st);
+  p.kb_per_split = kbs;
+  BL_TRY(outk == kTcDequant ? launch_tc_bn<kTcDequant>(bn, ta, tw, ty, p, sp, dev, st)
+                            : launch_tc_bn<kTcRawI32>(bn, ta, tw, ty, p, sp, dev, st));
+  if (sp == 1) return BL_OK;
+  const int64_t total = M * N;
+  int64_t blocks = (total / 4 + 255) / 256;
+  if (blocks > 16 * (int64_t)sms) blocks = 16 * (int64_t)sms;
+  if (blocks < 1) blocks = 1;
+  splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, st>>>(
+      reinterpret_cast<const int32_t*>(Yk), sp, M, N, out == kTcRawI32 ? 1 : 0, gamma, gammaA,
+      relu2, Y, y_bf16);
+  BL_CUDA(cudaGetLastError());
+  return BL_OK;
 }
 
 // --------------------------------------------------------------------------
@@ -580,7 +536,7 @@ bl_status run_skinny(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, 
 }
 
 // Contraction of pre-quantised tokens: the skinny kernel up to 64 tokens,
-// persistent tensor-core CTAs above. out: kTcDequant or kTcRawI32.
+// tensor-core tiles above. out: kTcDequant or kTcRawI32.
 // split_ws: optional scratch (tc2_ws_bytes) that lets under-filled tensor-core
 // launches split K.
 bl_status run_contract(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,
@@ -590,8 +546,8 @@ bl_status run_contract(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K
   if (M <= kSkMaxTokens)
     return run_skinny(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out == kTcRawI32 ? 1 : 0, relu2,
                       y_bf16, pdl, dev, sms, st);
-  return run_tc2(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out, relu2, y_bf16, split_ws,
-                 split_ws_bytes, dev, sms, st);
+  return run_tc(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out, relu2, y_bf16, split_ws,
+                split_ws_bytes, dev, sms, st);
 }
 
 bl_status run_quant_acts(const void* A, bl_dtype dt, int64_t M, int64_t K, float eps, int8_t* Aq,
@@ -852,7 +808,7 @@ bl_status bl_quant_acts(const void* A, bl_dtype a_dtype, int64_t M, int64_t K, f
 
 size_t bl_zero_gemm_workspace_bytes(int64_t M, int64_t K, int64_t N) {
   if (M <= kGemvMaxTokens) return 0;
-  return align_up((size_t)M * 4) + tc2_ws_bytes(M, N, K);
+  return align_up((size_t)M * 4) + tc_split_ws_bytes(M, N, K);
 }
 
 bl_status bl_zero_gemm(const int8_t* A_q, int64_t M, int64_t K, const uint8_t* W_packed,
@@ -896,7 +852,7 @@ bl_status bl_zero_gemm(const int8_t* A_q, int64_t M, int64_t K, const uint8_t* W
 
 size_t bl_linear_q_workspace_bytes(int64_t M, int64_t K, int64_t N) {
   if (M <= kGemvMaxTokens) return 0;
-  return align_up((size_t)M * 4) + tc2_ws_bytes(M, N, K);
+  return align_up((size_t)M * 4) + tc_split_ws_bytes(M, N, K);
 }
 
 bl_status bl_linear_q(const int8_t* A_q, const float* gamma_A, const int32_t* rowsum, int64_t M,
@@ -957,7 +913,7 @@ bl_status bl_linear_q(const int8_t* A_q, const float* gamma_A, const int32_t* ro
 
 size_t bl_linear_workspace_bytes(int64_t M, int64_t K, int64_t N) {
   if (M <= kGemvMaxTokens) return 0;
-  return act_ws(M, K).total + tc2_ws_bytes(M, N, K);
+  return act_ws(M, K).total + tc_split_ws_bytes(M, N, K);
 }
 
 static bl_status linear_impl(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
@@ -1043,7 +999,7 @@ bl_status bl_linear(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
 }
 
 size_t bl_ffn_workspace_bytes(int64_t M, int64_t K, int64_t H) {
-  const size_t up = tc2_ws_bytes(M, H, K), down = tc2_ws_bytes(M, K, H);
+  const size_t up = tc_split_ws_bytes(M, H, K), down = tc_split_ws_bytes(M, K, H);
   return ffn_ws(M, K, H).total + (up > down ? up : down);
 }
 
