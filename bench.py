@@ -320,6 +320,77 @@ def run_decode(bl, device, steps, warmup, peaks, world):
             lat.append(s.elapsed_time(e) * 1e3)
     res["single_call_us_median"] = statistics.median(lat[3:])
     del graph
+
+    # Floor of a dependent chain with the same launch shape: empty kernels
+    # (launch_dependents + wait only), 1000 per graph.
+    def floor_chain():
+        for _ in range(CALLS_PER_STEP):
+            bl.bl_probe_pdl_floor(M, K, N, stream=stream)
+    fg = capture(floor_chain, stream)
+    for _ in range(3):
+        fg.replay()
+    tf = time_graph(fg, stream, max(3, min(steps, 50)))
+    res["floor_us"] = tf / (max(3, min(steps, 50)) * CALLS_PER_STEP) * 1e6
+    del fg
+    res["pool_list"] = pool
+    res["gamma"] = gamma
+    res["tok"] = tok
+    return res
+
+
+def run_decode_storage_variants(bl, device, dec, peaks, reps=5):
+    """The decode chain of the headline on the other two weight storages:
+    radix-3 (5 weights per byte) and lookup-table index bytes. Same tokens,
+    same matrices (converted), 1000 chained calls with PDL."""
+    import torch
+    M, K, N = DECODE["M"], DECODE["K"], DECODE["N"]
+    stream = torch.cuda.Stream(device)
+    pool, gamma, tok = dec["pool_list"], dec["gamma"], dec["tok"]
+    Y = torch.empty((CALLS_PER_STEP, N), dtype=torch.bfloat16, device=device)
+    out = {}
+    r3 = [bl.bl_pack_radix3(w, K) for w in pool]
+    lut = [bl.bl_pack_lut_index(w) for w in pool]
+    torch.cuda.synchronize()
+    rb = r3[0].shape[1]
+    for name, mats, call, wbytes in (
+            ("radix3", r3, bl.bl_linear_radix3, N * rb),
+            ("lut_index", lut, bl.bl_linear_lut, N * K // 4)):
+        def chain():
+            for i in range(CALLS_PER_STEP):
+                call(tok[i:i + 1], mats[i % len(mats)], gamma, EPS, out=Y[i:i + 1], pdl=True,
+                     stream=stream)
+        g = capture(chain, stream)
+        for _ in range(3):
+            g.replay()
+        t = time_graph(g, stream, reps) / (reps * CALLS_PER_STEP)
+        alg = wbytes + M * K * 2 + M * N * 2
+        out[name] = {"us_per_call": t * 1e6, "tokens_per_s": M / t, "weight_bytes": wbytes,
+                     "gbs": alg / t / 1e9, "hbm_frac": alg / t / 1e9 / peaks["hbm_gbs"]}
+        del g
+    del r3, lut
+    return out
+
+
+def run_ste(bl, device, peaks, reps=10):
+    """STE backward at the prefill shape (2048 tokens, 4096 → 4096): dA and dW,
+    each 2·M·N·K flops on the bf16 tensor cores (layout kernels included)."""
+    import torch
+    M, N, K = 2048, 4096, 4096
+    stream = torch.cuda.Stream(device)
+    W = si.weights(N, K, seed=0, dtype="bf16").torch(device)
+    packed, gamma = bl.bl_quant_weights(W, EPS)
+    A = si.activations(M, K, seed=0, dtype="bf16").torch(device)
+    Aq, gA, _ = bl.bl_quant_acts(A, EPS)
+    dY = si.activations(M, N, seed=5, dtype="bf16").torch(device)
+    torch.cuda.synchronize()
+    flops = 2.0 * M * N * K
+    res = {"workload": "dY [2048, 4096] bf16; W 4096x4096; A_q [2048, 4096]; fp32 gradients"}
+    for name, fn in (("grad_input", lambda: bl.bl_ste_grad_input(dY, packed, gamma, stream=stream)),
+                     ("grad_weight", lambda: bl.bl_ste_grad_weight(dY, Aq, gA, W, gamma, EPS,
+                                                                   stream=stream))):
+        t = rotating_time([fn], stream, reps)
+        res[name] = {"us": t * 1e6, "tflops": flops / t / 1e12,
+                     "frac_of_bf16_peak": flops / t / 1e12 / peaks["bf16_tflops"]}
     return res
 
 
@@ -579,6 +650,51 @@ def run_reference(args):
 
 # ---------------------------------------------------------------------------
 
+# ---------------------------------------------------------------------------
+# Small cases for ncu captures (one kernel each; the summaries under profiles/
+# name these commands).
+
+def profile_case(name: str) -> int:
+    import torch
+    import ternary_weight_linear_absmax_b200 as bl
+    bl.load()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    st = torch.cuda.Stream(device)
+    if name in ("decode", "decode_radix3"):
+        # 20 chained decode calls (1 token, 2560 -> 6912) over 6 distinct matrices
+        K, N = DECODE["K"], DECODE["N"]
+        mats = []
+        for i in range(6):
+            pk, g = bl.bl_quant_weights(si.weights(N, K, seed=i, dtype="bf16").torch(device), EPS)
+            mats.append((bl.bl_pack_radix3(pk, K) if name == "decode_radix3" else pk, g))
+        tok = si.activations(20, K, seed=0, dtype="bf16").torch(device)
+        call = bl.bl_linear_radix3 if name == "decode_radix3" else bl.bl_linear
+        torch.cuda.synchronize()
+        for i in range(20):
+            w, g = mats[i % 6]
+            call(tok[i:i + 1], w, g, EPS, pdl=True, stream=st)
+    elif name in ("skinny", "prefill"):
+        M, K, N = (16, 4096, 11008) if name == "skinny" else (2048, 4096, 4096)
+        pk, g = bl.bl_quant_weights(si.weights(N, K, seed=0, dtype="bf16").torch(device), EPS)
+        Aq, gA, rs = bl.bl_quant_acts(si.activations(M, K, seed=0, dtype="bf16").torch(device), EPS)
+        torch.cuda.synchronize()
+        for _ in range(3):
+            bl.bl_linear_q(Aq, gA, pk, g, rowsum=rs, stream=st)
+    elif name == "ste":
+        M, N, K = 2048, 4096, 4096
+        W = si.weights(N, K, seed=0, dtype="bf16").torch(device)
+        pk, g = bl.bl_quant_weights(W, EPS)
+        dY = si.activations(M, N, seed=5, dtype="bf16").torch(device)
+        torch.cuda.synchronize()
+        for _ in range(2):
+            bl.bl_ste_grad_input(dY, pk, g, stream=st)
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    st.synchronize()
+    return int(bl.bl_check_device_error(st))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -587,7 +703,11 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--profile-case", choices=["decode", "decode_radix3", "skinny", "prefill", "ste"],
+                    help="run one small case for an ncu capture and exit")
     args = ap.parse_args(argv)
+    if args.profile_case:
+        return profile_case(args.profile_case)
     if args.impl == "reference":
         return run_reference(args)
     args.warmup = max(3, args.warmup)
@@ -614,6 +734,8 @@ def main(argv=None):
         extra["prefill"] = run_prefill(bl, device, peaks)
         extra["ffn"] = run_ffn(bl, device, peaks)
         extra["quant_weights"] = run_quant_weights(bl, device)
+        extra["decode_storage_variants"] = run_decode_storage_variants(bl, device, dec, peaks)
+        extra["ste_backward"] = run_ste(bl, device, peaks)
     cpu = None
     if rank == 0 and ws == 1:
         rate, n, cores = oracle_decode_rate(seconds=args.cpu_seconds)
@@ -649,6 +771,8 @@ def main(argv=None):
                      "unit": "GB/s", "frac": dec["achieved_gbs"] / peaks["hbm_gbs"],
                      "traffic": traffic, "kernel": "gemv_ternary_kernel",
                      "alg_bytes_per_launch": dec["alg_bytes"], "launch_us": dec["launch_us"],
+                     "chain_floor_us": dec["floor_us"],
+                     "above_floor_us": dec["launch_us"] - dec["floor_us"],
                      "peak_source": f"{peaks['source']} hbm_gbs"},
         "cpu_baseline": cpu,
         "e2e": dec["e2e"],

@@ -404,6 +404,14 @@ bl_status bl_ste_grad_weight(const void* dY, bl_dtype dy_dtype, int64_t M, int64
  */
 bl_status bl_check_device_error(bl_stream_t stream);
 
+/* Measurement aid (no counterpart on the pages): launches one empty kernel
+ * with exactly the launch shape bl_linear_ex uses for a decode call of
+ * (M ≤ bl_gemv_max_tokens(), K, N) — grid, 512 threads, dynamic shared
+ * memory, programmatic dependent launch — that only releases its dependents
+ * and waits for the previous kernel. A chain of these is the launch-to-launch
+ * floor of a dependent decode chain; the GEMV's time above it is its own. */
+bl_status bl_probe_pdl_floor(int64_t M, int64_t K, int64_t N, bl_stream_t stream);
+
 /* Self-test of the bounded-wait machinery: launches one tiny kernel that
  * waits on a shared-memory barrier nothing will ever complete, giving up
  * after `limit_ns` nanoseconds (1e3 .. 1e9), which raises the device error

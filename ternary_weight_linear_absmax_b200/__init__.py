@@ -24,7 +24,8 @@ __all__ = [
     "bl_quant_weights", "bl_quant_acts", "bl_zero_gemm", "bl_linear_q", "bl_linear",
     "bl_linear_noalloc", "bl_ffn_relu2", "bl_linear_taps", "bl_ffn_relu2_taps",
     "bl_ffn_tp_up", "bl_ffn_tp_down", "bl_dequant_i32", "bl_ste_grad_input", "bl_ste_grad_weight",
-    "bl_pack_radix3", "bl_linear_radix3", "bl_pack_lut_index", "bl_linear_lut", "bl_check_device_error", "bl_selftest_wait_timeout",
+    "bl_pack_radix3", "bl_linear_radix3", "bl_pack_lut_index", "bl_linear_lut",
+    "bl_probe_pdl_floor", "bl_check_device_error", "bl_selftest_wait_timeout",
     "bl_gemv_max_tokens", "workspace_bytes", "BitLinearError", "load", "BL_FLAG_PDL",
 ]
 
@@ -406,6 +407,11 @@ def bl_ste_grad_weight(dY, A_q, gamma_A, W, gamma, eps: float = 1e-5, *, stream=
                                float(eps), dW.data_ptr(), _ptr(ws), _nbytes(ws), _stream(stream)),
           "bl_ste_grad_weight")
     return dW
+
+
+def bl_probe_pdl_floor(M: int, K: int, N: int, *, stream=None) -> None:
+    """One empty kernel with the decode GEMV's launch shape for (M, K, N)."""
+    check(load().bl_probe_pdl_floor(M, K, N, _stream(stream)), "bl_probe_pdl_floor")
 
 
 def bl_check_device_error(stream=None) -> int:

@@ -77,6 +77,7 @@ SIGNATURES = {
     "bl_ste_grad_weight_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_ste_grad_weight": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _i64, _vp, _int, _vp, _f32,
                                   _vp, _vp, _sz, _vp]),
+    "bl_probe_pdl_floor": (_int, [_i64, _i64, _i64, _vp]),
     "bl_check_device_error": (_int, [_vp]),
     "bl_selftest_wait_timeout": (_int, [_i64, _vp]),
 }

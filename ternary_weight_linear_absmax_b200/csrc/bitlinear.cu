@@ -333,10 +333,16 @@ int tc_splits(int64_t M, int64_t N, int64_t K, int sms) {
   return sp < 1 ? 1 : (int)sp;
 }
 
+// Rows per split in the partial buffer: M rounded up to the token tile.
+int64_t tc_split_rows(int64_t M) {
+  const int bn = tc_pick_bn(M);
+  return (M + bn - 1) / bn * bn;
+}
+
 size_t tc_split_ws_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= kSkMaxTokens) return 0;
   const int sp = tc_splits(M, N, K, kSplitWsSms);
-  return sp > 1 ? align_up((size_t)sp * M * N * 4) : 0;
+  return sp > 1 ? align_up((size_t)sp * tc_split_rows(M) * N * 4) : 0;
 }
 
 // acc/Y[M,N] = epilogue(A_q[M,K] · W_q[N,K]ᵀ − rowsum).
@@ -369,7 +375,7 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
   if (((uint64_t)N * esz) % 16 == 0) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return BL_ERR_CUDA;
-    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M * (cuuint64_t)sp};
+    cuuint64_t dims[2] = {(cuuint64_t)N, sp > 1 ? (cuuint64_t)(tc_split_rows(M) * sp) : (cuuint64_t)M};
     cuuint64_t strides[1] = {(cuuint64_t)N * esz};
     cuuint32_t box[2] = {128, (cuuint32_t)(bn < 32 ? bn : 32)};  // stored 32 tokens at a time
     cuuint32_t estr[2] = {1, 1};
@@ -392,6 +398,7 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
   p.relu2 = relu2;
   p.y_bf16 = y_bf16;
   p.kb_per_split = kbs;
+  p.split_rows = sp > 1 ? tc_split_rows(M) : 0;
   BL_TRY(outk == kTcDequant ? launch_tc_bn<kTcDequant>(bn, ta, tw, ty, p, sp, dev, st)
                             : launch_tc_bn<kTcRawI32>(bn, ta, tw, ty, p, sp, dev, st));
   if (sp == 1) return BL_OK;
@@ -400,8 +407,8 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
   if (blocks > 16 * (int64_t)sms) blocks = 16 * (int64_t)sms;
   if (blocks < 1) blocks = 1;
   splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, st>>>(
-      reinterpret_cast<const int32_t*>(Yk), sp, M, N, out == kTcRawI32 ? 1 : 0, gamma, gammaA,
-      relu2, Y, y_bf16);
+      reinterpret_cast<const int32_t*>(Yk), sp, tc_split_rows(M) * N, M, N,
+      out == kTcRawI32 ? 1 : 0, gamma, gammaA, relu2, Y, y_bf16);
   BL_CUDA(cudaGetLastError());
   return BL_OK;
 }
@@ -1600,6 +1607,16 @@ extern "C" bl_status bl_linear_noalloc(const void* A, bl_dtype a_dtype, int64_t 
 
 namespace bl {
 namespace {
+// Measurement aid: the decode GEMV's launch (grid, 512 threads, dynamic
+// shared memory, programmatic dependent launch) with no work, so a chain of
+// it shows the launch-to-launch floor of a dependent chain.
+__global__ void __launch_bounds__(kGemvThreads, 2) pdl_floor_kernel() {
+  extern __shared__ uint8_t smem_unused[];
+  (void)smem_unused;
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();
+}
+
 __global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
@@ -1611,6 +1628,30 @@ __global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns) {
 }
 }  // namespace
 }  // namespace bl
+
+extern "C" bl_status bl_probe_pdl_floor(int64_t M, int64_t K, int64_t N, bl_stream_t stream) {
+  BL_TRY(check_k(K));
+  BL_TRY(check_rows(N));
+  if (M < 1 || M > kGemvMaxTokens || N == 0) return BL_ERR_SHAPE;
+  int dev, sms;
+  BL_TRY(current_device(&dev, &sms));
+  int rows, grid;
+  size_t smem;
+  BL_TRY(bl::gemv_plan(N, K, (int)M, sms, &rows, &grid, &smem));
+  BL_TRY(bl::ensure_smem(bl::pdl_floor_kernel, dev, smem));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(bl::kGemvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  BL_CUDA(cudaLaunchKernelEx(&cfg, bl::pdl_floor_kernel));
+  return BL_OK;
+}
 
 extern "C" bl_status bl_selftest_wait_timeout(int64_t limit_ns, bl_stream_t stream) {
   if (limit_ns < 1000 || limit_ns > 1000000000) return BL_ERR_INVALID_ARG;

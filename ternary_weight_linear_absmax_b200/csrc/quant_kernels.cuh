@@ -348,19 +348,20 @@ dequant_i32_kernel(const int32_t* __restrict__ acc, const float* __restrict__ ga
   }
 }
 
-// Sum of the INT32 partials of a K-split contraction ([splits, M, N]; split
-// 0 already subtracted the row sums), then the epilogue: raw INT32, or
-// y = v · ((γ_A·γ)/127) in fp32 (ReLU² optional) as fp32/bf16.
+// Sum of the INT32 partials of a K-split contraction (split z at
+// part + z·stride, rows of N; split 0 already subtracted the row sums), then
+// the epilogue: raw INT32, or y = v · ((γ_A·γ)/127) in fp32 (ReLU² optional)
+// as fp32/bf16.
 __global__ void __launch_bounds__(256)
-splitk_reduce_kernel(const int32_t* __restrict__ part, int splits, int64_t M, int64_t N, int raw,
-                     const float* __restrict__ gamma, const float* __restrict__ gammaA, int relu2,
-                     void* Y, int y_bf16) {
+splitk_reduce_kernel(const int32_t* __restrict__ part, int splits, int64_t stride, int64_t M,
+                     int64_t N, int raw, const float* __restrict__ gamma,
+                     const float* __restrict__ gammaA, int relu2, void* Y, int y_bf16) {
   const int64_t total = M * N;
   const float g = raw ? 0.0f : __ldg(gamma);
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
     int v = 0;
-    for (int z = 0; z < splits; ++z) v += __ldg(part + (int64_t)z * total + i);
+    for (int z = 0; z < splits; ++z) v += __ldg(part + (int64_t)z * stride + i);
     if (raw) {
       reinterpret_cast<int32_t*>(Y)[i] = v;
       continue;

@@ -53,8 +53,11 @@ struct TcParams {
                   //    writes it with tensor stores of 32 tokens through tm_y (needs
                   //    N·element bytes % 16 == 0)
   int kb_per_split;  // K blocks per blockIdx.z (a multiple of 4); all of K when unsplit.
-                     // Split z writes raw INT32 partials to rows [z·M, z·M + M) of Y
-                     // (only split 0 subtracts the row sums).
+                     // Split z writes raw INT32 partials to rows [z·Mp, z·Mp + M) of Y,
+                     // Mp = M rounded up to the token tile, so a tile's rows past M
+                     // (stored whole by the tensor stores) stay in z's own padding.
+                     // Only split 0 subtracts the row sums.
+  int64_t split_rows;  // Mp (0 when unsplit)
 };
 
 template <int BN>
@@ -267,7 +270,7 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
   const int KBall = (int)((p.K + kTcBK - 1) / kTcBK);
   const int kb_lo = (int)blockIdx.z * p.kb_per_split;
   const int KB = min(KBall, kb_lo + p.kb_per_split) - kb_lo;
-  const int64_t zrow = (int64_t)blockIdx.z * p.M;  // output row offset of this split
+  const int64_t zrow = (int64_t)blockIdx.z * p.split_rows;  // output row offset of this split
 
   if (tid == 0) {
     for (int s = 0; s < SS; ++s) {

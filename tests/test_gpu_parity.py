@@ -208,10 +208,12 @@ def test_zero_gemm_worked_example(bl):
         assert np.all(acc.cpu().numpy() == -149)
 
 
-@pytest.mark.parametrize("M,K,N", [(256, 4096, 2048), (130, 1024, 640)])
+@pytest.mark.parametrize("M,K,N", [(256, 4096, 2048), (300, 2560, 640)])
 def test_zero_gemm_split_k(bl, M, K, N):
     """Few output tiles: the tensor-core launch splits K into ranges whose INT32
-    partials the last range to finish sums; results must stay exact."""
+    partials a second pass sums; results must stay exact, also when M is not a
+    multiple of the token tile (300: the last tile's rows past M must not
+    reach the next range's partials)."""
     Aq = random_int8(M, K, seed=M + 11)
     codes = random_codes(N, K, seed=N + 13)
     acc = bl.bl_zero_gemm(to_dev(Aq), to_dev(oracle.pack_ternary(codes))).cpu().numpy()
