@@ -409,7 +409,7 @@ def run_small_batch(bl, device, peaks, reps=200):
 
     def chain():
         for i in range(calls):
-            bl.bl_linear(A, pool[i], gamma, EPS, out=Y, workspace=ws, stream=stream)
+            bl.bl_linear(A, pool[i], gamma, EPS, out=Y, workspace=ws, pdl=True, stream=stream)
 
     g = capture(chain, stream)
     for _ in range(3):
@@ -417,7 +417,8 @@ def run_small_batch(bl, device, peaks, reps=200):
     t = time_graph(g, stream, max(1, reps // calls)) / max(1, reps // calls) / calls
     alg = N * K // 4 + M * K * 2 + M * N * 2
     del g
-    return {"workload": "16 tokens, K=4096 -> N=11008, bf16, rotating weight pool > L2",
+    return {"workload": "16 tokens, K=4096 -> N=11008, bf16, rotating weight pool > L2, "
+                        "chained calls with programmatic dependent launch",
             "tokens_per_s": M / t, "us_per_call": t * 1e6,
             "gbs": alg / t / 1e9, "hbm_frac": alg / t / 1e9 / peaks["hbm_gbs"],
             "tops": 2.0 * M * N * K / t / 1e12}

@@ -87,7 +87,11 @@ enum {
    * stream, and lets the next kernel start early. Only valid when the weight
    * buffer was NOT written by the kernel immediately preceding this call on
    * `stream` (true for a decode chain over static weights). Activations and
-   * outputs are still ordered after the previous kernel. */
+   * outputs are still ordered after the previous kernel. Above
+   * bl_gemv_max_tokens() tokens the flag makes the activation quantiser
+   * launch early too (it waits for the previous kernel before touching
+   * memory), so the contraction's CTAs can stream their weights during the
+   * previous call. */
   BL_FLAG_PDL = 1,
   /* bl_linear_radix3 / bl_linear_lut only: Y is the raw INT32
    * accumulator [M, N]. */
@@ -179,7 +183,7 @@ bl_status bl_linear_q(const int8_t* A_q, const float* gamma_A,
  * early (the quantiser does not write it).
  *   A [M, K] fp32/bf16; W_packed [N, K/4]; gamma 1 fp32; Y [M, N] fp32/bf16.
  *   workspace ≥ bl_linear_workspace_bytes(M, K, N) (may be 0 → NULL ok).
- * bl_linear_ex adds `flags` (BL_FLAG_PDL; only honoured on the GEMV path).
+ * bl_linear_ex adds `flags` (BL_FLAG_PDL).
  */
 size_t bl_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
 bl_status bl_linear(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,

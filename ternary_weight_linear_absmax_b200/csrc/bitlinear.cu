@@ -417,8 +417,11 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
 // Skinny launches (5 ≤ M ≤ 64 tokens, mma.sync over all SMs).
 template <int MTT, int NTW, int KPS>
 bl_status launch_skinny_t(const CUtensorMap& tw, const CUtensorMap& ta, const SkinnyParams& p,
-                          int grid, size_t smem, bool pdl, int dev, cudaStream_t st) {
-  auto* k = skinny_ternary_kernel<MTT, NTW, KPS>;
+                          int grid, size_t smem, bool pdl, bool res, int dev, cudaStream_t st) {
+  auto* k = skinny_ternary_kernel<MTT, NTW, KPS, false>;
+  if constexpr (MTT <= 2) {
+    if (res) k = skinny_ternary_kernel<MTT, NTW, KPS, true>;
+  }
   BL_TRY(ensure_smem(k, dev, smem));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -443,22 +446,22 @@ constexpr SkinnySplit kSkSplits[] = {{1, 2}, {2, 2}, {3, 2}, {5, 2}, {2, 4}, {3,
 
 template <int MTT>
 bl_status launch_skinny_split(SkinnySplit sp, const CUtensorMap& tw, const CUtensorMap& ta,
-                              const SkinnyParams& p, int grid, size_t smem, bool pdl, int dev,
-                              cudaStream_t st) {
+                              const SkinnyParams& p, int grid, size_t smem, bool pdl, bool res,
+                              int dev, cudaStream_t st) {
   if (sp.kps == 2) {
     switch (sp.ntw) {
-      case 1: return launch_skinny_t<MTT, 1, 2>(tw, ta, p, grid, smem, pdl, dev, st);
-      case 2: return launch_skinny_t<MTT, 2, 2>(tw, ta, p, grid, smem, pdl, dev, st);
-      case 3: return launch_skinny_t<MTT, 3, 2>(tw, ta, p, grid, smem, pdl, dev, st);
+      case 1: return launch_skinny_t<MTT, 1, 2>(tw, ta, p, grid, smem, pdl, res, dev, st);
+      case 2: return launch_skinny_t<MTT, 2, 2>(tw, ta, p, grid, smem, pdl, res, dev, st);
+      case 3: return launch_skinny_t<MTT, 3, 2>(tw, ta, p, grid, smem, pdl, res, dev, st);
       default:
-        if constexpr (MTT <= 2) return launch_skinny_t<MTT, 5, 2>(tw, ta, p, grid, smem, pdl, dev, st);
+        if constexpr (MTT <= 2) return launch_skinny_t<MTT, 5, 2>(tw, ta, p, grid, smem, pdl, res, dev, st);
         return BL_ERR_SHAPE;
     }
   }
   switch (sp.ntw) {
-    case 2: return launch_skinny_t<MTT, 2, 4>(tw, ta, p, grid, smem, pdl, dev, st);
-    case 3: return launch_skinny_t<MTT, 3, 4>(tw, ta, p, grid, smem, pdl, dev, st);
-    default: return launch_skinny_t<MTT, 4, 4>(tw, ta, p, grid, smem, pdl, dev, st);
+    case 2: return launch_skinny_t<MTT, 2, 4>(tw, ta, p, grid, smem, pdl, res, dev, st);
+    case 3: return launch_skinny_t<MTT, 3, 4>(tw, ta, p, grid, smem, pdl, res, dev, st);
+    default: return launch_skinny_t<MTT, 4, 4>(tw, ta, p, grid, smem, pdl, res, dev, st);
   }
 }
 
@@ -472,7 +475,7 @@ inline int skinny_mtt(int64_t M) { return M <= 16 ? 1 : (M <= 32 ? 2 : 4); }
 // the K-lanes' partial sums once. The ring is as deep as shared memory
 // allows.
 bl_status skinny_plan(int64_t M, int64_t N, int64_t K, int sms, SkinnyParams* p,
-                      SkinnySplit* split, int* grid, size_t* smem) {
+                      SkinnySplit* split, int* grid, size_t* smem, bool* res) {
   const int mtt = skinny_mtt(M);
   int64_t r = (N + sms - 1) / sms;
   if (r < 8) r = 8;
@@ -497,6 +500,26 @@ bl_status skinny_plan(int64_t M, int64_t N, int64_t K, int sms, SkinnyParams* p,
     }
   }
   if (best.ntw == 0) return BL_ERR_SHAPE;
+  // Resident weights (two CTAs per SM) when the whole slab and a token ring
+  // of at least two stages fit in half of an SM's shared memory, for the warp
+  // splits that fit 64 registers without spilling.
+  const bool res_split = mtt == 1 ? !(best.ntw == 4 && best.kps == 4)
+                                  : (mtt == 2 && (best.kps == 2 ? best.ntw <= 3 : best.ntw <= 2));
+  if (res_split && nchunk >= 2) {
+    int ts = nchunk < 4 ? nchunk : 4;
+    while (ts > 2 && skinny_res_smem_bytes(rp, mtt, ts, best.ntw, nchunk) > kGemvSmemCap) --ts;
+    if (skinny_res_smem_bytes(rp, mtt, ts, best.ntw, nchunk) <= kGemvSmemCap) {
+      p->rows_per_cta = (int)r;
+      p->rows_pad = rp;
+      p->stages = ts;
+      *split = best;
+      *grid = (int)((N + r - 1) / r);
+      *smem = skinny_res_smem_bytes(rp, mtt, ts, best.ntw, nchunk);
+      *res = true;
+      return BL_OK;
+    }
+  }
+  *res = false;
   int stages = nchunk;
   while (stages > 1 && skinny_smem_bytes(rp, mtt, stages, best.ntw) > kSkSmemCap) --stages;
   if (skinny_smem_bytes(rp, mtt, stages, best.ntw) > kSkSmemCap) return BL_ERR_SHAPE;
@@ -520,7 +543,8 @@ bl_status run_skinny(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, 
   SkinnySplit split;
   int grid;
   size_t smem;
-  BL_TRY(skinny_plan(M, N, K, sms, &p, &split, &grid, &smem));
+  bool res;
+  BL_TRY(skinny_plan(M, N, K, sms, &p, &split, &grid, &smem, &res));
   const int mtt = skinny_mtt(M);
   CUtensorMap tw, ta;
   BL_TRY(make_map_u8(&tw, Wp, (uint64_t)N, (uint64_t)(K / 4), 128, (uint32_t)p.rows_pad,
@@ -537,9 +561,9 @@ bl_status run_skinny(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, 
   p.relu2 = relu2;
   p.y_bf16 = y_bf16;
   p.raw = raw;
-  if (mtt == 1) return launch_skinny_split<1>(split, tw, ta, p, grid, smem, pdl, dev, st);
-  if (mtt == 2) return launch_skinny_split<2>(split, tw, ta, p, grid, smem, pdl, dev, st);
-  return launch_skinny_split<4>(split, tw, ta, p, grid, smem, pdl, dev, st);
+  if (mtt == 1) return launch_skinny_split<1>(split, tw, ta, p, grid, smem, pdl, res, dev, st);
+  if (mtt == 2) return launch_skinny_split<2>(split, tw, ta, p, grid, smem, pdl, res, dev, st);
+  return launch_skinny_split<4>(split, tw, ta, p, grid, smem, pdl, false, dev, st);
 }
 
 // Contraction of pre-quantised tokens: the skinny kernel up to 64 tokens,
@@ -557,16 +581,27 @@ bl_status run_contract(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K
                 split_ws_bytes, dev, sms, st);
 }
 
+// pdl: launch with programmatic dependent launch (the kernel waits for the
+// previous grid before it touches global memory), so in a chain it is
+// resident and ready when its predecessor completes.
 bl_status run_quant_acts(const void* A, bl_dtype dt, int64_t M, int64_t K, float eps, int8_t* Aq,
-                         float* gA, int32_t* rs, cudaStream_t st) {
+                         float* gA, int32_t* rs, cudaStream_t st, bool pdl = false) {
   if (M == 0) return BL_OK;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)M);
+  cfg.blockDim = dim3(kQuantThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
   if (dt == BL_BF16)
-    quant_acts_kernel<__nv_bfloat16><<<(unsigned)M, kQuantThreads, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16*>(A), K, eps, Aq, gA, rs);
+    BL_CUDA(cudaLaunchKernelEx(&cfg, quant_acts_kernel<__nv_bfloat16>,
+                               reinterpret_cast<const __nv_bfloat16*>(A), K, eps, Aq, gA, rs));
   else
-    quant_acts_kernel<float><<<(unsigned)M, kQuantThreads, 0, st>>>(
-        reinterpret_cast<const float*>(A), K, eps, Aq, gA, rs);
-  BL_CUDA(cudaGetLastError());
+    BL_CUDA(cudaLaunchKernelEx(&cfg, quant_acts_kernel<float>, reinterpret_cast<const float*>(A), K,
+                               eps, Aq, gA, rs));
   return BL_OK;
 }
 
@@ -970,7 +1005,7 @@ static bl_status linear_impl(const void* A, bl_dtype a_dtype, int64_t M, int64_t
   int8_t* Aq = reinterpret_cast<int8_t*>(base + w.aq);
   float* gA = reinterpret_cast<float*>(base + w.gamma);
   int32_t* rs = reinterpret_cast<int32_t*>(base + w.rowsum);
-  BL_TRY(run_quant_acts(A, a_dtype, M, K, eps, Aq, gA, rs, st));
+  BL_TRY(run_quant_acts(A, a_dtype, M, K, eps, Aq, gA, rs, st, (flags & BL_FLAG_PDL) != 0));
   BL_TRY(run_contract(Aq, W_packed, M, K, N, gamma, gA, rs, Y, kTcDequant, relu2 ? 1 : 0,
                       y_dtype == BL_BF16, true, dev, sms, st, base + w.total, ws_bytes - w.total));
   if (taps) {

@@ -117,7 +117,10 @@ quant_acts_kernel(const T* __restrict__ A, int64_t K, float eps, int8_t* __restr
                   float* __restrict__ gammaA, int32_t* __restrict__ rowsum) {
   // A kernel launched after this one with programmatic dependent launch may
   // start its own independent work now; it waits for this grid's results.
+  // This grid itself, when launched early, reads and writes global memory
+  // only after the previous kernel has completed.
   pdl_launch_dependents();
+  pdl_wait_prior_grid();
   const int64_t m = blockIdx.x;
   const T* row = A + m * K;
   constexpr int VEC = 16 / sizeof(T);

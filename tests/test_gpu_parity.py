@@ -410,3 +410,27 @@ def test_skinny_chain_shared_workspace(bl):
     refs = [oracle.bitlinear(A.f32, codes, g, EPS)["Y"] for A, codes, g in cases]
     for y, r in zip(outs, refs):
         assert_close(y.float().cpu().numpy(), r, torch.bfloat16)
+
+
+@pytest.mark.parametrize("M", [16, 20, 40])
+def test_small_batch_pdl_chain_shared_workspace(bl, M):
+    """Chained calls with programmatic dependent launch sharing one workspace:
+    each call's quantiser launches early but must wait for the previous call
+    before overwriting the shared int8 tokens; the contraction keeps its
+    weights resident (two CTAs per SM) at 16 and 20 tokens, the stage ring at
+    40. Every call must give its own result."""
+    K, N = 4096, 3000
+    ws = torch.empty(bl.workspace_bytes("linear", M, K, N), dtype=torch.uint8, device=DEV)
+    cases, args = [], []
+    for i in range(6):
+        W = si.weights(N, K, seed=500 + i, dtype="bf16")
+        codes, g = oracle.quant_weights(W.f32, EPS)
+        A = si.activations(M, K, seed=600 + i, dtype="bf16", outliers=True)
+        cases.append((A, codes, g))
+        args.append((A.torch(DEV), to_dev(oracle.pack_ternary(codes)),
+                     to_dev(np.array([g], np.float32))))
+    torch.cuda.synchronize()
+    outs = [bl.bl_linear(a, p, g, EPS, workspace=ws, pdl=True) for a, p, g in args]
+    torch.cuda.synchronize()
+    for (A, codes, g), y in zip(cases, outs):
+        assert_close(y.float().cpu().numpy(), oracle.bitlinear(A.f32, codes, g, EPS)["Y"], torch.bfloat16)
