@@ -682,6 +682,25 @@ def profile_case(name: str) -> int:
         torch.cuda.synchronize()
         for _ in range(3):
             bl.bl_linear_q(Aq, gA, pk, g, rowsum=rs, stream=st)
+    elif name in ("ffn512", "small_chain"):
+        K, H = 4096, 11008
+        if name == "ffn512":
+            pu, gu = bl.bl_quant_weights(si.weights(H, K, seed=1, dtype="bf16").torch(device), EPS)
+            pd, gd = bl.bl_quant_weights(si.weights(K, H, seed=2, dtype="bf16").torch(device), EPS)
+            X = si.activations(512, K, seed=0, dtype="bf16").torch(device)
+            ws = torch.empty(bl.workspace_bytes("ffn", 512, K, H), dtype=torch.uint8, device=device)
+            torch.cuda.synchronize()
+            for _ in range(3):
+                bl.bl_ffn_relu2(X, pu, gu, pd, gd, EPS, workspace=ws, stream=st)
+        else:  # 10 chained 16-token calls over 5 distinct 11008 x 4096 matrices
+            mats = [bl.bl_quant_weights(si.weights(H, K, seed=i, dtype="bf16").torch(device), EPS)
+                    for i in range(5)]
+            A = si.activations(16, K, seed=0, dtype="bf16").torch(device)
+            ws = torch.empty(bl.workspace_bytes("linear", 16, K, H), dtype=torch.uint8, device=device)
+            torch.cuda.synchronize()
+            for i in range(10):
+                w, g = mats[i % 5]
+                bl.bl_linear(A, w, g, EPS, workspace=ws, pdl=True, stream=st)
     elif name == "ste":
         M, N, K = 2048, 4096, 4096
         W = si.weights(N, K, seed=0, dtype="bf16").torch(device)
@@ -704,7 +723,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--profile-case", choices=["decode", "decode_radix3", "skinny", "prefill", "ste"],
+    ap.add_argument("--profile-case", choices=["decode", "decode_radix3", "skinny", "prefill", "ste",
+                                               "ffn512", "small_chain"],
                     help="run one small case for an ncu capture and exit")
     args = ap.parse_args(argv)
     if args.profile_case:
