@@ -194,16 +194,34 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(__uint_as_float(d[j]), scale);
         if constexpr (MASK) {
+          // This thread's 16 contiguous latent weights in 16-byte loads
+          // (cols is a multiple of 64 and col of 16, so they are aligned).
+          float w[16];
+          const int64_t o = r * p.cols + col;
+          if (p.mask_bf16) {
+            const uint4* src = reinterpret_cast<const uint4*>(
+                reinterpret_cast<const __nv_bfloat16*>(p.mask_w) + o);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (col + j < p.cols) {
-              const int64_t o = r * p.cols + col + j;
-              const float w = p.mask_bf16
-                                  ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.mask_w)[o])
-                                  : reinterpret_cast<const float*>(p.mask_w)[o];
-              if (fabs((double)w) > thr) v[j] = 0.0f;
+            for (int h = 0; h < 2; ++h) {
+              const uint4 u = __ldg(src + h);
+              const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) w[8 * h + j] = __bfloat162float(e[j]);
+            }
+          } else {
+            const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.mask_w) + o);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float4 f = __ldg(src + h);
+              w[4 * h] = f.x;
+              w[4 * h + 1] = f.y;
+              w[4 * h + 2] = f.z;
+              w[4 * h + 3] = f.w;
             }
           }
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (fabs((double)w[j]) > thr) v[j] = 0.0f;
         }
         float* out = p.C + r * p.cols + col;
         if (col + 16 <= p.cols && (p.cols & 3) == 0) {
@@ -232,28 +250,32 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
 // Layout kernels (32 × 32 tiles through shared memory, 256 threads).
 
 // W_qᵀ [K, Np] bf16 from the packed codes [N, K/4]: element (k, n) = c(n,k) - 1
-// (columns n ≥ N are zero). Block (x: 32 n, y: 32 k).
+// (columns n ≥ N are zero). Block tile: 32 rows n × 64 weights k. 128 threads
+// each load one 32-bit word (16 codes) and expand it into the tile; then all
+// 256 threads write 64 rows k × 32 columns n (64 contiguous bytes per row).
 __global__ void __launch_bounds__(256)
 expand_wqt_kernel(const uint8_t* __restrict__ W, int64_t N, int64_t K, int64_t Np,
                   __nv_bfloat16* __restrict__ out) {
-  __shared__ float tile[32][33];
-  const int64_t n0 = (int64_t)blockIdx.x * 32, k0 = (int64_t)blockIdx.y * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 × 8
-  for (int i = ty; i < 32; i += 8) {  // read row n0+i, weights k0+tx
-    const int64_t n = n0 + i, k = k0 + tx;
-    float w = 0.0f;
-    if (n < N) {
-      // weight k = 16·g + 4·j + i2 sits at bits 8·i2 + 2·j of word g
-      const uint32_t word = __ldg(reinterpret_cast<const uint32_t*>(W + n * (K / 4)) + (k >> 4));
-      const int j = (int)((k >> 2) & 3), i2 = (int)(k & 3);
-      w = (float)(int)((word >> (8 * i2 + 2 * j)) & 3u) - 1.0f;
+  __shared__ __nv_bfloat16 tile[64][34];
+  const int64_t n0 = (int64_t)blockIdx.x * 32, k0 = (int64_t)blockIdx.y * 64;
+  const int tid = threadIdx.x;
+  if (tid < 128) {
+    const int i = tid >> 2, q = tid & 3;  // row n0+i, word q of the 64 weights
+    const int64_t n = n0 + i;
+    uint32_t word = 0x55555555u;          // codes 1 (w = 0) past N
+    if (n < N) word = __ldg(reinterpret_cast<const uint32_t*>(W + n * (K / 4)) + (k0 >> 4) + q);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {  // weight 16q + 4j + i2 at bits 8·i2 + 2·j
+      const int j = e >> 2, i2 = e & 3;
+      const int c = (int)((word >> (8 * i2 + 2 * j)) & 3u);
+      tile[16 * q + e][i] = __float2bfloat16_rn((float)(c - 1));
     }
-    tile[i][tx] = w;
   }
   __syncthreads();
-  for (int i = ty; i < 32; i += 8) {  // write row k0+i, columns n0+tx
-    const int64_t k = k0 + i, n = n0 + tx;
-    if (k < K && n < Np) out[k * Np + n] = __float2bfloat16_rn(tile[tx][i]);
+  const int tx = tid & 31, ty = tid >> 5;
+  for (int r = ty; r < 64; r += 8) {
+    const int64_t k = k0 + r, n = n0 + tx;
+    if (k < K && n < Np) out[k * Np + n] = tile[r][tx];
   }
 }
 
