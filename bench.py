@@ -500,7 +500,7 @@ def run_ffn(bl, device, peaks, Ms=(1, 64, 512), reps=10):
                          torch.empty((M, K), dtype=torch.bfloat16, device=device),
                          torch.empty(wsb, dtype=torch.uint8, device=device)))
         t = rotating_time([lambda s=s_: bl.bl_ffn_relu2(s[0], s[1], gu, s[2], gd, EPS, out=s[3],
-                                                        workspace=s[4], stream=stream)
+                                                        workspace=s[4], pdl=True, stream=stream)
                            for s_ in sets], stream, reps)
         wbytes = 2 * H * K // 4
         out[f"M{M}"] = {"us": t * 1e6, "tokens_per_s": M / t, "weight_gbs": wbytes / t / 1e9,

@@ -285,6 +285,17 @@ bl_status bl_ffn_relu2(const void* X, bl_dtype x_dtype, int64_t M, int64_t K,
                        float eps, void* Y, bl_dtype y_dtype, void* workspace,
                        size_t ws_bytes, bl_stream_t stream);
 
+/* bl_ffn_relu2 with flags: BL_FLAG_PDL launches the block's first kernel
+ * (the up-projection GEMV, or the quantiser above bl_gemv_max_tokens()
+ * tokens) with programmatic dependent launch, under the same contract as
+ * bl_linear_ex: W_up and W_down were not written by the kernel preceding
+ * this call on `stream`. */
+bl_status bl_ffn_relu2_ex(const void* X, bl_dtype x_dtype, int64_t M, int64_t K,
+                          int64_t H, const uint8_t* W_up, const float* gamma_up,
+                          const uint8_t* W_down, const float* gamma_down, float eps,
+                          void* Y, bl_dtype y_dtype, void* workspace, size_t ws_bytes,
+                          unsigned flags, bl_stream_t stream);
+
 /* bl_ffn_relu2 with taps: act_* report the quantised block input X_q, acc_up
  * the up-projection, req_* the requantised ReLU² tokens fed to the
  * down-projection (see bl_taps). */

@@ -183,7 +183,7 @@ def bl_linear_noalloc(A, W_packed, gamma, eps: float = 1e-5, *, relu2=False,
 
 
 def bl_ffn_relu2(X, W_up, gamma_up, W_down, gamma_down, eps: float = 1e-5, *,
-                 out_dtype=torch.bfloat16, out=None, workspace=None, stream=None):
+                 out_dtype=torch.bfloat16, out=None, workspace=None, pdl=False, stream=None):
     """Ternary FFN block: BitLinear up (K→H), ReLU², per-token requant, BitLinear down (H→K)."""
     for t, n in ((X, "X"), (W_up, "W_up"), (gamma_up, "gamma_up"), (W_down, "W_down"),
                  (gamma_down, "gamma_down")):
@@ -197,10 +197,10 @@ def bl_ffn_relu2(X, W_up, gamma_up, W_down, gamma_down, eps: float = 1e-5, *,
     L = load()
     if workspace is None:
         workspace = _ws(int(L.bl_ffn_workspace_bytes(M, K, H)), X.device)
-    check(L.bl_ffn_relu2(X.data_ptr(), _dt(X, "X"), M, K, H, W_up.data_ptr(), gamma_up.data_ptr(),
-                         W_down.data_ptr(), gamma_down.data_ptr(), float(eps), out.data_ptr(),
-                         _dt(out, "out"), _ptr(workspace), _nbytes(workspace), _stream(stream)),
-          "bl_ffn_relu2")
+    check(L.bl_ffn_relu2_ex(X.data_ptr(), _dt(X, "X"), M, K, H, W_up.data_ptr(), gamma_up.data_ptr(),
+                            W_down.data_ptr(), gamma_down.data_ptr(), float(eps), out.data_ptr(),
+                            _dt(out, "out"), _ptr(workspace), _nbytes(workspace),
+                            BL_FLAG_PDL if pdl else 0, _stream(stream)), "bl_ffn_relu2")
     return out
 
 

@@ -57,6 +57,8 @@ SIGNATURES = {
     "bl_ffn_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_ffn_relu2": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _f32, _vp, _int,
                             _vp, _sz, _vp]),
+    "bl_ffn_relu2_ex": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _f32, _vp, _int,
+                               _vp, _sz, _uint, _vp]),
     "bl_ffn_relu2_taps": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _f32, _vp,
                                  _int, _vp, _sz, ctypes.POINTER(BlTaps), _vp]),
     "bl_radix3_row_bytes": (_i64, [_i64]),

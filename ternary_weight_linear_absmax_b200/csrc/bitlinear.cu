@@ -1048,8 +1048,10 @@ size_t bl_ffn_workspace_bytes(int64_t M, int64_t K, int64_t H) {
 static bl_status ffn_impl(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, int64_t H,
                           const uint8_t* W_up, const float* gamma_up, const uint8_t* W_down,
                           const float* gamma_down, float eps, void* Y, bl_dtype y_dtype,
-                          void* workspace, size_t ws_bytes, const bl_taps* taps,
+                          void* workspace, size_t ws_bytes, const bl_taps* taps, unsigned flags,
                           cudaStream_t st) {
+  if ((flags & ~(unsigned)BL_FLAG_PDL) != 0) return BL_ERR_INVALID_ARG;
+  const bool pdl = (flags & BL_FLAG_PDL) != 0;
   BL_TRY(check_dtype(x_dtype));
   BL_TRY(check_dtype(y_dtype));
   BL_TRY(check_k(K));
@@ -1083,7 +1085,7 @@ static bl_status ffn_impl(const void* X, bl_dtype x_dtype, int64_t M, int64_t K,
     up.M = (int)M;
     up.eps = eps;
     if (taps) gemv_taps(up, taps->act_q, taps->act_gamma, taps->act_rowsum, taps->cta);
-    BL_TRY(run_gemv(kSrcFloat, kOutRawI32, x_dtype, up, false, dev, sms, st));
+    BL_TRY(run_gemv(kSrcFloat, kOutRawI32, x_dtype, up, pdl, dev, sms, st));
     GemvParams dn = {};
     dn.A = acc_up;
     dn.a_scale = gX;
@@ -1109,7 +1111,7 @@ static bl_status ffn_impl(const void* X, bl_dtype x_dtype, int64_t M, int64_t K,
   int8_t* Rq = reinterpret_cast<int8_t*>(base + w.rq);
   float* gR = reinterpret_cast<float*>(base + w.gamma_r);
   int32_t* rsR = reinterpret_cast<int32_t*>(base + w.rs_r);
-  BL_TRY(run_quant_acts(X, x_dtype, M, K, eps, Xq, gX, rsX, st));
+  BL_TRY(run_quant_acts(X, x_dtype, M, K, eps, Xq, gX, rsX, st, pdl));
   // Each contraction follows one of this call's own kernels, which write
   // neither W_up nor W_down: the weights may stream early (PDL).
   void* split_ws = base + w.total;
@@ -1138,7 +1140,15 @@ bl_status bl_ffn_relu2(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, in
                        const float* gamma_down, float eps, void* Y, bl_dtype y_dtype,
                        void* workspace, size_t ws_bytes, bl_stream_t stream) {
   return ffn_impl(X, x_dtype, M, K, H, W_up, gamma_up, W_down, gamma_down, eps, Y, y_dtype,
-                  workspace, ws_bytes, nullptr, reinterpret_cast<cudaStream_t>(stream));
+                  workspace, ws_bytes, nullptr, 0u, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bl_status bl_ffn_relu2_ex(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, int64_t H,
+                          const uint8_t* W_up, const float* gamma_up, const uint8_t* W_down,
+                          const float* gamma_down, float eps, void* Y, bl_dtype y_dtype,
+                          void* workspace, size_t ws_bytes, unsigned flags, bl_stream_t stream) {
+  return ffn_impl(X, x_dtype, M, K, H, W_up, gamma_up, W_down, gamma_down, eps, Y, y_dtype,
+                  workspace, ws_bytes, nullptr, flags, reinterpret_cast<cudaStream_t>(stream));
 }
 
 bl_status bl_ffn_relu2_taps(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, int64_t H,
@@ -1147,7 +1157,7 @@ bl_status bl_ffn_relu2_taps(const void* X, bl_dtype x_dtype, int64_t M, int64_t 
                             void* workspace, size_t ws_bytes, const bl_taps* taps,
                             bl_stream_t stream) {
   return ffn_impl(X, x_dtype, M, K, H, W_up, gamma_up, W_down, gamma_down, eps, Y, y_dtype,
-                  workspace, ws_bytes, taps, reinterpret_cast<cudaStream_t>(stream));
+                  workspace, ws_bytes, taps, 0u, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------

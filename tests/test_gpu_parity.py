@@ -434,3 +434,27 @@ def test_small_batch_pdl_chain_shared_workspace(bl, M):
     torch.cuda.synchronize()
     for (A, codes, g), y in zip(cases, outs):
         assert_close(y.float().cpu().numpy(), oracle.bitlinear(A.f32, codes, g, EPS)["Y"], torch.bfloat16)
+
+
+@pytest.mark.parametrize("M", [1, 16, 130])
+def test_ffn_pdl_chain_shared_workspace(bl, M):
+    """Chained FFN blocks with programmatic dependent launch on one shared
+    workspace: the next block's first kernel starts early but must not touch
+    the workspace or read its input before the previous block is done."""
+    K, H = 1024, 2752
+    ws = torch.empty(bl.workspace_bytes("ffn", M, K, H), dtype=torch.uint8, device=DEV)
+    blocks = []
+    for i in range(4):
+        cu, gu = oracle.quant_weights(si.weights(H, K, seed=700 + i, dtype="bf16").f32, EPS)
+        cd, gd = oracle.quant_weights(si.weights(K, H, seed=800 + i, dtype="bf16").f32, EPS)
+        X = si.activations(M, K, seed=900 + i, dtype="bf16", outliers=True)
+        blocks.append((X, cu, gu, cd, gd))
+    dev = [(X.torch(DEV), to_dev(oracle.pack_ternary(cu)), to_dev(np.array([gu], np.float32)),
+            to_dev(oracle.pack_ternary(cd)), to_dev(np.array([gd], np.float32)))
+           for X, cu, gu, cd, gd in blocks]
+    torch.cuda.synchronize()
+    outs = [bl.bl_ffn_relu2(*d, EPS, workspace=ws, pdl=True) for d in dev]
+    torch.cuda.synchronize()
+    for (X, cu, gu, cd, gd), y in zip(blocks, outs):
+        assert_close(y.float().cpu().numpy(), oracle.ffn_relu2(X.f32, cu, gu, cd, gd, EPS)["Y"],
+                     torch.bfloat16)
