@@ -682,16 +682,17 @@ def profile_case(name: str) -> int:
         torch.cuda.synchronize()
         for _ in range(3):
             bl.bl_linear_q(Aq, gA, pk, g, rowsum=rs, stream=st)
-    elif name in ("ffn512", "small_chain"):
+    elif name in ("ffn1", "ffn512", "small_chain"):
         K, H = 4096, 11008
-        if name == "ffn512":
+        if name.startswith("ffn"):
+            M = int(name[3:])
             pu, gu = bl.bl_quant_weights(si.weights(H, K, seed=1, dtype="bf16").torch(device), EPS)
             pd, gd = bl.bl_quant_weights(si.weights(K, H, seed=2, dtype="bf16").torch(device), EPS)
-            X = si.activations(512, K, seed=0, dtype="bf16").torch(device)
-            ws = torch.empty(bl.workspace_bytes("ffn", 512, K, H), dtype=torch.uint8, device=device)
+            X = si.activations(M, K, seed=0, dtype="bf16").torch(device)
+            ws = torch.empty(bl.workspace_bytes("ffn", M, K, H), dtype=torch.uint8, device=device)
             torch.cuda.synchronize()
             for _ in range(3):
-                bl.bl_ffn_relu2(X, pu, gu, pd, gd, EPS, workspace=ws, stream=st)
+                bl.bl_ffn_relu2(X, pu, gu, pd, gd, EPS, workspace=ws, pdl=True, stream=st)
         else:  # 10 chained 16-token calls over 5 distinct 11008 x 4096 matrices
             mats = [bl.bl_quant_weights(si.weights(H, K, seed=i, dtype="bf16").torch(device), EPS)
                     for i in range(5)]
@@ -724,7 +725,7 @@ def main(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--profile-case", choices=["decode", "decode_radix3", "skinny", "prefill", "ste",
-                                               "ffn512", "small_chain"],
+                                               "ffn1", "ffn512", "small_chain"],
                     help="run one small case for an ncu capture and exit")
     args = ap.parse_args(argv)
     if args.profile_case:

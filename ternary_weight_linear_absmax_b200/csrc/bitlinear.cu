@@ -402,13 +402,11 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
   BL_TRY(outk == kTcDequant ? launch_tc_bn<kTcDequant>(bn, ta, tw, ty, p, sp, dev, st)
                             : launch_tc_bn<kTcRawI32>(bn, ta, tw, ty, p, sp, dev, st));
   if (sp == 1) return BL_OK;
-  const int64_t total = M * N;
-  int64_t blocks = (total / 4 + 255) / 256;
-  if (blocks > 16 * (int64_t)sms) blocks = 16 * (int64_t)sms;
-  if (blocks < 1) blocks = 1;
-  splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, st>>>(
+  const dim3 rgrid((unsigned)((N + 1023) / 1024), (unsigned)M);
+  splitk_reduce_kernel<<<rgrid, 256, 0, st>>>(
       reinterpret_cast<const int32_t*>(Yk), sp, tc_split_rows(M) * N, M, N,
-      out == kTcRawI32 ? 1 : 0, gamma, gammaA, relu2, Y, y_bf16);
+      out == kTcRawI32 ? 1 : 0, gamma, gammaA, relu2, Y, y_bf16,
+      (N % 4 == 0 && (reinterpret_cast<uintptr_t>(Y) & 15) == 0) ? 1 : 0);
   BL_CUDA(cudaGetLastError());
   return BL_OK;
 }
@@ -417,11 +415,8 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
 // Skinny launches (5 ≤ M ≤ 64 tokens, mma.sync over all SMs).
 template <int MTT, int NTW, int KPS>
 bl_status launch_skinny_t(const CUtensorMap& tw, const CUtensorMap& ta, const SkinnyParams& p,
-                          int grid, size_t smem, bool pdl, bool res, int dev, cudaStream_t st) {
-  auto* k = skinny_ternary_kernel<MTT, NTW, KPS, false>;
-  if constexpr (MTT <= 2) {
-    if (res) k = skinny_ternary_kernel<MTT, NTW, KPS, true>;
-  }
+                          int grid, size_t smem, bool pdl, int dev, cudaStream_t st) {
+  auto* k = skinny_ternary_kernel<MTT, NTW, KPS>;
   BL_TRY(ensure_smem(k, dev, smem));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -446,22 +441,22 @@ constexpr SkinnySplit kSkSplits[] = {{1, 2}, {2, 2}, {3, 2}, {5, 2}, {2, 4}, {3,
 
 template <int MTT>
 bl_status launch_skinny_split(SkinnySplit sp, const CUtensorMap& tw, const CUtensorMap& ta,
-                              const SkinnyParams& p, int grid, size_t smem, bool pdl, bool res,
-                              int dev, cudaStream_t st) {
+                              const SkinnyParams& p, int grid, size_t smem, bool pdl, int dev,
+                              cudaStream_t st) {
   if (sp.kps == 2) {
     switch (sp.ntw) {
-      case 1: return launch_skinny_t<MTT, 1, 2>(tw, ta, p, grid, smem, pdl, res, dev, st);
-      case 2: return launch_skinny_t<MTT, 2, 2>(tw, ta, p, grid, smem, pdl, res, dev, st);
-      case 3: return launch_skinny_t<MTT, 3, 2>(tw, ta, p, grid, smem, pdl, res, dev, st);
+      case 1: return launch_skinny_t<MTT, 1, 2>(tw, ta, p, grid, smem, pdl, dev, st);
+      case 2: return launch_skinny_t<MTT, 2, 2>(tw, ta, p, grid, smem, pdl, dev, st);
+      case 3: return launch_skinny_t<MTT, 3, 2>(tw, ta, p, grid, smem, pdl, dev, st);
       default:
-        if constexpr (MTT <= 2) return launch_skinny_t<MTT, 5, 2>(tw, ta, p, grid, smem, pdl, res, dev, st);
+        if constexpr (MTT <= 2) return launch_skinny_t<MTT, 5, 2>(tw, ta, p, grid, smem, pdl, dev, st);
         return BL_ERR_SHAPE;
     }
   }
   switch (sp.ntw) {
-    case 2: return launch_skinny_t<MTT, 2, 4>(tw, ta, p, grid, smem, pdl, res, dev, st);
-    case 3: return launch_skinny_t<MTT, 3, 4>(tw, ta, p, grid, smem, pdl, res, dev, st);
-    default: return launch_skinny_t<MTT, 4, 4>(tw, ta, p, grid, smem, pdl, res, dev, st);
+    case 2: return launch_skinny_t<MTT, 2, 4>(tw, ta, p, grid, smem, pdl, dev, st);
+    case 3: return launch_skinny_t<MTT, 3, 4>(tw, ta, p, grid, smem, pdl, dev, st);
+    default: return launch_skinny_t<MTT, 4, 4>(tw, ta, p, grid, smem, pdl, dev, st);
   }
 }
 
@@ -475,7 +470,7 @@ inline int skinny_mtt(int64_t M) { return M <= 16 ? 1 : (M <= 32 ? 2 : 4); }
 // the K-lanes' partial sums once. The ring is as deep as shared memory
 // allows.
 bl_status skinny_plan(int64_t M, int64_t N, int64_t K, int sms, SkinnyParams* p,
-                      SkinnySplit* split, int* grid, size_t* smem, bool* res) {
+                      SkinnySplit* split, int* grid, size_t* smem) {
   const int mtt = skinny_mtt(M);
   int64_t r = (N + sms - 1) / sms;
   if (r < 8) r = 8;
@@ -500,26 +495,6 @@ bl_status skinny_plan(int64_t M, int64_t N, int64_t K, int sms, SkinnyParams* p,
     }
   }
   if (best.ntw == 0) return BL_ERR_SHAPE;
-  // Resident weights (two CTAs per SM) when the whole slab and a token ring
-  // of at least two stages fit in half of an SM's shared memory, for the warp
-  // splits that fit 64 registers without spilling.
-  const bool res_split = mtt == 1 ? !(best.ntw == 4 && best.kps == 4)
-                                  : (mtt == 2 && (best.kps == 2 ? best.ntw <= 3 : best.ntw <= 2));
-  if (res_split && nchunk >= 2) {
-    int ts = nchunk < 4 ? nchunk : 4;
-    while (ts > 2 && skinny_res_smem_bytes(rp, mtt, ts, best.ntw, nchunk) > kGemvSmemCap) --ts;
-    if (skinny_res_smem_bytes(rp, mtt, ts, best.ntw, nchunk) <= kGemvSmemCap) {
-      p->rows_per_cta = (int)r;
-      p->rows_pad = rp;
-      p->stages = ts;
-      *split = best;
-      *grid = (int)((N + r - 1) / r);
-      *smem = skinny_res_smem_bytes(rp, mtt, ts, best.ntw, nchunk);
-      *res = true;
-      return BL_OK;
-    }
-  }
-  *res = false;
   int stages = nchunk;
   while (stages > 1 && skinny_smem_bytes(rp, mtt, stages, best.ntw) > kSkSmemCap) --stages;
   if (skinny_smem_bytes(rp, mtt, stages, best.ntw) > kSkSmemCap) return BL_ERR_SHAPE;
@@ -543,8 +518,7 @@ bl_status run_skinny(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, 
   SkinnySplit split;
   int grid;
   size_t smem;
-  bool res;
-  BL_TRY(skinny_plan(M, N, K, sms, &p, &split, &grid, &smem, &res));
+  BL_TRY(skinny_plan(M, N, K, sms, &p, &split, &grid, &smem));
   const int mtt = skinny_mtt(M);
   CUtensorMap tw, ta;
   BL_TRY(make_map_u8(&tw, Wp, (uint64_t)N, (uint64_t)(K / 4), 128, (uint32_t)p.rows_pad,
@@ -561,9 +535,9 @@ bl_status run_skinny(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, 
   p.relu2 = relu2;
   p.y_bf16 = y_bf16;
   p.raw = raw;
-  if (mtt == 1) return launch_skinny_split<1>(split, tw, ta, p, grid, smem, pdl, res, dev, st);
-  if (mtt == 2) return launch_skinny_split<2>(split, tw, ta, p, grid, smem, pdl, res, dev, st);
-  return launch_skinny_split<4>(split, tw, ta, p, grid, smem, pdl, false, dev, st);
+  if (mtt == 1) return launch_skinny_split<1>(split, tw, ta, p, grid, smem, pdl, dev, st);
+  if (mtt == 2) return launch_skinny_split<2>(split, tw, ta, p, grid, smem, pdl, dev, st);
+  return launch_skinny_split<4>(split, tw, ta, p, grid, smem, pdl, dev, st);
 }
 
 // Contraction of pre-quantised tokens: the skinny kernel up to 64 tokens,

@@ -289,6 +289,12 @@ __device__ __forceinline__ void relu2_row_quant(const int4* __restrict__ a4, int
   }
 }
 
+// The single-device kernel keeps each thread's first kRequantRegVecs
+// 16-byte vectors of accumulators in registers between the max and the
+// quantise pass (rows up to 12288 accumulators), so the row is read from
+// memory once, and all of a thread's loads are in flight together.
+constexpr int kRequantRegVecs = 12;
+
 __global__ void __launch_bounds__(kQuantThreads)
 relu2_requant_kernel(const int32_t* __restrict__ acc, int64_t H, const float* __restrict__ gammaX,
                      const float* __restrict__ g_up, float eps, int8_t* __restrict__ Rq,
@@ -296,10 +302,67 @@ relu2_requant_kernel(const int32_t* __restrict__ acc, int64_t H, const float* __
   pdl_launch_dependents();
   const int64_t m = blockIdx.x;
   const int4* a4 = reinterpret_cast<const int4*>(acc + m * H);
+  const int64_t nvec = H / 4;
+  __shared__ float redf[kQuantThreads / 32];
+  __shared__ int redi[kQuantThreads / 32];
+  __shared__ float s_scale;
   const float sc = __fdiv_rn(__fmul_rn(gammaX[m], *g_up), 127.0f);
-  const float g = relu2_row_max(a4, H, sc);
-  if (threadIdx.x == 0) gammaR[m] = g;
-  relu2_row_quant(a4, H, sc, g, eps, Rq + m * H, rowsum + m);
+  int4 reg[kRequantRegVecs];
+#pragma unroll
+  for (int r = 0; r < kRequantRegVecs; ++r) {
+    const int64_t v = threadIdx.x + (int64_t)r * kQuantThreads;
+    if (v < nvec) reg[r] = __ldg(a4 + v);
+  }
+  float mx = 0.0f;
+  auto vmax = [&](const int4& u) {
+    mx = fmaxf(fmaxf(mx, fmaxf(relu2_of(u.x, sc), relu2_of(u.y, sc))),
+               fmaxf(relu2_of(u.z, sc), relu2_of(u.w, sc)));
+  };
+#pragma unroll
+  for (int r = 0; r < kRequantRegVecs; ++r)
+    if (threadIdx.x + (int64_t)r * kQuantThreads < nvec) vmax(reg[r]);
+  for (int64_t v = threadIdx.x + (int64_t)kRequantRegVecs * kQuantThreads; v < nvec;
+       v += kQuantThreads)
+    vmax(__ldg(a4 + v));
+  mx = warp_max(mx);
+  if ((threadIdx.x & 31) == 0) redf[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float t = threadIdx.x < kQuantThreads / 32 ? redf[threadIdx.x] : 0.0f;
+    t = warp_max(t);
+    if (threadIdx.x == 0) {
+      gammaR[m] = t;
+      s_scale = __fdiv_rn(127.0f, __fadd_rn(t, eps));
+    }
+  }
+  __syncthreads();
+  const float s = s_scale;
+  int8_t* q_row = Rq + m * H;
+  int sum = 0;
+  auto emit = [&](const int4& u, int64_t v) {
+    const uint32_t w = pack4_low_bytes(quant_i8_bits(relu2_of(u.x, sc), s),
+                                       quant_i8_bits(relu2_of(u.y, sc), s),
+                                       quant_i8_bits(relu2_of(u.z, sc), s),
+                                       quant_i8_bits(relu2_of(u.w, sc), s));
+    sum = dp4a(w, 0x01010101u, sum);
+    *reinterpret_cast<uint32_t*>(q_row + v * 4) = w;
+  };
+#pragma unroll
+  for (int r = 0; r < kRequantRegVecs; ++r) {
+    const int64_t v = threadIdx.x + (int64_t)r * kQuantThreads;
+    if (v < nvec) emit(reg[r], v);
+  }
+  for (int64_t v = threadIdx.x + (int64_t)kRequantRegVecs * kQuantThreads; v < nvec;
+       v += kQuantThreads)
+    emit(__ldg(a4 + v), v);
+  sum = warp_sum_i(sum);
+  if ((threadIdx.x & 31) == 0) redi[threadIdx.x >> 5] = sum;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    int t = threadIdx.x < kQuantThreads / 32 ? redi[threadIdx.x] : 0;
+    t = warp_sum_i(t);
+    if (threadIdx.x == 0) rowsum[m] = t;
+  }
 }
 
 // Tensor-parallel FFN, pass 1 on one rank's shard: rmax[m] = max_n r.
@@ -351,34 +414,62 @@ dequant_i32_kernel(const int32_t* __restrict__ acc, const float* __restrict__ ga
   }
 }
 
+__device__ __forceinline__ float dequant_value(int v, float sc, int relu2) {
+  float y = __fmul_rn((float)v, sc);
+  if (relu2) {
+    y = fmaxf(y, 0.0f);
+    y = __fmul_rn(y, y);
+  }
+  return y;
+}
+
 // Sum of the INT32 partials of a K-split contraction (split z at
 // part + z·stride, rows of N; split 0 already subtracted the row sums), then
 // the epilogue: raw INT32, or y = v · ((γ_A·γ)/127) in fp32 (ReLU² optional)
-// as fp32/bf16.
+// as fp32/bf16. One block per output row (blockIdx.y) and 1024 columns per
+// block (blockIdx.x), four columns per thread: 16-byte loads and stores
+// when vec (N a multiple of 4, part and Y 16-byte aligned), else scalar.
 __global__ void __launch_bounds__(256)
 splitk_reduce_kernel(const int32_t* __restrict__ part, int splits, int64_t stride, int64_t M,
                      int64_t N, int raw, const float* __restrict__ gamma,
-                     const float* __restrict__ gammaA, int relu2, void* Y, int y_bf16) {
-  const int64_t total = M * N;
-  const float g = raw ? 0.0f : __ldg(gamma);
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    int v = 0;
-    for (int z = 0; z < splits; ++z) v += __ldg(part + (int64_t)z * stride + i);
+                     const float* __restrict__ gammaA, int relu2, void* Y, int y_bf16,
+                     int vec) {
+  const int64_t m = blockIdx.y;
+  const float sc = raw ? 0.0f : __fdiv_rn(__fmul_rn(__ldg(gammaA + m), __ldg(gamma)), 127.0f);
+  auto finish = [sc, relu2](int v) -> float { return dequant_value(v, sc, relu2); };
+  const int64_t c = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (c >= N) return;
+  const int64_t o = m * N + c;
+  if (vec) {
+    int4 v = __ldg(reinterpret_cast<const int4*>(part + o));
+    for (int z = 1; z < splits; ++z) {
+      const int4 u = __ldg(reinterpret_cast<const int4*>(part + (int64_t)z * stride + o));
+      v.x += u.x;
+      v.y += u.y;
+      v.z += u.z;
+      v.w += u.w;
+    }
     if (raw) {
-      reinterpret_cast<int32_t*>(Y)[i] = v;
-      continue;
+      *reinterpret_cast<int4*>(reinterpret_cast<int32_t*>(Y) + o) = v;
+    } else if (y_bf16) {
+      __nv_bfloat162* yp = reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(Y) + o);
+      yp[0] = __floats2bfloat162_rn(finish(v.x), finish(v.y));
+      yp[1] = __floats2bfloat162_rn(finish(v.z), finish(v.w));
+    } else {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(Y) + o) =
+          make_float4(finish(v.x), finish(v.y), finish(v.z), finish(v.w));
     }
-    const float sc = __fdiv_rn(__fmul_rn(__ldg(gammaA + i / N), g), 127.0f);
-    float y = __fmul_rn((float)v, sc);
-    if (relu2) {
-      y = fmaxf(y, 0.0f);
-      y = __fmul_rn(y, y);
-    }
-    if (y_bf16)
-      reinterpret_cast<__nv_bfloat16*>(Y)[i] = __float2bfloat16_rn(y);
+    return;
+  }
+  for (int64_t cc = c; cc < c + 4 && cc < N; ++cc) {
+    int v = 0;
+    for (int z = 0; z < splits; ++z) v += __ldg(part + (int64_t)z * stride + m * N + cc);
+    if (raw)
+      reinterpret_cast<int32_t*>(Y)[m * N + cc] = v;
+    else if (y_bf16)
+      reinterpret_cast<__nv_bfloat16*>(Y)[m * N + cc] = __float2bfloat16_rn(finish(v));
     else
-      reinterpret_cast<float*>(Y)[i] = y;
+      reinterpret_cast<float*>(Y)[m * N + cc] = finish(v);
   }
 }
 

@@ -107,27 +107,11 @@ __device__ __forceinline__ void mma_s8_16832(int (&c)[4], const uint32_t (&a)[4]
 __device__ __forceinline__ int skinny_t_box(int warp) { return warp & 3; }
 __device__ __forceinline__ int skinny_t_first(int warp) { return ((warp >> 2) + 2) & 3; }
 
-// Resident mode: the CTA's whole weight slab (every K chunk) has its own
-// slot and one-shot barrier and is requested before the dependency wait; only
-// the token boxes go through a ring of S stages. With at most 113 KB of shared
-// memory two CTAs fit on an SM, so in a chain of calls the next call's CTA
-// streams all its weights while this one computes.
-// [weights nchunk·wbox (the partial sums alias it)][tokens S·4 boxes]
-// [scale 64][row sums 64][wfull nchunk][tfull S][tempty S]
-__host__ __device__ inline size_t skinny_res_smem_bytes(int rows_pad, int mtt, int stages, int ntw,
-                                                        int nchunk) {
-  size_t wreg = (size_t)nchunk * rows_pad * 128;
-  const size_t red = skinny_red_bytes(ntw, mtt);
-  if (red > wreg) wreg = red;
-  return 1024 + wreg + (size_t)stages * 4 * (16 * mtt) * 128 + 2 * kSkMaxTokens * 4 +
-         ((size_t)nchunk + 2 * (size_t)stages) * 8;
-}
-
 // MTT: token m-tiles (16 tokens each; rows past M read as zero).
 // NTW: n-tiles (8 weight rows each) per warp. KPS: 32-K steps per warp and
-// stage (warps = KPS n-tile groups × 16/KPS K-lanes). RES: resident weights.
-template <int MTT, int NTW, int KPS, bool RES>
-__global__ void __launch_bounds__(kSkThreads, RES ? 2 : 1)
+// stage (warps = KPS n-tile groups × 16/KPS K-lanes).
+template <int MTT, int NTW, int KPS>
+__global__ void __launch_bounds__(kSkThreads, 1)
 skinny_ternary_kernel(const __grid_constant__ CUtensorMap tm_w,
                       const __grid_constant__ CUtensorMap tm_a, const SkinnyParams p) {
   constexpr int MB = 16 * MTT;  // token rows per box
@@ -138,68 +122,49 @@ skinny_ternary_kernel(const __grid_constant__ CUtensorMap tm_w,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int RP = p.rows_pad, NT = RP / 8;
   const int S = p.stages;
-  const int nchunk = skinny_chunks(p.K);
   const uint32_t wbox = (uint32_t)RP * 128;
-  // Ring mode: stage = weight box + 4 token boxes. Resident mode: weights in
-  // their own slots, stage = 4 token boxes.
-  const uint32_t stage_bytes = RES ? 4 * kTokBox : wbox + 4 * kTokBox;
-  const size_t red_bytes = skinny_red_bytes(NTW, MTT);
-  size_t wreg = RES ? (size_t)nchunk * wbox : 0;
-  if (RES && red_bytes > wreg) wreg = red_bytes;
-  uint8_t* s_tok = smem + wreg;  // resident mode: the token ring
+  const uint32_t stage_bytes = wbox + 4 * kTokBox;
   size_t ring = (size_t)S * stage_bytes;
-  if (!RES && red_bytes > ring) ring = red_bytes;
-  float* s_sc = reinterpret_cast<float*>(smem + wreg + ring);
+  const size_t red_bytes = skinny_red_bytes(NTW, MTT);
+  if (red_bytes > ring) ring = red_bytes;
+  float* s_sc = reinterpret_cast<float*>(smem + ring);
   int* s_rs = reinterpret_cast<int*>(s_sc + kSkMaxTokens);
-  uint64_t* full = reinterpret_cast<uint64_t*>(s_rs + kSkMaxTokens);  // ring: [S]; resident: wfull [nchunk]
-  uint64_t* tfull = full + (RES ? nchunk : 0);                         // resident: [S]
-  uint64_t* empty = tfull + S;
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_rs + kSkMaxTokens);
+  uint64_t* empty = full + S;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;  // mma fragment coordinates
   const int64_t r0 = (int64_t)blockIdx.x * p.rows_per_cta;
+  const int nchunk = skinny_chunks(p.K);
   const int rot = (int)(blockIdx.x % (unsigned)nchunk);
   const int M = (int)p.M;
 
-  // Weight box of sequence c: ring mode into stage st, resident mode into
-  // slot c (st == c).
-  auto issue_w = [&](int c, int st) {
+  auto issue_w = [&](int c, int st) {  // weight box of sequence c into stage st
     const int cc = (c + rot) % nchunk;
     mbar_arrive_expect_tx(&full[st], wbox);
-    uint8_t* dst = RES ? smem + (size_t)c * wbox : smem + (size_t)st * stage_bytes;
-    tma_load_2d(dst, &tm_w, cc * 128, (int32_t)r0, &full[st]);
+    tma_load_2d(smem + (size_t)st * stage_bytes, &tm_w, cc * 128, (int32_t)r0, &full[st]);
   };
   auto issue_t = [&](int c, int st, int q) {  // token box q of sequence c into stage st
     const int cc = (c + rot) % nchunk;
-    uint64_t* bar = RES ? &tfull[st] : &full[st];
-    mbar_arrive_expect_tx(bar, kTokBox);
-    uint8_t* dst = RES ? s_tok + (size_t)st * stage_bytes + q * kTokBox
-                       : smem + (size_t)st * stage_bytes + wbox + q * kTokBox;
-    tma_load_2d(dst, &tm_a, cc * kSkKC + q * 128, 0, bar);
+    mbar_arrive_expect_tx(&full[st], kTokBox);
+    tma_load_2d(smem + (size_t)st * stage_bytes + wbox + q * kTokBox, &tm_a, cc * kSkKC + q * 128, 0,
+                &full[st]);
   };
 
-  // 1. Barriers (one arrival per request of a fill), then the weight boxes of
-  //    the first S stages (ring) or of every chunk (resident): they do not
-  //    depend on the previous kernel.
+  // 1. Barriers (one arrival per request of a fill: the weight box and four
+  //    token boxes), then the weight boxes of the first S stages: they do
+  //    not depend on the previous kernel.
   if (tid == 0) {
-    if constexpr (RES) {
-      for (int c = 0; c < nchunk; ++c) mbar_init(&full[c], 1);
-      for (int s = 0; s < S; ++s) {
-        mbar_init(&tfull[s], 4);
-        mbar_init(&empty[s], kSkWarps);
-      }
-    } else {
-      for (int s = 0; s < S; ++s) {
-        mbar_init(&full[s], 5);
-        mbar_init(&empty[s], kSkWarps);
-      }
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 5);
+      mbar_init(&empty[s], kSkWarps);
     }
     fence_barrier_init();
   }
   __syncthreads();
   if (lane == 0) {
     if (warp == 1) prefetch_tensormap(&tm_a);
-    for (int c = warp; c < (RES ? nchunk : S); c += kSkWarps) issue_w(c, c);
+    for (int c = warp; c < S; c += kSkWarps) issue_w(c, c);
   }
   pdl_launch_dependents();
   // 2. Tokens, their scales and row sums come from the previous kernel.
@@ -252,27 +217,19 @@ skinny_ternary_kernel(const __grid_constant__ CUtensorMap tm_w,
   uint32_t par = 0, ppar = 0;
   for (int c = 0; c < nchunk; ++c) {
     // Refill the stage that sequence c-1 used (sp) with sequence c-1+S once
-    // every warp has released it (resident mode: its token boxes only).
+    // every warp has released it.
     if (lane == 0 && c >= 1 && c - 1 + S < nchunk) {
       const int cn = c - 1 + S;
-      const bool wi = !RES && (cn & (kSkWarps - 1)) == warp, ti = ((cn - tc0) & 3) == 0;
+      const bool wi = (cn & (kSkWarps - 1)) == warp, ti = ((cn - tc0) & 3) == 0;
       if ((wi || ti) && mbar_wait(&empty[sp], ppar)) {
         if (wi) issue_w(cn, sp);
         if (ti) issue_t(cn, sp, tq);
       }
     }
-    const uint8_t* wst;
-    const uint8_t* tk;
-    if constexpr (RES) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&full[c], 0) && mbar_wait(&tfull[s], par));
-      wst = smem + (size_t)c * wbox;
-      tk = s_tok + (size_t)s * stage_bytes;
-    } else {
-      ok = __all_sync(0xffffffffu, mbar_wait(&full[s], par));
-      wst = smem + (size_t)s * stage_bytes;
-      tk = wst + wbox;
-    }
+    ok = __all_sync(0xffffffffu, mbar_wait(&full[s], par));
     if (!ok) break;
+    const uint8_t* wst = smem + (size_t)s * stage_bytes;
+    const uint8_t* tk = wst + wbox;
 #pragma unroll
     for (int q = 0; q < KPS / 2; ++q) {
       uint4 w[NTW];

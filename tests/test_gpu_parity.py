@@ -416,9 +416,9 @@ def test_skinny_chain_shared_workspace(bl):
 def test_small_batch_pdl_chain_shared_workspace(bl, M):
     """Chained calls with programmatic dependent launch sharing one workspace:
     each call's quantiser launches early but must wait for the previous call
-    before overwriting the shared int8 tokens; the contraction keeps its
-    weights resident (two CTAs per SM) at 16 and 20 tokens, the stage ring at
-    40. Every call must give its own result."""
+    before overwriting the shared int8 tokens, and the contraction streams its
+    weights before it waits for the quantiser. Every call must give its own
+    result."""
     K, N = 4096, 3000
     ws = torch.empty(bl.workspace_bytes("linear", M, K, N), dtype=torch.uint8, device=DEV)
     cases, args = [], []
