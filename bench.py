@@ -126,6 +126,48 @@ def profiled_traffic():
         return None
 
 
+TRAFFIC_COMMAND = ("python bench.py --profile-case decode  (then) ncu --metrics "
+                   "gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum "
+                   "--clock-control none -k regex:gemv_ternary -s 5 -c 5 --csv "
+                   "--log-file gpurun_out/ncu_decode.csv python bench.py --profile-case decode")
+
+
+def write_traffic_json(csv_path):
+    """Summarise the decode GEMV's ncu capture (TRAFFIC_COMMAND) into the
+    JSON that profiled_traffic() reads, stamped with the kernel source hash."""
+    import csv
+    per = {}
+    with open(csv_path) as f:
+        rows = [r for r in csv.reader(f) if len(r) > 10]
+    head = rows[0]
+    ki, ni, vi, ii = (head.index("Kernel Name"), head.index("Metric Name"),
+                      head.index("Metric Value"), head.index("ID"))
+    kernel = None
+    for r in rows[1:]:
+        if "gemv_ternary" not in r[ki]:
+            continue
+        kernel = r[ki].split("(")[0]
+        per.setdefault(r[ni], {})[r[ii]] = float(r[vi].replace(",", ""))
+    mean = {k: sum(v.values()) / len(v) for k, v in per.items()}
+    n = len(per["dram__bytes_read.sum"])
+    M, K, N = DECODE["M"], DECODE["K"], DECODE["N"]
+    out = {"kernel": kernel,
+           "workload": f"decode GEMV, {M} token, K={K}, N={N}, bf16 in/out",
+           "command": TRAFFIC_COMMAND,
+           "launches_averaged": n,
+           "dram_bytes_read_per_launch": mean["dram__bytes_read.sum"],
+           "dram_bytes_write_per_launch": mean["dram__bytes_write.sum"],
+           "dram_bytes_per_launch": mean["dram__bytes_read.sum"] + mean["dram__bytes_write.sum"],
+           "algorithmic_bytes_per_launch": N * K // 4 + 2 * K * M + 2 * N * M,
+           "gpu_time_duration_ns_per_launch_cold_serialised": mean["gpu__time_duration.sum"],
+           "kernel_source_sha256": sha256_file(GEMV_SOURCE)}
+    with open(PROFILE_TRAFFIC, "w") as f:
+        json.dump(out, f, indent=1)
+        f.write("\n")
+    print(json.dumps(out))
+    return 0
+
+
 # ---------------------------------------------------------------------------
 # clocks sampler (nvidia-smi during the timed region)
 
@@ -209,6 +251,17 @@ def time_graph(graph, stream, reps: int):
         end.record(stream)
     end.synchronize()
     return start.elapsed_time(end) / 1e3
+
+
+def settled_time(graph, stream, reps: int, windows: int = 5):
+    """Device seconds per replay of a captured graph for the secondary
+    figures: after the caller's warm-up replays, synchronise, then time
+    `windows` windows of `reps` replays and take the median window. (The
+    first window after capture measured up to 1.6x slower than the rest.)"""
+    import torch
+    torch.cuda.synchronize()
+    ts = [time_graph(graph, stream, reps) / reps for _ in range(windows)]
+    return statistics.median(ts)
 
 
 def capture(fn, stream):
@@ -329,8 +382,8 @@ def run_decode(bl, device, steps, warmup, peaks, world):
     fg = capture(floor_chain, stream)
     for _ in range(3):
         fg.replay()
-    tf = time_graph(fg, stream, max(3, min(steps, 50)))
-    res["floor_us"] = tf / (max(3, min(steps, 50)) * CALLS_PER_STEP) * 1e6
+    tf = settled_time(fg, stream, max(3, min(steps, 10)))
+    res["floor_us"] = tf / CALLS_PER_STEP * 1e6
     del fg
     res["pool_list"] = pool
     res["gamma"] = gamma
@@ -362,7 +415,7 @@ def run_decode_storage_variants(bl, device, dec, peaks, reps=5):
         g = capture(chain, stream)
         for _ in range(3):
             g.replay()
-        t = time_graph(g, stream, reps) / (reps * CALLS_PER_STEP)
+        t = settled_time(g, stream, reps) / CALLS_PER_STEP
         alg = wbytes + M * K * 2 + M * N * 2
         out[name] = {"us_per_call": t * 1e6, "tokens_per_s": M / t, "weight_bytes": wbytes,
                      "gbs": alg / t / 1e9, "hbm_frac": alg / t / 1e9 / peaks["hbm_gbs"]}
@@ -414,7 +467,7 @@ def run_small_batch(bl, device, peaks, reps=200):
     g = capture(chain, stream)
     for _ in range(3):
         g.replay()
-    t = time_graph(g, stream, max(1, reps // calls)) / max(1, reps // calls) / calls
+    t = settled_time(g, stream, max(1, reps // calls)) / calls
     alg = N * K // 4 + M * K * 2 + M * N * 2
     del g
     return {"workload": "16 tokens, K=4096 -> N=11008, bf16, rotating weight pool > L2, "
@@ -435,9 +488,9 @@ def rotating_time(calls, stream, reps):
     g = capture(run, stream)
     for _ in range(3):
         g.replay()
-    t = time_graph(g, stream, reps)
+    t = settled_time(g, stream, reps)
     del g
-    return t / (reps * len(calls))
+    return t / len(calls)
 
 
 def n_sets(bytes_per_set, device_index, factor=1.1):
@@ -727,7 +780,12 @@ def main(argv=None):
     ap.add_argument("--profile-case", choices=["decode", "decode_radix3", "skinny", "prefill", "ste",
                                                "ffn1", "ffn512", "small_chain"],
                     help="run one small case for an ncu capture and exit")
+    ap.add_argument("--traffic-json", metavar="NCU_CSV",
+                    help="write the decode GEMV traffic summary read by the bench line "
+                         "from an ncu CSV of the --profile-case decode capture, and exit")
     args = ap.parse_args(argv)
+    if args.traffic_json:
+        return write_traffic_json(args.traffic_json)
     if args.profile_case:
         return profile_case(args.profile_case)
     if args.impl == "reference":

@@ -236,15 +236,29 @@ constexpr size_t kGemvSmemCap = 112 * 1024;
 
 // Choose rows per CTA: one wave over the SMs when shared memory allows,
 // at most kGemvMaxRows rows.
+// Grid of the one-CTA-per-row-slab kernels, rows split evenly: every SM
+// gets the same number of CTAs of a launch (one when a slab of at most
+// r_cap rows per SM covers N, else a multiple of the SM count). A launch
+// with one CTA fewer than SMs leaves an SM free, which in a chain of
+// programmatic dependent launches then takes two CTAs of the next launch
+// and finishes it late. Returns the rows of the largest slab.
+int even_grid(int64_t N, int64_t r_cap, int sms, int* grid) {
+  const int64_t g0 = (N + r_cap - 1) / r_cap;
+  int64_t g = g0 <= sms ? sms : (g0 + sms - 1) / sms * sms;
+  if (g > N) g = N;
+  if (g < 1) g = 1;
+  *grid = (int)g;
+  return (int)((N + g - 1) / g);
+}
+
 bl_status gemv_plan(int64_t N, int64_t K, int M, int sms, int* rows, int* grid, size_t* smem) {
   int64_t r = (N + sms - 1) / sms;
   if (r < 1) r = 1;
   if (r > kGemvMaxRows) r = kGemvMaxRows;
   while (r > 1 && gemv_smem_bytes(K, (int)r, M) > kGemvSmemCap) r = (r + 1) / 2;
   if (gemv_smem_bytes(K, (int)r, M) > kGemvSmemCap) return BL_ERR_SHAPE;
-  *rows = (int)r;
-  *grid = (int)((N + r - 1) / r);
-  *smem = gemv_smem_bytes(K, (int)r, M);
+  *rows = even_grid(N, r, sms, grid);
+  *smem = gemv_smem_bytes(K, *rows, M);
   return BL_OK;
 }
 
@@ -607,11 +621,11 @@ bl_status run_r3(bl_dtype a_dtype, GemvR3Params p, bool pdl, int dev, int sms, c
   if (r < 1) r = 1;
   if (r > kGemvMaxRows) r = kGemvMaxRows;
   while (r > 1 && gemv_r3_smem_bytes(p.rb, (int)r, p.M) > cap) r = (r + 1) / 2;
-  const size_t smem = gemv_r3_smem_bytes(p.rb, (int)r, p.M);
-  if (smem > cap) return BL_ERR_SHAPE;
-  p.rows_per_cta = (int)r;
-  p.rows_pad = gemv_rows_pad((int)r);
-  const int grid = (int)((p.N + r - 1) / r);
+  if (gemv_r3_smem_bytes(p.rb, (int)r, p.M) > cap) return BL_ERR_SHAPE;
+  int grid;
+  p.rows_per_cta = even_grid(p.N, r, sms, &grid);
+  p.rows_pad = gemv_rows_pad(p.rows_per_cta);
+  const size_t smem = gemv_r3_smem_bytes(p.rb, p.rows_per_cta, p.M);
   CUtensorMap tw;
   BL_TRY(make_map_u8(&tw, p.W, (uint64_t)p.N, (uint64_t)p.rb, 128, (uint32_t)p.rows_pad,
                      CU_TENSOR_MAP_SWIZZLE_128B));
@@ -1360,8 +1374,10 @@ bl_status bl_linear_lut(const void* A, bl_dtype a_dtype, int64_t M, int64_t K, c
   if (r < 1) r = 1;
   if (r > kGemvMaxRows) r = kGemvMaxRows;
   while (r > 1 && gemv_lut_smem_bytes(K, (int)r) > kGemvSmemCap) r = (r + 1) / 2;
+  if (gemv_lut_smem_bytes(K, (int)r) > kSkSmemCap) return BL_ERR_SHAPE;  // tables of very long rows do not fit
+  int grid;
+  r = even_grid(N, r, sms, &grid);
   const size_t smem = gemv_lut_smem_bytes(K, (int)r);
-  if (smem > kSkSmemCap) return BL_ERR_SHAPE;  // tables of very long rows do not fit
   GemvLutParams p = {};
   p.A = A;
   p.W = W_idx;
@@ -1374,7 +1390,6 @@ bl_status bl_linear_lut(const void* A, bl_dtype a_dtype, int64_t M, int64_t K, c
   p.eps = eps;
   p.y_bf16 = y_dtype == BL_BF16;
   p.raw = (flags & BL_FLAG_RAW_I32) != 0;
-  const int grid = (int)((N + r - 1) / r);
   CUtensorMap tw;
   BL_TRY(make_map_u8(&tw, W_idx, (uint64_t)N, (uint64_t)(K / 4), 128, (uint32_t)p.rows_pad,
                      CU_TENSOR_MAP_SWIZZLE_128B));

@@ -140,8 +140,9 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int64_t K = p.K;
-  const int64_t r0 = (int64_t)blockIdx.x * p.rows_per_cta;
-  const int R = (int)min((int64_t)p.rows_per_cta, p.N - r0);
+  // Rows [r0, r1) of an even split over the grid (at most rows_per_cta).
+  const int64_t r0 = (int64_t)blockIdx.x * p.N / gridDim.x;
+  const int R = (int)((int64_t)(blockIdx.x + 1) * p.N / gridDim.x - r0);
   const int M = p.M;
 
   uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem);

@@ -77,8 +77,9 @@ gemv_lut_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvLutParams p)
   __shared__ int s_wok;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t K = p.K, G = K / 4;
-  const int64_t r0 = (int64_t)blockIdx.x * p.rows_per_cta;
-  const int R = (int)min((int64_t)p.rows_per_cta, p.N - r0);
+  // Rows [r0, r1) of an even split over the grid (at most rows_per_cta).
+  const int64_t r0 = (int64_t)blockIdx.x * p.N / gridDim.x;
+  const int R = (int)((int64_t)(blockIdx.x + 1) * p.N / gridDim.x - r0);
   const int nbox = gemv_boxes(K);
   const int box_bytes = p.rows_pad * 128;
   uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem);

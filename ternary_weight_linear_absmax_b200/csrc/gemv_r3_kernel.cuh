@@ -104,8 +104,9 @@ gemv_r3_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvR3Params p) {
   __shared__ int s_wok;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t K = p.K, rb = p.rb, Kp = 5 * rb;
-  const int64_t r0 = (int64_t)blockIdx.x * p.rows_per_cta;
-  const int R = (int)min((int64_t)p.rows_per_cta, p.N - r0);
+  // Rows [r0, r1) of an even split over the grid (at most rows_per_cta).
+  const int64_t r0 = (int64_t)blockIdx.x * p.N / gridDim.x;
+  const int R = (int)((int64_t)(blockIdx.x + 1) * p.N / gridDim.x - r0);
   const int M = p.M;
   const int nbox = gemv_r3_boxes(rb);
   const int box_bytes = p.rows_pad * 128;
