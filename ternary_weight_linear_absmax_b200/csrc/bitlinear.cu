@@ -89,6 +89,12 @@ bl_status ensure_smem(F* kernel, int dev, size_t bytes) {
     if (cache[i].fn == (const void*)kernel && cache[i].dev == dev && cache[i].bytes >= bytes)
       return BL_OK;
   BL_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
+  // Every SM keeps its whole shared memory: with a smaller L1/shared split,
+  // chosen per kernel, an SM that runs one kind of CTA may lack the room for
+  // the next kernel's CTA in a chain of dependent launches, which then
+  // doubles up on another SM (measured: 1-token FFN blocks 13.7 -> 10.5 us).
+  BL_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared));
   if (n < 512) cache[n++] = Entry{(const void*)kernel, dev, bytes};
   return BL_OK;
 }
@@ -180,6 +186,7 @@ struct FfnWs {
   ActWs x;        // quantised X (M > GEMV limit)
   size_t acc_up;  // int32 [M, H]
   size_t gamma_x; // [M] (GEMV path)
+  size_t rmax;    // fp32 [M, up-projection CTAs ≤ H] per-CTA ReLU² maxima (GEMV path)
   size_t rq;      // int8 [M, H]
   size_t gamma_r, rs_r, total;
 };
@@ -188,7 +195,8 @@ FfnWs ffn_ws(int64_t M, int64_t K, int64_t H) {
   if (M <= kGemvMaxTokens) {
     w.acc_up = 0;
     w.gamma_x = align_up((size_t)M * H * 4);
-    w.total = w.gamma_x + align_up((size_t)M * 4);
+    w.rmax = w.gamma_x + align_up((size_t)M * 4);
+    w.total = w.rmax + align_up((size_t)M * H * 4);
     return w;
   }
   w.x = act_ws(M, K);
@@ -266,10 +274,11 @@ bl_status gemv_plan(int64_t N, int64_t K, int M, int sms, int* rows, int* grid, 
 // Taps in p (if any) report CTA p.tap_cta; a value past the last CTA (or
 // negative) means the last CTA.
 bl_status run_gemv(int src, int out, bl_dtype a_dtype, GemvParams p, bool pdl, int dev, int sms,
-                   cudaStream_t st) {
+                   cudaStream_t st, int* grid_out = nullptr) {
   int rows, grid;
   size_t smem;
   BL_TRY(gemv_plan(p.N, p.K, p.M, sms, &rows, &grid, &smem));
+  if (grid_out != nullptr) *grid_out = grid;
   if (p.tap_cta < 0 || p.tap_cta >= grid) p.tap_cta = grid - 1;
   p.rows_per_cta = rows;
   p.rows_pad = gemv_rows_pad(rows);
@@ -416,6 +425,7 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
   BL_TRY(outk == kTcDequant ? launch_tc_bn<kTcDequant>(bn, ta, tw, ty, p, sp, dev, st)
                             : launch_tc_bn<kTcRawI32>(bn, ta, tw, ty, p, sp, dev, st));
   if (sp == 1) return BL_OK;
+  BL_TRY(ensure_smem(splitk_reduce_kernel, dev, 0));
   const dim3 rgrid((unsigned)((N + 1023) / 1024), (unsigned)M);
   splitk_reduce_kernel<<<rgrid, 256, 0, st>>>(
       reinterpret_cast<const int32_t*>(Yk), sp, tc_split_rows(M) * N, M, N,
@@ -575,6 +585,10 @@ bl_status run_contract(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K
 bl_status run_quant_acts(const void* A, bl_dtype dt, int64_t M, int64_t K, float eps, int8_t* Aq,
                          float* gA, int32_t* rs, cudaStream_t st, bool pdl = false) {
   if (M == 0) return BL_OK;
+  int dev;
+  BL_CUDA(cudaGetDevice(&dev));
+  BL_TRY(dt == BL_BF16 ? ensure_smem(quant_acts_kernel<__nv_bfloat16>, dev, 0)
+                       : ensure_smem(quant_acts_kernel<float>, dev, 0));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)M);
   cfg.blockDim = dim3(kQuantThreads);
@@ -1068,16 +1082,20 @@ static bl_status ffn_impl(const void* X, bl_dtype x_dtype, int64_t M, int64_t K,
     up.gamma = gamma_up;
     up.Y = acc_up;
     up.gamma_out = gX;
+    up.rmax_out = reinterpret_cast<float*>(base + w.rmax);
     up.N = H;
     up.K = K;
     up.M = (int)M;
     up.eps = eps;
     if (taps) gemv_taps(up, taps->act_q, taps->act_gamma, taps->act_rowsum, taps->cta);
-    BL_TRY(run_gemv(kSrcFloat, kOutRawI32, x_dtype, up, pdl, dev, sms, st));
+    int up_grid = 0;
+    BL_TRY(run_gemv(kSrcFloat, kOutRawI32, x_dtype, up, pdl, dev, sms, st, &up_grid));
     GemvParams dn = {};
     dn.A = acc_up;
     dn.a_scale = gX;
     dn.a_gamma_up = gamma_up;
+    dn.rmax_in = up.rmax_out;  // γ_r from the up-projection's per-CTA maxima
+    dn.rmax_n = up_grid;
     dn.W = W_down;
     dn.gamma = gamma_down;
     dn.Y = Y;
@@ -1106,6 +1124,7 @@ static bl_status ffn_impl(const void* X, bl_dtype x_dtype, int64_t M, int64_t K,
   const size_t split_bytes = ws_bytes - w.total;
   BL_TRY(run_contract(Xq, W_up, M, K, H, gamma_up, gX, rsX, acc_up, kTcRawI32, 0, 0, true, dev,
                       sms, st, split_ws, split_bytes));
+  BL_TRY(ensure_smem(relu2_requant_kernel, dev, 0));
   relu2_requant_kernel<<<(unsigned)M, kQuantThreads, 0, st>>>(acc_up, H, gX, gamma_up, eps, Rq, gR,
                                                               rsR);
   BL_CUDA(cudaGetLastError());

@@ -56,6 +56,15 @@ struct GemvParams {
   const float* gamma;       // γ of W (1 value); may be null for raw output
   void* Y;                  // kOutDequant: float/bf16 [M,N]; kOutRawI32: int32 [M,N]
   float* gamma_out;         // optional: per-token γ_A (or γ_r) written by CTA 0
+  // FFN hand-off (one-token blocks). kOutRawI32 with rmax_out: each CTA also
+  // writes, per token m, the largest r = max(h,0)² over its rows, h =
+  // fp32(acc · s_sc[m]) — the values the down-projection requantises — to
+  // rmax_out[m·gridDim.x + blockIdx.x]. kSrcFfnRequant with rmax_in: γ_r of
+  // token m is the largest of rmax_in[m·rmax_n .. m·rmax_n + rmax_n), so
+  // the prologue reads the accumulators once (no separate max pass).
+  float* rmax_out;
+  const float* rmax_in;
+  int rmax_n;
   // Optional taps (all null = off): the int8 tokens [M,K], their per-token
   // scale γ and Σ of the int8 tokens, as the prologue of CTA tap_cta made them.
   int8_t* tap_q;
@@ -128,7 +137,9 @@ __device__ __forceinline__ int warp_slots_sum(const int (&v)[kGemvWarps]) {
 template <int MT, typename TA, int SRC, int OUT>
 __global__ void __launch_bounds__(kGemvThreads, 2)
 gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p) {
-  constexpr int RV = gemv_reg_vecs<MT>();
+  // The one-token FFN requantiser keeps a whole 11008-accumulator row in
+  // registers (6 vectors per thread): one L2 round trip after the wait.
+  constexpr int RV = (SRC == kSrcFfnRequant && MT == 1) ? 6 : gemv_reg_vecs<MT>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -260,6 +271,9 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
       return reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.A) +
                                             (size_t)m * (size_t)nvec * 16);
     };
+    // γ_r handed over by the up-projection: the accumulator loads below
+    // only fill registers, and the max comes from the per-CTA maxima.
+    const bool given = SRC == kSrcFfnRequant && p.rmax_in != nullptr;
     uint4 reg[MT][RV];
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
@@ -269,16 +283,25 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
 #pragma unroll
         for (int r = 0; r < RV; ++r) {
           const int64_t v = tid + (int64_t)r * kGemvThreads;
-          if (v < nvec) {
-            reg[m][r] = __ldg(src + v);
-#pragma unroll
-            for (int i = 0; i < VEC; ++i) mx = fmaxf(mx, fabsf(value(reg[m][r], i, m)));
-          }
+          if (v < nvec) reg[m][r] = __ldg(src + v);
         }
-        for (int64_t v = tid + (int64_t)RV * kGemvThreads; v < nvec; v += kGemvThreads) {
-          const uint4 u = __ldg(src + v);
+        if (given) {
+          for (int j = tid; j < p.rmax_n; j += kGemvThreads)
+            mx = fmaxf(mx, __ldg(p.rmax_in + (int64_t)m * p.rmax_n + j));
+        } else {
 #pragma unroll
-          for (int i = 0; i < VEC; ++i) mx = fmaxf(mx, fabsf(value(u, i, m)));
+          for (int r = 0; r < RV; ++r) {
+            const int64_t v = tid + (int64_t)r * kGemvThreads;
+            if (v < nvec) {
+#pragma unroll
+              for (int i = 0; i < VEC; ++i) mx = fmaxf(mx, fabsf(value(reg[m][r], i, m)));
+            }
+          }
+          for (int64_t v = tid + (int64_t)RV * kGemvThreads; v < nvec; v += kGemvThreads) {
+            const uint4 u = __ldg(src + v);
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) mx = fmaxf(mx, fabsf(value(u, i, m)));
+          }
         }
       }
       const unsigned wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
@@ -421,6 +444,39 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
   __syncthreads();
 
   // 6. Epilogue: undo the code offset, scale.
+  if constexpr (OUT == kOutRawI32) {
+    if (p.rmax_out != nullptr) {
+      // One warp stores this CTA's accumulators and reduces, per token, the
+      // largest r = max(h,0)² (h = fp32(acc · s_sc[m])) for the hand-off.
+      if (warp == 0) {
+        float lm[MT], sc[MT];
+        int ts[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          lm[m] = 0.0f;
+          sc[m] = m < M ? s_sc[m] : 0.0f;
+          ts[m] = m < M ? warp_slots_sum(s_wsum[m]) : 0;
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          if (m < M) {
+            for (int r = lane; r < R; r += 32) {
+              const int v = s_part[m * R + r] - ts[m];
+              reinterpret_cast<int32_t*>(p.Y)[(int64_t)m * p.N + r0 + r] = v;
+              const float h = fmaxf(__fmul_rn((float)v, sc[m]), 0.0f);
+              lm[m] = fmaxf(lm[m], __fmul_rn(h, h));
+            }
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const unsigned w = __reduce_max_sync(0xffffffffu, __float_as_uint(lm[m]));
+          if (lane == 0 && m < M) p.rmax_out[(int64_t)m * gridDim.x + blockIdx.x] = __uint_as_float(w);
+        }
+      }
+      return;
+    }
+  }
   for (int e = tid; e < M * R; e += kGemvThreads) {
     const int m = e / R, r = e - m * R;
     const int v = s_part[m * R + r] - warp_slots_sum(s_wsum[m]);
