@@ -333,10 +333,12 @@ bl_status launch_tc_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tw,
                        const CUtensorMap& ty, const TcParams& p, int splits, int dev,
                        cudaStream_t st) {
   if (bn == 128) return launch_tc_t<128, OUT>(ta, tw, ty, p, splits, dev, st);
+  if (bn == 192) return launch_tc_t<192, OUT>(ta, tw, ty, p, splits, dev, st);
   return launch_tc_t<256, OUT>(ta, tw, ty, p, splits, dev, st);
 }
 
-int tc_pick_bn(int64_t M) { return M <= 128 ? 128 : 256; }
+// Token tile of K-split launches (and of the partial buffer's row padding).
+int tc_split_bn(int64_t M) { return M <= 128 ? 128 : 256; }
 
 // ---------------------------------------------------------------------------
 // K ranges for tensor-core launches whose tiles fill at most half of the SMs
@@ -346,7 +348,7 @@ int tc_pick_bn(int64_t M) { return M <= 128 ? 128 : 256; }
 constexpr int kSplitWsSms = 148;  // B200: the SM count workspaces are sized for
 
 int tc_splits(int64_t M, int64_t N, int64_t K, int sms) {
-  const int64_t tiles = ((N + 127) / 128) * ((M + tc_pick_bn(M) - 1) / tc_pick_bn(M));
+  const int64_t tiles = ((N + 127) / 128) * ((M + tc_split_bn(M) - 1) / tc_split_bn(M));
   const int64_t KB = (K + kTcBK - 1) / kTcBK;
   if (tiles * 2 > sms) return 1;
   int64_t sp = sms / tiles;
@@ -358,7 +360,7 @@ int tc_splits(int64_t M, int64_t N, int64_t K, int sms) {
 
 // Rows per split in the partial buffer: M rounded up to the token tile.
 int64_t tc_split_rows(int64_t M) {
-  const int bn = tc_pick_bn(M);
+  const int bn = tc_split_bn(M);
   return (M + bn - 1) / bn * bn;
 }
 
@@ -368,18 +370,40 @@ size_t tc_split_ws_bytes(int64_t M, int64_t N, int64_t K) {
   return sp > 1 ? align_up((size_t)sp * tc_split_rows(M) * N * 4) : 0;
 }
 
+// Token tile of an unsplit launch: the one with the fewest tile-time units,
+// rounds of tiles over the SMs × (64 + tile width). A 128 × 256 tile costs
+// about the MMAs of its 256 tokens plus a fixed part (expanding the weight
+// tile, set-up, epilogue) worth ≈64 tokens; 512 tokens × 11008 rows make 172
+// tiles of 256 (two rounds on 148 SMs) but 258 of 192 (also two, each 20 %
+// cheaper).
+int tc_pick_bn(int64_t M, int64_t N, int sms) {
+  if (M <= 128) return 128;
+  const int64_t rt = (N + 127) / 128;
+  int best = 256;
+  int64_t best_cost = -1;
+  for (int bn : {256, 192, 128}) {
+    const int64_t rounds = (rt * ((M + bn - 1) / bn) + sms - 1) / sms;
+    const int64_t cost = rounds * (64 + bn);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
 // acc/Y[M,N] = epilogue(A_q[M,K] · W_q[N,K]ᵀ − rowsum).
 bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,
                  const float* gamma, const float* gammaA, const int32_t* rowsum, void* Y,
                  int out, int relu2, int y_bf16, void* split_ws, size_t split_ws_bytes, int dev,
                  int sms, cudaStream_t st) {
   if (M > 0x7FFFFFFF || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
-  const int bn = tc_pick_bn(M);
   const int KBall = (int)((K + kTcBK - 1) / kTcBK);
   int sp = tc_splits(M, N, K, sms);
   const int sp_ws = tc_splits(M, N, K, kSplitWsSms);
   if (sp > sp_ws) sp = sp_ws;
   if (sp > 1 && (split_ws == nullptr || split_ws_bytes < tc_split_ws_bytes(M, N, K))) sp = 1;
+  const int bn = sp > 1 ? tc_split_bn(M) : tc_pick_bn(M, N, sms);
   const int kbs = sp > 1 ? ((KBall + sp - 1) / sp + 3) / 4 * 4 : KBall;
   if (sp > 1) sp = (KBall + kbs - 1) / kbs;  // no empty ranges
   void* Yk = sp > 1 ? split_ws : Y;        // where the kernel writes

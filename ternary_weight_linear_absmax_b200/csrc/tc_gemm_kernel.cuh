@@ -66,12 +66,12 @@ struct TcConfig {
   static constexpr int kBStage = BN * kTcBK;
   // Deep enough that the producer can run ahead over every weight stage
   // (4 K blocks per weight stage): small token tiles are cheap to stage.
-  static constexpr int kSStages = BN >= 256 ? 4 : (BN >= 128 ? 6 : (BN >= 64 ? 12 : (BN >= 32 ? 16 : 24)));
+  static constexpr int kSStages = BN > 128 ? 4 : (BN >= 128 ? 6 : (BN >= 64 ? 12 : (BN >= 32 ? 16 : 24)));
   // Weight ring: 128 rows × 128 packed bytes (4 K blocks) per stage, 128-byte
   // swizzle. Wide rows keep the number of TMA requests per byte low, which is
   // what bounds the stream when few tokens share each weight byte.
   static constexpr int kWStage = 128 * 128;
-  static constexpr int kWStages = BN >= 256 ? 2 : (BN >= 128 ? 3 : (BN >= 64 ? 4 : 6));
+  static constexpr int kWStages = BN > 128 ? 2 : (BN >= 128 ? 3 : (BN >= 64 ? 4 : 6));
   static constexpr int kTStages = 4;  // TMEM A stages (32 columns = one K block each)
   // Independent accumulators: consecutive MMAs into one accumulator are
   // serialised by its read-modify-write, which dominates for small N. The

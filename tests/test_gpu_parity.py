@@ -171,6 +171,7 @@ ZG_CASES = [
     (7, 64, 20000), (64, 4096, 4096), (32, 4096, 11008),
     (65, 256, 200), (100, 320, 256), (128, 256, 128), (129, 640, 260),  # tensor-core path
     (256, 512, 384), (300, 384, 512), (520, 128, 136),
+    (384, 128, 7680), (300, 256, 9000),  # 192-token tiles (one round instead of two of 128)
 ]
 
 
@@ -294,7 +295,8 @@ def test_linear_prefill_sampled(bl):
                  rows=list(range(0, 160)) + list(range(4000, 4096)))
 
 
-@pytest.mark.parametrize("M,K,N", [(5, 192, 200), (37, 512, 300), (200, 320, 128), (64, 2560, 512)])
+@pytest.mark.parametrize("M,K,N", [(5, 192, 200), (37, 512, 300), (200, 320, 128), (64, 2560, 512),
+                                   (330, 256, 9000)])
 @pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
 def test_linear_ragged(bl, M, K, N, out):
     _linear_case(bl, M, K, N, "f32", "f32", True, out, relu2=(M % 2 == 1))
