@@ -304,11 +304,11 @@ bl_status run_gemv(int src, int out, bl_dtype a_dtype, GemvParams p, bool pdl, i
 
 // --------------------------------------------------------------------------
 // Tensor-core launches.
-template <int BN, int OUT>
+template <int BN, bool DUAL, int OUT>
 bl_status launch_tc_t(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& ty,
                       const TcParams& p, int splits, int dev, cudaStream_t st) {
-  auto* k = tc_ternary_gemm_kernel<BN, OUT>;
-  constexpr size_t smem = TcConfig<BN>::kSmemBytes;
+  auto* k = tc_ternary_gemm_kernel<TcConfig<BN, DUAL>, OUT>;
+  constexpr size_t smem = TcConfig<BN, DUAL>::kSmemBytes;
   BL_TRY(ensure_smem(k, dev, smem));
   // Always with programmatic dependent launch: the kernel waits for the
   // previous grid before it touches global memory.
@@ -326,15 +326,24 @@ bl_status launch_tc_t(const CUtensorMap& ta, const CUtensorMap& tw, const CUtens
   return BL_OK;
 }
 
-// Token tiles of 128 or 256: the tensor-core path only sees M > 64 (fewer
-// tokens take the skinny kernel).
+// Token tile of a launch: width 128, 192 or 256 (the tensor-core path only
+// sees M > 64; fewer tokens take the skinny kernel), one or two CTAs per SM.
+struct TcTile {
+  int bn;
+  bool dual;
+};
+
 template <int OUT>
-bl_status launch_tc_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tw,
+bl_status launch_tc_bn(TcTile t, const CUtensorMap& ta, const CUtensorMap& tw,
                        const CUtensorMap& ty, const TcParams& p, int splits, int dev,
                        cudaStream_t st) {
-  if (bn == 128) return launch_tc_t<128, OUT>(ta, tw, ty, p, splits, dev, st);
-  if (bn == 192) return launch_tc_t<192, OUT>(ta, tw, ty, p, splits, dev, st);
-  return launch_tc_t<256, OUT>(ta, tw, ty, p, splits, dev, st);
+  if (t.bn == 128)
+    return t.dual ? launch_tc_t<128, true, OUT>(ta, tw, ty, p, splits, dev, st)
+                  : launch_tc_t<128, false, OUT>(ta, tw, ty, p, splits, dev, st);
+  if (t.bn == 192)
+    return t.dual ? launch_tc_t<192, true, OUT>(ta, tw, ty, p, splits, dev, st)
+                  : launch_tc_t<192, false, OUT>(ta, tw, ty, p, splits, dev, st);
+  return launch_tc_t<256, false, OUT>(ta, tw, ty, p, splits, dev, st);
 }
 
 // Token tile of K-split launches (and of the partial buffer's row padding).
@@ -376,8 +385,8 @@ size_t tc_split_ws_bytes(int64_t M, int64_t N, int64_t K) {
 // tile, set-up, epilogue) worth ≈64 tokens; 512 tokens × 11008 rows make 172
 // tiles of 256 (two rounds on 148 SMs) but 258 of 192 (also two, each 20 %
 // cheaper).
-int tc_pick_bn(int64_t M, int64_t N, int sms) {
-  if (M <= 128) return 128;
+TcTile tc_pick_tile(int64_t M, int64_t N, int sms) {
+  if (M <= 128) return TcTile{128, false};
   const int64_t rt = (N + 127) / 128;
   int best = 256;
   int64_t best_cost = -1;
@@ -389,7 +398,15 @@ int tc_pick_bn(int64_t M, int64_t N, int sms) {
       best = bn;
     }
   }
-  return best;
+  // Two CTAs per SM with 192-token tiles when those fit in one co-resident
+  // wave and the best single-CTA tile needs two or more rounds: one CTA's
+  // epilogue and set-up then overlap the other's MMAs (512 tokens × 11008
+  // rows: 258 tiles; FFN block 65.7 -> 60.8 us). The prefill shape (352
+  // tiles of 192) stays on 256-token single tiles (32.4 us vs 37.4 dual).
+  const int64_t t192 = rt * ((M + 191) / 192);
+  const int64_t tbest = rt * ((M + best - 1) / best);
+  if (t192 <= 2 * (int64_t)sms && tbest > sms) return TcTile{192, true};
+  return TcTile{best, false};
 }
 
 // acc/Y[M,N] = epilogue(A_q[M,K] · W_q[N,K]ᵀ − rowsum).
@@ -403,7 +420,8 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
   const int sp_ws = tc_splits(M, N, K, kSplitWsSms);
   if (sp > sp_ws) sp = sp_ws;
   if (sp > 1 && (split_ws == nullptr || split_ws_bytes < tc_split_ws_bytes(M, N, K))) sp = 1;
-  const int bn = sp > 1 ? tc_split_bn(M) : tc_pick_bn(M, N, sms);
+  const TcTile tile = sp > 1 ? TcTile{tc_split_bn(M), false} : tc_pick_tile(M, N, sms);
+  const int bn = tile.bn;
   const int kbs = sp > 1 ? ((KBall + sp - 1) / sp + 3) / 4 * 4 : KBall;
   if (sp > 1) sp = (KBall + kbs - 1) / kbs;  // no empty ranges
   void* Yk = sp > 1 ? split_ws : Y;        // where the kernel writes
@@ -446,8 +464,8 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
   p.y_bf16 = y_bf16;
   p.kb_per_split = kbs;
   p.split_rows = sp > 1 ? tc_split_rows(M) : 0;
-  BL_TRY(outk == kTcDequant ? launch_tc_bn<kTcDequant>(bn, ta, tw, ty, p, sp, dev, st)
-                            : launch_tc_bn<kTcRawI32>(bn, ta, tw, ty, p, sp, dev, st));
+  BL_TRY(outk == kTcDequant ? launch_tc_bn<kTcDequant>(tile, ta, tw, ty, p, sp, dev, st)
+                            : launch_tc_bn<kTcRawI32>(tile, ta, tw, ty, p, sp, dev, st));
   if (sp == 1) return BL_OK;
   BL_TRY(ensure_smem(splitk_reduce_kernel, dev, 0));
   const dim3 rgrid((unsigned)((N + 1023) / 1024), (unsigned)M);

@@ -60,24 +60,32 @@ struct TcParams {
   int64_t split_rows;  // Mp (0 when unsplit)
 };
 
-template <int BN>
+// DUAL: two CTAs per SM (BN 128 or 192). Each CTA then fits in half of the
+// SM's shared memory and TMEM (256 columns: one accumulator, and 4 or 2 A
+// stages), so one CTA's epilogue and set-up overlap the other's MMAs.
+template <int BN_, bool DUAL_ = false>
 struct TcConfig {
+  static constexpr int BN = BN_;
+  static constexpr bool kDual = DUAL_;
+  static_assert(!DUAL_ || BN_ == 128 || BN_ == 192, "two CTAs per SM need BN 128 or 192");
   // Token ring: one 128-byte-wide K block (BN rows, 128-byte swizzle) per stage.
   static constexpr int kBStage = BN * kTcBK;
   // Deep enough that the producer can run ahead over every weight stage
   // (4 K blocks per weight stage): small token tiles are cheap to stage.
-  static constexpr int kSStages = BN > 128 ? 4 : (BN >= 128 ? 6 : (BN >= 64 ? 12 : (BN >= 32 ? 16 : 24)));
+  static constexpr int kSStages = DUAL_ ? (BN > 128 ? 3 : 4)
+                                        : BN > 128 ? 4 : (BN >= 128 ? 6 : (BN >= 64 ? 12 : (BN >= 32 ? 16 : 24)));
   // Weight ring: 128 rows × 128 packed bytes (4 K blocks) per stage, 128-byte
   // swizzle. Wide rows keep the number of TMA requests per byte low, which is
   // what bounds the stream when few tokens share each weight byte.
   static constexpr int kWStage = 128 * 128;
-  static constexpr int kWStages = BN > 128 ? 2 : (BN >= 128 ? 3 : (BN >= 64 ? 4 : 6));
-  static constexpr int kTStages = 4;  // TMEM A stages (32 columns = one K block each)
+  static constexpr int kWStages = DUAL_ ? 2 : BN > 128 ? 2 : (BN >= 128 ? 3 : (BN >= 64 ? 4 : 6));
+  // TMEM A stages (32 columns = one K block each).
+  static constexpr int kTStages = DUAL_ && BN > 128 ? 2 : 4;
   // Independent accumulators: consecutive MMAs into one accumulator are
   // serialised by its read-modify-write, which dominates for small N. The
   // four MMAs of a stage rotate over kAcc accumulators, summed in the
   // epilogue (exact integer addition).
-  static constexpr int kAcc = BN <= 64 ? 4 : (BN <= 128 ? 2 : 1);
+  static constexpr int kAcc = DUAL_ ? 1 : BN <= 64 ? 4 : (BN <= 128 ? 2 : 1);
   static constexpr int kDCols = BN < 32 ? 32 : BN;  // columns per accumulator
   static constexpr int kACol = kAcc * kDCols;
   static constexpr int kColsNeeded = kACol + kTStages * 32;
@@ -92,11 +100,13 @@ struct TcConfig {
   static constexpr int kBarBytes =
       ((2 * kSStages + 2 * kWStages + 2 * kTStages + 2 + kStoreChunks) * 8 + 15) / 16 * 16;
   static constexpr int kParamBytes = BN * 8;
-  // 1 KiB slack for aligning the dynamic buffer to 1024 bytes. At least
-  // 116 KiB are requested so that only one CTA is resident per SM: every CTA
-  // then gets its TMEM columns without waiting on another CTA's allocation.
+  // 1 KiB slack for aligning the dynamic buffer to 1024 bytes. Single
+  // configurations request at least 116 KiB so that only one CTA is resident
+  // per SM: every CTA then gets its TMEM columns without waiting on another
+  // CTA's allocation. Dual ones fit two per SM, 256 TMEM columns each.
   static constexpr int kSmemUsed = 1024 + kRingBytes + kBarBytes + kParamBytes + 64;
-  static constexpr int kSmemBytes = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
+  static constexpr int kSmemBytes = DUAL_ ? kSmemUsed : (kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024);
+  static_assert(!DUAL_ || (kTmemCols <= 256 && kSmemBytes <= 112 * 1024), "dual CTA too large");
   // The output staging tile reuses the ring.
   static_assert(BN * 128 * 4 <= kRingBytes, "staging tile must fit in the ring");
 };
@@ -189,11 +199,11 @@ __device__ __forceinline__ void tc_epilogue_chunk(const uint32_t (&d)[CW], int c
 // Whole-tile epilogue for one thread's TMEM lane: loads CW columns at a time
 // (summing the kAcc accumulators), with the next chunk's load issued before
 // the current chunk is processed.
-template <int BN, int OUT, bool RELU, bool BF16, bool STAGE>
+template <class C, int OUT, bool RELU, bool BF16, bool STAGE>
 __device__ __forceinline__ void tc_epilogue(uint32_t t_lane, int row, int half, const float* s_sc,
                                             const int* s_rs, uint8_t* stage, const TcParams& p,
                                             int64_t m0, int64_t n, int64_t zrow, uint64_t* staged) {
-  using C = TcConfig<BN>;
+  constexpr int BN = C::BN;
   // 16-column chunks, alternating between the two warps of a lane quarter.
   constexpr int CW = 16;
   const int c_begin = half * CW;
@@ -234,12 +244,12 @@ __device__ __forceinline__ void tc_epilogue(uint32_t t_lane, int row, int half, 
   }
 }
 
-template <int BN, int OUT>
-__global__ void __launch_bounds__(kTcThreads, 1)
+template <class C, int OUT>
+__global__ void __launch_bounds__(kTcThreads, C::kDual ? 2 : 1)
 tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
                        const __grid_constant__ CUtensorMap tm_w,
                        const __grid_constant__ CUtensorMap tm_y, const TcParams p) {
-  using C = TcConfig<BN>;
+  constexpr int BN = C::BN;
   constexpr int SS = C::kSStages, WS = C::kWStages, TS = C::kTStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -439,20 +449,20 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
       const uint32_t t_lane = tmem + lane_addr;
       if constexpr (OUT == kTcRawI32) {
         if (p.tma_store)
-          tc_epilogue<BN, OUT, false, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged);
+          tc_epilogue<C, OUT, false, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged);
         else
-          tc_epilogue<BN, OUT, false, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged);
+          tc_epilogue<C, OUT, false, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged);
       } else {
         const int sel = (p.tma_store ? 4 : 0) | (p.y_bf16 ? 2 : 0) | (p.relu2 ? 1 : 0);
         switch (sel) {
-          case 0: tc_epilogue<BN, OUT, false, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
-          case 1: tc_epilogue<BN, OUT, true, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
-          case 2: tc_epilogue<BN, OUT, false, true, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
-          case 3: tc_epilogue<BN, OUT, true, true, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
-          case 4: tc_epilogue<BN, OUT, false, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
-          case 5: tc_epilogue<BN, OUT, true, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
-          case 6: tc_epilogue<BN, OUT, false, true, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
-          default: tc_epilogue<BN, OUT, true, true, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
+          case 0: tc_epilogue<C, OUT, false, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
+          case 1: tc_epilogue<C, OUT, true, false, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
+          case 2: tc_epilogue<C, OUT, false, true, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
+          case 3: tc_epilogue<C, OUT, true, true, false>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
+          case 4: tc_epilogue<C, OUT, false, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
+          case 5: tc_epilogue<C, OUT, true, false, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
+          case 6: tc_epilogue<C, OUT, false, true, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
+          default: tc_epilogue<C, OUT, true, true, true>(t_lane, row, hw, s_sc, s_rs, smem, p, m0, n, zrow, staged); break;
         }
       }
     }

@@ -172,6 +172,7 @@ ZG_CASES = [
     (65, 256, 200), (100, 320, 256), (128, 256, 128), (129, 640, 260),  # tensor-core path
     (256, 512, 384), (300, 384, 512), (520, 128, 136),
     (384, 128, 7680), (300, 256, 9000),  # 192-token tiles (one round instead of two of 128)
+    (512, 128, 11008),  # 192-token tiles, two CTAs per SM
 ]
 
 
@@ -296,7 +297,7 @@ def test_linear_prefill_sampled(bl):
 
 
 @pytest.mark.parametrize("M,K,N", [(5, 192, 200), (37, 512, 300), (200, 320, 128), (64, 2560, 512),
-                                   (330, 256, 9000)])
+                                   (330, 256, 9000), (400, 256, 11008)])
 @pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
 def test_linear_ragged(bl, M, K, N, out):
     _linear_case(bl, M, K, N, "f32", "f32", True, out, relu2=(M % 2 == 1))
