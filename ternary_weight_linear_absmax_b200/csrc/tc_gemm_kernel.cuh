@@ -70,10 +70,12 @@ struct TcConfig {
   static_assert(!DUAL_ || BN_ == 128 || BN_ == 192, "two CTAs per SM need BN 128 or 192");
   // Token ring: one 128-byte-wide K block (BN rows, 128-byte swizzle) per stage.
   static constexpr int kBStage = BN * kTcBK;
-  // Deep enough that the producer can run ahead over every weight stage
-  // (4 K blocks per weight stage): small token tiles are cheap to stage.
+  // Deep enough to cover the L2 latency of the token tiles at the rate the
+  // MMAs consume them (one 256-token tile, 32 KB, per ≈640 cycles): with four
+  // stages the loads alone, without any MMA, bounded the prefill at 29 us.
+  // Single configurations use what the 227 KB of shared memory allows.
   static constexpr int kSStages = DUAL_ ? (BN > 128 ? 3 : 4)
-                                        : BN > 128 ? 4 : (BN >= 128 ? 6 : (BN >= 64 ? 12 : (BN >= 32 ? 16 : 24)));
+                                        : BN > 192 ? 5 : (BN > 128 ? 7 : (BN >= 128 ? 10 : (BN >= 64 ? 12 : (BN >= 32 ? 16 : 24))));
   // Weight ring: 128 rows × 128 packed bytes (4 K blocks) per stage, 128-byte
   // swizzle. Wide rows keep the number of TMA requests per byte low, which is
   // what bounds the stream when few tokens share each weight byte.
@@ -107,6 +109,7 @@ struct TcConfig {
   static constexpr int kSmemUsed = 1024 + kRingBytes + kBarBytes + kParamBytes + 64;
   static constexpr int kSmemBytes = DUAL_ ? kSmemUsed : (kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024);
   static_assert(!DUAL_ || (kTmemCols <= 256 && kSmemBytes <= 112 * 1024), "dual CTA too large");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory of one CTA");
   // The output staging tile reuses the ring.
   static_assert(BN * 128 * 4 <= kRingBytes, "staging tile must fit in the ring");
 };
