@@ -761,8 +761,13 @@ def profile_case(name: str) -> int:
         pk, g = bl.bl_quant_weights(W, EPS)
         dY = si.activations(M, N, seed=5, dtype="bf16").torch(device)
         torch.cuda.synchronize()
+        A = si.activations(M, K, seed=0, dtype="bf16").torch(device)
+        Aq, gA, _ = bl.bl_quant_acts(A, EPS)
+        torch.cuda.synchronize()
         for _ in range(2):
             bl.bl_ste_grad_input(dY, pk, g, stream=st)
+        for _ in range(2):
+            bl.bl_ste_grad_weight(dY, Aq, gA, W, g, EPS, stream=st)
     else:
         raise SystemExit(f"unknown profile case {name}")
     st.synchronize()

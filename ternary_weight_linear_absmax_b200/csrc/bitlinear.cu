@@ -1552,16 +1552,17 @@ bl_status bl_ste_grad_weight(const void* dY, bl_dtype dy_dtype, int64_t M, int64
   uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
   __nv_bfloat16* dyt = reinterpret_cast<__nv_bfloat16*>(base);
   __nv_bfloat16* aht = reinterpret_cast<__nv_bfloat16*>(base + align_up((size_t)N * Mp * 2));
-  const dim3 gt((unsigned)((N + 31) / 32), (unsigned)((Mp + 31) / 32));
+  // dYᵀ [N, Mp] and Âᵀ [K, Mp] (N, K multiples of 8; Mp of 8).
+  const dim3 gy((unsigned)((N + 63) / 64), (unsigned)((Mp + 63) / 64));
   if (dy_dtype == BL_BF16)
-    transpose_bf16_kernel<__nv_bfloat16><<<gt, 256, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16*>(dY), M, N, Mp, dyt);
+    transpose64_bf16_kernel<__nv_bfloat16><<<gy, 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(dY), nullptr, M, N, Mp, dyt);
   else
-    transpose_bf16_kernel<float><<<gt, 256, 0, st>>>(reinterpret_cast<const float*>(dY), M, N, Mp,
-                                                     dyt);
+    transpose64_bf16_kernel<float><<<gy, 256, 0, st>>>(reinterpret_cast<const float*>(dY), nullptr,
+                                                       M, N, Mp, dyt);
   BL_CUDA(cudaGetLastError());
-  ahat_t_kernel<<<dim3((unsigned)((K + 31) / 32), (unsigned)((Mp + 31) / 32)), 256, 0, st>>>(
-      A_q, gamma_A, M, K, Mp, aht);
+  transpose64_bf16_kernel<int8_t><<<dim3((unsigned)((K + 63) / 64), (unsigned)((Mp + 63) / 64)), 256,
+                                    0, st>>>(A_q, gamma_A, M, K, Mp, aht);
   BL_CUDA(cudaGetLastError());
   GmParams p = {};
   p.rows = N;

@@ -172,37 +172,26 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
     // ---- epilogue: warps 2..5, TMEM lane quarter warp % 4 ----
     const int q = warp & 3;
     const int64_t r = r0 + 32 * q + lane;
-    bool ok = mbar_wait(done, 0);
-    ok = __all_sync(0xffffffffu, ok && !*s_abort);  // tcgen05.ld is warp-collective
-    if (ok) {
-      tc_fence_after();
-      const float scale = p.scale != nullptr ? __ldg(p.scale) : 1.0f;
-      double thr = 0.0;
-      if constexpr (MASK) {
-        const float g = __fadd_rn(__ldg(p.mask_gamma), p.eps);
-        thr = (double)g * (1.0 + 0x1p-24);  // |fl32(W ÷ g)| ≤ 1  ⟺  |W| ≤ g·(1 + 2^-24)
-      }
-      const uint32_t t_lane = tmem + ((uint32_t)(32 * q) << 16);
-#pragma unroll 1
-      for (int cc = 0; cc < BN; cc += 16) {
-        uint32_t d[16];
-        tmem_ld_32x32b_x16(t_lane + cc, d);
-        tmem_wait_ld();
-        const int64_t col = c0 + cc;
-        if (r >= p.rows || col >= p.cols) continue;
-        float v[16];
+    // STE mask of this thread's row, read while the MMAs run (the latent
+    // weights are read once): bit c of mbits[c/32] keeps column c0 + c.
+    // |fl32(W ÷ g)| ≤ 1 ⟺ |W| ≤ g·(1 + 2^-24) (exact in double); for an fp32
+    // W that equals |W| ≤ the largest fp32 not above that bound.
+    uint32_t mbits[MASK ? BN / 32 : 1];
+    if constexpr (MASK) {
+      const float g = __fadd_rn(__ldg(p.mask_gamma), p.eps);
+      const float thr = __double2float_rd((double)g * (1.0 + 0x1p-24));
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(__uint_as_float(d[j]), scale);
-        if constexpr (MASK) {
-          // This thread's 16 contiguous latent weights in 16-byte loads
-          // (cols is a multiple of 64 and col of 16, so they are aligned).
-          float w[16];
+      for (int cw = 0; cw < BN / 32; ++cw) {
+        uint32_t bits = 0u;
+        const int64_t col = c0 + 32 * cw;
+        if (r < p.rows && col < p.cols) {  // cols is a multiple of 64: whole groups of 32
           const int64_t o = r * p.cols + col;
+          float w[32];
           if (p.mask_bf16) {
             const uint4* src = reinterpret_cast<const uint4*>(
                 reinterpret_cast<const __nv_bfloat16*>(p.mask_w) + o);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < 4; ++h) {
               const uint4 u = __ldg(src + h);
               const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&u);
 #pragma unroll
@@ -211,7 +200,7 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
           } else {
             const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.mask_w) + o);
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
+            for (int h = 0; h < 8; ++h) {
               const float4 f = __ldg(src + h);
               w[4 * h] = f.x;
               w[4 * h + 1] = f.y;
@@ -220,8 +209,35 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
             }
           }
 #pragma unroll
+          for (int j = 0; j < 32; ++j) bits |= (fabsf(w[j]) <= thr ? 1u : 0u) << j;
+        }
+        mbits[cw] = bits;
+      }
+    }
+    bool ok = mbar_wait(done, 0);
+    ok = __all_sync(0xffffffffu, ok && !*s_abort);  // tcgen05.ld is warp-collective
+    if (ok) {
+      tc_fence_after();
+      const float scale = p.scale != nullptr ? __ldg(p.scale) : 1.0f;
+      const uint32_t t_lane = tmem + ((uint32_t)(32 * q) << 16);
+      // Chunk cc+16 is loaded (warp-collective) while chunk cc is processed.
+      uint32_t d[2][16];
+      tmem_ld_32x32b_x16(t_lane, d[0]);
+#pragma unroll
+      for (int cc = 0; cc < BN; cc += 16) {
+        tmem_wait_ld();
+        if (cc + 16 < BN) tmem_ld_32x32b_x16(t_lane + cc + 16, d[((cc >> 4) + 1) & 1]);
+        const uint32_t(&dc)[16] = d[(cc >> 4) & 1];
+        const int64_t col = c0 + cc;
+        if (r >= p.rows || col >= p.cols) continue;
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(__uint_as_float(dc[j]), scale);
+        if constexpr (MASK) {
+          const uint32_t bits = mbits[cc >> 5] >> (cc & 31);
+#pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (fabs((double)w[j]) > thr) v[j] = 0.0f;
+            if (!((bits >> j) & 1u)) v[j] = 0.0f;
         }
         float* out = p.C + r * p.cols + col;
         if (col + 16 <= p.cols && (p.cols & 3) == 0) {
@@ -279,24 +295,83 @@ expand_wqt_kernel(const uint8_t* __restrict__ W, int64_t N, int64_t K, int64_t N
   }
 }
 
-// Transpose-convert an [R, Cc] fp32/bf16 matrix, with rows scaled by an
-// optional per-row factor, into [Cc, Rp] bf16 (columns r ≥ R zero).
-// Used for dYᵀ (factor none) and for Âᵀ from int8 A_q (see below).
+// Transpose-convert an [R, Cc] matrix (bf16, fp32 or int8; Cc a multiple of
+// 8) into [Cc, Rp] bf16 (Rp a multiple of 8; rows r ≥ R give zeros), row r
+// optionally scaled by fp32(rscale[r] ÷ 127): dYᵀ, and Âᵀ from int8 A_q with
+// Â[m, k] = fp32(γ_A[m] ÷ 127) · A_q[m, k]. 64 × 64 tiles: each thread reads
+// 8 consecutive elements of a row and writes 8 consecutive bf16 of an output
+// row; the tile's 16-byte chunks are swizzled by row ÷ 8 so that both passes
+// are free of shared-memory bank conflicts.
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+}
+
+template <typename T>
+__device__ __forceinline__ void load8_f32(const T* p, float (&v)[8]) {
+  if constexpr (sizeof(T) == 1) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    const int8_t* b = reinterpret_cast<const int8_t*>(&u);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = (float)b[j];
+  } else if constexpr (sizeof(T) == 2) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = __bfloat162float(b[j]);
+  } else {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256)
-transpose_bf16_kernel(const T* __restrict__ in, int64_t R, int64_t Cc, int64_t Rp,
-                      __nv_bfloat16* __restrict__ out) {
-  __shared__ float tile[32][33];
-  const int64_t c0 = (int64_t)blockIdx.x * 32, rr0 = (int64_t)blockIdx.y * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int i = ty; i < 32; i += 8) {
-    const int64_t r = rr0 + i, c = c0 + tx;
-    tile[i][tx] = (r < R && c < Cc) ? to_f32<T>(in[r * Cc + c]) : 0.0f;
+transpose64_bf16_kernel(const T* __restrict__ in, const float* __restrict__ rscale, int64_t R,
+                        int64_t Cc, int64_t Rp, __nv_bfloat16* __restrict__ out) {
+  __shared__ __align__(16) uint4 tile[64][8];  // 64 rows × 64 bf16
+  const int64_t c0 = (int64_t)blockIdx.x * 64, r0 = (int64_t)blockIdx.y * 64;
+  const int tid = threadIdx.x;
+  for (int e = tid; e < 64 * 8; e += 256) {
+    const int i = e >> 3, g = e & 7;
+    const int64_t r = r0 + i, c = c0 + 8 * g;
+    float v[8];
+    if (r < R && c < Cc) {
+      load8_f32<T>(in + r * Cc + c, v);
+      if (rscale != nullptr) {
+        const float sc = __fdiv_rn(__ldg(rscale + r), 127.0f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(sc, v[j]);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = 0.0f;
+    }
+    uint4 w;
+    w.x = bf16x2_bits(v[0], v[1]);
+    w.y = bf16x2_bits(v[2], v[3]);
+    w.z = bf16x2_bits(v[4], v[5]);
+    w.w = bf16x2_bits(v[6], v[7]);
+    tile[i][g ^ ((i >> 3) & 7)] = w;
   }
   __syncthreads();
-  for (int i = ty; i < 32; i += 8) {
-    const int64_t c = c0 + i, r = rr0 + tx;
-    if (c < Cc && r < Rp) out[c * Rp + r] = __float2bfloat16_rn(tile[tx][i]);
+  const uint16_t* tb = reinterpret_cast<const uint16_t*>(&tile[0][0]);
+  for (int e = tid; e < 64 * 8; e += 256) {
+    const int cc = e >> 3, l = e & 7;  // output row c0 + cc, columns r0 + 8l .. + 7
+    const int64_t c = c0 + cc, r = r0 + 8 * l;
+    if (c >= Cc || r >= Rp) continue;
+    uint32_t h[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)  // tile row 8l + j: its chunk cc/8 sits at slot (cc/8) ^ l
+      h[j] = tb[(8 * l + j) * 64 + ((((cc >> 3) ^ l)) << 3) + (cc & 7)];
+    uint4 w;
+    w.x = h[0] | (h[1] << 16);
+    w.y = h[2] | (h[3] << 16);
+    w.z = h[4] | (h[5] << 16);
+    w.w = h[6] | (h[7] << 16);
+    *reinterpret_cast<uint4*>(out + c * Rp + r) = w;
   }
 }
 
@@ -309,26 +384,6 @@ convert_bf16_kernel(const float* __restrict__ in, int64_t n, __nv_bfloat16* __re
     __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(out + 4 * i);
     o[0] = __floats2bfloat162_rn(v.x, v.y);
     o[1] = __floats2bfloat162_rn(v.z, v.w);
-  }
-}
-
-// Âᵀ [K, Mp] bf16: Â[m, k] = fp32(γ_A[m] ÷ 127) · A_q[m, k] (columns m ≥ M zero).
-__global__ void __launch_bounds__(256)
-ahat_t_kernel(const int8_t* __restrict__ Aq, const float* __restrict__ gammaA, int64_t M,
-              int64_t K, int64_t Mp, __nv_bfloat16* __restrict__ out) {
-  __shared__ float tile[32][33];
-  const int64_t k0 = (int64_t)blockIdx.x * 32, m0 = (int64_t)blockIdx.y * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int i = ty; i < 32; i += 8) {
-    const int64_t m = m0 + i, k = k0 + tx;
-    float a = 0.0f;
-    if (m < M && k < K) a = __fmul_rn(__fdiv_rn(__ldg(gammaA + m), 127.0f), (float)Aq[m * K + k]);
-    tile[i][tx] = a;
-  }
-  __syncthreads();
-  for (int i = ty; i < 32; i += 8) {
-    const int64_t k = k0 + i, m = m0 + tx;
-    if (k < K && m < Mp) out[k * Mp + m] = __float2bfloat16_rn(tile[tx][i]);
   }
 }
 
