@@ -1491,7 +1491,7 @@ bl_status bl_ste_grad_input(const void* dY, bl_dtype dy_dtype, int64_t M, int64_
   uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
   __nv_bfloat16* wqt = reinterpret_cast<__nv_bfloat16*>(base);
   const int64_t Np = round8(N);
-  expand_wqt_kernel<<<dim3((unsigned)((Np + 31) / 32), (unsigned)(K / 64)), 256, 0, st>>>(
+  expand_wqt_kernel<<<dim3((unsigned)((Np + 63) / 64), (unsigned)(K / 64)), 256, 0, st>>>(
       W_packed, N, K, Np, wqt);
   BL_CUDA(cudaGetLastError());
   const void* a = dY;

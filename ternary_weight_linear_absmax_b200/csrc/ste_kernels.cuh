@@ -263,22 +263,24 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
 }
 
 // ---------------------------------------------------------------------------
-// Layout kernels (32 × 32 tiles through shared memory, 256 threads).
+// Layout kernels (64 × 64 tiles through shared memory, 256 threads).
 
 // W_qᵀ [K, Np] bf16 from the packed codes [N, K/4]: element (k, n) = c(n,k) - 1
-// (columns n ≥ N are zero). Block tile: 32 rows n × 64 weights k. 128 threads
-// each load one 32-bit word (16 codes) and expand it into the tile; then all
-// 256 threads write 64 rows k × 32 columns n (64 contiguous bytes per row).
+// (columns n ≥ N are zero; Np a multiple of 8). Block tile: 64 rows n × 64
+// weights k. Each thread loads one 32-bit word (16 codes; the 32 lanes of a
+// warp take 32 rows n at the same word) and expands it into the tile's
+// column n; then each thread writes 8 consecutive n of an output row k with
+// one 16-byte store.
 __global__ void __launch_bounds__(256)
 expand_wqt_kernel(const uint8_t* __restrict__ W, int64_t N, int64_t K, int64_t Np,
                   __nv_bfloat16* __restrict__ out) {
-  __shared__ __nv_bfloat16 tile[64][34];
-  const int64_t n0 = (int64_t)blockIdx.x * 32, k0 = (int64_t)blockIdx.y * 64;
+  __shared__ __align__(16) __nv_bfloat16 tile[64][72];  // [k][n], rows 16-byte aligned
+  const int64_t n0 = (int64_t)blockIdx.x * 64, k0 = (int64_t)blockIdx.y * 64;
   const int tid = threadIdx.x;
-  if (tid < 128) {
-    const int i = tid >> 2, q = tid & 3;  // row n0+i, word q of the 64 weights
+  {
+    const int i = tid & 63, q = tid >> 6;  // row n0+i, word q of the 64 weights
     const int64_t n = n0 + i;
-    uint32_t word = 0x55555555u;          // codes 1 (w = 0) past N
+    uint32_t word = 0x55555555u;           // codes 1 (w = 0) past N
     if (n < N) word = __ldg(reinterpret_cast<const uint32_t*>(W + n * (K / 4)) + (k0 >> 4) + q);
 #pragma unroll
     for (int e = 0; e < 16; ++e) {  // weight 16q + 4j + i2 at bits 8·i2 + 2·j
@@ -288,10 +290,11 @@ expand_wqt_kernel(const uint8_t* __restrict__ W, int64_t N, int64_t K, int64_t N
     }
   }
   __syncthreads();
-  const int tx = tid & 31, ty = tid >> 5;
-  for (int r = ty; r < 64; r += 8) {
-    const int64_t k = k0 + r, n = n0 + tx;
-    if (k < K && n < Np) out[k * Np + n] = tile[r][tx];
+  for (int e = tid; e < 64 * 8; e += 256) {
+    const int r = e >> 3, g = e & 7;  // output row k0 + r, columns n0 + 8g .. + 7
+    const int64_t n = n0 + 8 * g;
+    if (n < Np)
+      *reinterpret_cast<uint4*>(out + (k0 + r) * Np + n) = *reinterpret_cast<const uint4*>(&tile[r][8 * g]);
   }
 }
 
