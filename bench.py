@@ -562,6 +562,41 @@ def run_ffn(bl, device, peaks, Ms=(1, 64, 512), reps=10):
     return out
 
 
+def run_tp_ffn_shard(bl, device, worlds=(2, 4, 8), Ms=(1, 64, 512), reps=10):
+    """One rank's compute in the tensor-parallel FFN block (4096 -> 11008 ->
+    4096; the hidden dimension split over `world` ranks): the up step on its
+    shard, the requantised down step and the final dequantisation, timed on
+    one GPU over rotating weight shards larger than L2. The two all-reduces
+    between them (MAX of M fp32, SUM of M x 4096 INT32) are not included;
+    their payloads are reported."""
+    import torch
+    from ternary_weight_linear_absmax_b200.tp_ffn import shard_packed
+    K, H = 4096, 11008
+    stream = torch.cuda.Stream(device)
+    pu, gu = bl.bl_quant_weights(si.weights(H, K, seed=1, dtype="bf16").torch(device), EPS)
+    pd, gd = bl.bl_quant_weights(si.weights(K, H, seed=2, dtype="bf16").torch(device), EPS)
+    out = {"note": "per-rank compute only; collectives excluded", "workload": "FFN 4096->11008->4096"}
+    for world in worlds:
+        pu_r, pd_r = shard_packed(pu, pd, H, world, 0)
+        H_r = pu_r.shape[0]
+        res = {"H_r": H_r}
+        for M in Ms:
+            X = si.activations(M, K, seed=0, dtype="bf16").torch(device)
+            P = n_sets(pu_r.numel() + pd_r.numel() + M * H_r * 4, device.index)
+            sets = [(torch.roll(pu_r, shifts=37 * i, dims=0).contiguous(),
+                     torch.roll(pd_r, shifts=41 * i, dims=0).contiguous()) for i in range(P)]
+
+            def step(s):
+                acc, gx, rmax = bl.bl_ffn_tp_up(X, s[0], gu, EPS, stream=stream)
+                part = bl.bl_ffn_tp_down(acc, gx, gu, rmax, s[1], EPS, stream=stream)
+                bl.bl_dequant_i32(part, rmax, gd, stream=stream)
+            t = rotating_time([lambda s=s_: step(s) for s_ in sets], stream, reps)
+            res[f"M{M}"] = {"us": t * 1e6, "allreduce_bytes": M * 4 + M * K * 4, "input_sets": P}
+            del sets
+        out[f"world{world}"] = res
+    return out
+
+
 def run_quant_weights(bl, device, reps=5):
     import torch
     N, K = 11008, 4096
@@ -821,6 +856,7 @@ def main(argv=None):
         extra["quant_weights"] = run_quant_weights(bl, device)
         extra["decode_storage_variants"] = run_decode_storage_variants(bl, device, dec, peaks)
         extra["ste_backward"] = run_ste(bl, device, peaks)
+        extra["tp_ffn_shard"] = run_tp_ffn_shard(bl, device)
     cpu = None
     if rank == 0 and ws == 1:
         rate, n, cores = oracle_decode_rate(seconds=args.cpu_seconds)

@@ -296,7 +296,9 @@ bl_status run_gemv(int src, int out, bl_dtype a_dtype, GemvParams p, bool pdl, i
                : launch_gemv_mt<float, kSrcFloat, kOutRawI32>(tw, p, grid, smem, pdl, dev, st);
   }
   if (src == kSrcFfnRequant)
-    return launch_gemv_mt<float, kSrcFfnRequant, kOutDequant>(tw, p, grid, smem, pdl, dev, st);
+    return out == kOutDequant
+               ? launch_gemv_mt<float, kSrcFfnRequant, kOutDequant>(tw, p, grid, smem, pdl, dev, st)
+               : launch_gemv_mt<float, kSrcFfnRequant, kOutRawI32>(tw, p, grid, smem, pdl, dev, st);
   return out == kOutDequant
              ? launch_gemv_mt<float, kSrcInt8, kOutDequant>(tw, p, grid, smem, pdl, dev, st)
              : launch_gemv_mt<float, kSrcInt8, kOutRawI32>(tw, p, grid, smem, pdl, dev, st);
@@ -1248,11 +1250,15 @@ bl_status bl_ffn_tp_up(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, in
     up.gamma = gamma_up;
     up.Y = acc_up;
     up.gamma_out = gamma_x;
+    // The shard's largest r per token, raised by every CTA from its rows.
+    up.rmax_out = rmax;
+    up.rmax_atomic = 1;
     up.N = H_r;
     up.K = K;
     up.M = (int)M;
     up.eps = eps;
-    BL_TRY(run_gemv(kSrcFloat, kOutRawI32, x_dtype, up, false, dev, sms, st));
+    BL_CUDA(cudaMemsetAsync(rmax, 0, (size_t)M * 4, st));
+    return run_gemv(kSrcFloat, kOutRawI32, x_dtype, up, false, dev, sms, st);
   } else {
     uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
     int8_t* Xq = reinterpret_cast<int8_t*>(base);
@@ -1291,23 +1297,28 @@ bl_status bl_ffn_tp_down(const int32_t* acc_up, const float* gamma_x, const floa
   int dev, sms;
   BL_TRY(current_device(&dev, &sms));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (M <= kGemvMaxTokens) {
+    // One launch: the GEMV's prologue requantises the shard with γ_r.
+    GemvParams p = {};
+    p.A = acc_up;
+    p.a_scale = gamma_x;
+    p.a_gamma_up = gamma_up;
+    p.rmax_in = gamma_r;
+    p.rmax_n = 1;
+    p.W = W_down_r;
+    p.Y = acc_down;
+    p.N = K_out;
+    p.K = H_r;
+    p.M = (int)M;
+    p.eps = eps;
+    return run_gemv(kSrcFfnRequant, kOutRawI32, BL_F32, p, false, dev, sms, st);
+  }
   uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
   int8_t* Rq = reinterpret_cast<int8_t*>(base);
   int32_t* rs = reinterpret_cast<int32_t*>(base + align_up((size_t)M * H_r));
   relu2_requant_given_kernel<<<(unsigned)M, kQuantThreads, 0, st>>>(acc_up, H_r, gamma_x, gamma_up,
                                                                     gamma_r, eps, Rq, rs);
   BL_CUDA(cudaGetLastError());
-  if (M <= kGemvMaxTokens) {
-    GemvParams p = {};
-    p.A = Rq;
-    p.W = W_down_r;
-    p.Y = acc_down;
-    p.N = K_out;
-    p.K = H_r;
-    p.M = (int)M;
-    p.eps = 1.0f;
-    return run_gemv(kSrcInt8, kOutRawI32, BL_F32, p, false, dev, sms, st);
-  }
   return run_contract(Rq, W_down_r, M, H_r, K_out, nullptr, nullptr, rs, acc_down, kTcRawI32, 0, 0,
                       true, dev, sms, st);
 }

@@ -62,9 +62,12 @@ struct GemvParams {
   // rmax_out[m·gridDim.x + blockIdx.x]. kSrcFfnRequant with rmax_in: γ_r of
   // token m is the largest of rmax_in[m·rmax_n .. m·rmax_n + rmax_n), so
   // the prologue reads the accumulators once (no separate max pass).
+  // rmax_atomic: instead, every CTA raises rmax_out[m] (zeroed by the caller)
+  // to its maximum with an atomic max on the float bits (r ≥ 0).
   float* rmax_out;
   const float* rmax_in;
   int rmax_n;
+  int rmax_atomic;
   // Optional taps (all null = off): the int8 tokens [M,K], their per-token
   // scale γ and Σ of the int8 tokens, as the prologue of CTA tap_cta made them.
   int8_t* tap_q;
@@ -471,7 +474,12 @@ gemv_ternary_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
           const unsigned w = __reduce_max_sync(0xffffffffu, __float_as_uint(lm[m]));
-          if (lane == 0 && m < M) p.rmax_out[(int64_t)m * gridDim.x + blockIdx.x] = __uint_as_float(w);
+          if (lane == 0 && m < M) {
+            if (p.rmax_atomic)
+              atomicMax(reinterpret_cast<unsigned*>(p.rmax_out) + m, w);
+            else
+              p.rmax_out[(int64_t)m * gridDim.x + blockIdx.x] = __uint_as_float(w);
+          }
         }
       }
       return;
