@@ -51,6 +51,19 @@ def _cuda(t: torch.Tensor, what: str) -> torch.Tensor:
     return t
 
 
+def _shape(t: torch.Tensor, shape: tuple, what: str) -> None:
+    """The library takes plain pointers and sizes: every tensor handed to it
+    must have exactly the shape the sizes describe, or a kernel would read or
+    write past it."""
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{what} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _atleast(t: torch.Tensor, n: int, what: str) -> None:
+    if t.numel() < n:
+        raise ValueError(f"{what} must hold at least {n} elements, got {t.numel()}")
+
+
 def _ws(nbytes: int, device) -> torch.Tensor | None:
     if nbytes == 0:
         return None
@@ -85,11 +98,17 @@ def bl_quant_weights(W: torch.Tensor, eps: float = 1e-5, *, out=None, gamma=None
     N, K = W.shape
     if out is None:
         out = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    _cuda(out, "out")
+    _shape(out, (N, K // 4), "out")
     if gamma is None:
         gamma = torch.empty((1,), dtype=torch.float32, device=W.device)
+    _cuda(gamma, "gamma")
+    _atleast(gamma, 1, "gamma")
     L = load()
     if workspace is None:
         workspace = _ws(int(L.bl_quant_weights_workspace_bytes(N, K)), W.device)
+    else:
+        _cuda(workspace, "workspace")
     check(L.bl_quant_weights(W.data_ptr(), _dt(W, "W"), N, K, float(eps), out.data_ptr(),
                              gamma.data_ptr(), _ptr(workspace), _nbytes(workspace),
                              _stream(stream)), "bl_quant_weights")
@@ -131,8 +150,18 @@ def bl_linear_q(A_q, gamma_A, W_packed, gamma, *, rowsum=None, relu2=False,
         _cuda(t, n)
     M, K = A_q.shape
     N = W_packed.shape[0]
+    _shape(W_packed, (N, K // 4), "W_packed")
+    if K % 4:
+        raise ValueError("K must be a multiple of 4")
+    _atleast(gamma_A, M, "gamma_A")
+    _atleast(gamma, 1, "gamma")
+    if rowsum is not None:
+        _cuda(rowsum, "rowsum")
+        _atleast(rowsum, M, "rowsum")
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=A_q.device)
+    _cuda(out, "out")
+    _shape(out, (M, N), "out")
     L = load()
     ws = None if rowsum is not None else _ws(int(L.bl_linear_q_workspace_bytes(M, K, N)), A_q.device)
     check(L.bl_linear_q(A_q.data_ptr(), gamma_A.data_ptr(), _ptr(rowsum), M, K,
@@ -150,11 +179,17 @@ def bl_linear(A, W_packed, gamma, eps: float = 1e-5, *, relu2=False, out_dtype=t
     _cuda(gamma, "gamma")
     M, K = A.shape
     N = W_packed.shape[0]
+    _shape(W_packed, (N, K // 4), "W_packed")
+    _atleast(gamma, 1, "gamma")
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    _cuda(out, "out")
+    _shape(out, (M, N), "out")
     L = load()
     if workspace is None:
         workspace = _ws(int(L.bl_linear_workspace_bytes(M, K, N)), A.device)
+    else:
+        _cuda(workspace, "workspace")
     check(L.bl_linear_ex(A.data_ptr(), _dt(A, "A"), M, K, W_packed.data_ptr(), gamma.data_ptr(),
                          N, float(eps), int(bool(relu2)), out.data_ptr(), _dt(out, "out"),
                          _ptr(workspace), _nbytes(workspace), BL_FLAG_PDL if pdl else 0,
@@ -173,8 +208,12 @@ def bl_linear_noalloc(A, W_packed, gamma, eps: float = 1e-5, *, relu2=False,
     _cuda(gamma, "gamma")
     M, K = A.shape
     N = W_packed.shape[0]
+    _shape(W_packed, (N, K // 4), "W_packed")
+    _atleast(gamma, 1, "gamma")
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    _cuda(out, "out")
+    _shape(out, (M, N), "out")
     check(load().bl_linear_noalloc(A.data_ptr(), _dt(A, "A"), M, K, W_packed.data_ptr(),
                                    gamma.data_ptr(), N, float(eps), int(bool(relu2)),
                                    out.data_ptr(), _dt(out, "out"), _stream(stream)),
@@ -190,13 +229,19 @@ def bl_ffn_relu2(X, W_up, gamma_up, W_down, gamma_down, eps: float = 1e-5, *,
         _cuda(t, n)
     M, K = X.shape
     H = W_up.shape[0]
-    if W_up.shape[1] * 4 != K or W_down.shape[0] != K or W_down.shape[1] * 4 != H:
-        raise ValueError("W_up must be [H, K/4] and W_down [K, H/4]")
+    _shape(W_up, (H, K // 4), "W_up")
+    _shape(W_down, (K, H // 4), "W_down")
+    _atleast(gamma_up, 1, "gamma_up")
+    _atleast(gamma_down, 1, "gamma_down")
     if out is None:
         out = torch.empty((M, K), dtype=out_dtype, device=X.device)
+    _cuda(out, "out")
+    _shape(out, (M, K), "out")
     L = load()
     if workspace is None:
         workspace = _ws(int(L.bl_ffn_workspace_bytes(M, K, H)), X.device)
+    else:
+        _cuda(workspace, "workspace")
     check(L.bl_ffn_relu2_ex(X.data_ptr(), _dt(X, "X"), M, K, H, W_up.data_ptr(), gamma_up.data_ptr(),
                             W_down.data_ptr(), gamma_down.data_ptr(), float(eps), out.data_ptr(),
                             _dt(out, "out"), _ptr(workspace), _nbytes(workspace),
@@ -228,6 +273,8 @@ def bl_linear_taps(A, W_packed, gamma, eps: float = 1e-5, *, relu2=False,
     _cuda(gamma, "gamma")
     M, K = A.shape
     N = W_packed.shape[0]
+    _shape(W_packed, (N, K // 4), "W_packed")
+    _atleast(gamma, 1, "gamma")
     out = torch.empty((M, N), dtype=out_dtype, device=A.device)
     L = load()
     ws = _ws(int(L.bl_linear_workspace_bytes(M, K, N)), A.device)
@@ -249,6 +296,8 @@ def bl_ffn_relu2_taps(X, W_up, gamma_up, W_down, gamma_down, eps: float = 1e-5, 
         _cuda(t, n)
     M, K = X.shape
     H = W_up.shape[0]
+    _shape(W_up, (H, K // 4), "W_up")
+    _shape(W_down, (K, H // 4), "W_down")
     out = torch.empty((M, K), dtype=out_dtype, device=X.device)
     L = load()
     ws = _ws(int(L.bl_ffn_workspace_bytes(M, K, H)), X.device)
@@ -317,10 +366,13 @@ def bl_pack_radix3(W_packed, K: int, *, out=None, stream=None):
     """2-bit packed [N, K/4] → radix-3 storage [N, row_bytes] (5 weights/byte)."""
     _cuda(W_packed, "W_packed")
     N = W_packed.shape[0]
+    _shape(W_packed, (N, K // 4), "W_packed")
     L = load()
     rb = int(L.bl_radix3_row_bytes(K))
     if out is None:
         out = torch.empty((N, rb), dtype=torch.uint8, device=W_packed.device)
+    _cuda(out, "out")
+    _shape(out, (N, rb), "out")
     check(L.bl_pack_radix3(W_packed.data_ptr(), N, K, out.data_ptr(), _stream(stream)),
           "bl_pack_radix3")
     return out
@@ -334,8 +386,14 @@ def bl_linear_radix3(A, W_r3, gamma, eps: float = 1e-5, *, relu2=False, out_dtyp
     _cuda(gamma, "gamma")
     M, K = A.shape
     N = W_r3.shape[0]
+    _shape(W_r3, (N, int(load().bl_radix3_row_bytes(K))), "W_r3")
+    _atleast(gamma, 1, "gamma")
     if out is None:
         out = torch.empty((M, N), dtype=torch.int32 if raw else out_dtype, device=A.device)
+    _cuda(out, "out")
+    _shape(out, (M, N), "out")
+    if raw and out.dtype != torch.int32:
+        raise TypeError("out must be int32 when raw=True")
     flags = (BL_FLAG_PDL if pdl else 0) | (BL_FLAG_RAW_I32 if raw else 0)
     ydt = BL_F32 if raw else _dt(out, "out")
     check(load().bl_linear_radix3(A.data_ptr(), _dt(A, "A"), M, K, W_r3.data_ptr(), gamma.data_ptr(),
@@ -350,6 +408,8 @@ def bl_pack_lut_index(W_packed, *, out=None, stream=None):
     N, Kq = W_packed.shape
     if out is None:
         out = torch.empty((N, Kq), dtype=torch.uint8, device=W_packed.device)
+    _cuda(out, "out")
+    _shape(out, (N, Kq), "out")
     check(load().bl_pack_lut_index(W_packed.data_ptr(), N, 4 * Kq, out.data_ptr(), _stream(stream)),
           "bl_pack_lut_index")
     return out
@@ -363,8 +423,14 @@ def bl_linear_lut(A, W_idx, gamma, eps: float = 1e-5, *, out_dtype=torch.bfloat1
     _cuda(gamma, "gamma")
     M, K = A.shape
     N = W_idx.shape[0]
+    _shape(W_idx, (N, K // 4), "W_idx")
+    _atleast(gamma, 1, "gamma")
     if out is None:
         out = torch.empty((M, N), dtype=torch.int32 if raw else out_dtype, device=A.device)
+    _cuda(out, "out")
+    _shape(out, (M, N), "out")
+    if raw and out.dtype != torch.int32:
+        raise TypeError("out must be int32 when raw=True")
     flags = (BL_FLAG_PDL if pdl else 0) | (BL_FLAG_RAW_I32 if raw else 0)
     check(load().bl_linear_lut(A.data_ptr(), _dt(A, "A"), M, K, W_idx.data_ptr(), gamma.data_ptr(),
                                N, float(eps), out.data_ptr(), BL_F32 if raw else _dt(out, "out"),

@@ -136,3 +136,19 @@ def test_lut_host_checks(lib):
     assert lib.bl_linear_lut(p, 1, 2, 512, p, p, 64, 1e-5, p, 1, 0, None) == BL_ERR_SHAPE
     assert lib.bl_linear_lut(p, 1, 1, 512, p, p, 64, 1e-5, p, 1, 8, None) == BL_ERR_INVALID_ARG
     assert lib.bl_pack_lut_index(p, 8, 100, p, None) == BL_ERR_SHAPE
+
+
+def test_binding_shape_checks():
+    """The library takes plain pointers and sizes, so the binding refuses
+    tensors whose shapes do not match the sizes it passes (a packed matrix
+    with a different K would be read past its end)."""
+    import torch
+    from ternary_weight_linear_absmax_b200 import _atleast, _shape
+    _shape(torch.empty(8, 16), (8, 16), "W_packed")
+    with pytest.raises(ValueError, match="W_packed must have shape"):
+        _shape(torch.empty(8, 12), (8, 16), "W_packed")
+    with pytest.raises(ValueError, match="out must have shape"):
+        _shape(torch.empty(4, 8), (8, 4), "out")
+    _atleast(torch.empty(3), 3, "gamma_A")
+    with pytest.raises(ValueError, match="gamma_A must hold at least 4"):
+        _atleast(torch.empty(3), 4, "gamma_A")

@@ -173,6 +173,7 @@ ZG_CASES = [
     (256, 512, 384), (300, 384, 512), (520, 128, 136),
     (384, 128, 7680), (300, 256, 9000),  # 192-token tiles (one round instead of two of 128)
     (512, 128, 11008),  # 192-token tiles, two CTAs per SM
+    (100, 192, 300), (520, 64, 136),  # K not a multiple of the 128-wide K block
 ]
 
 
