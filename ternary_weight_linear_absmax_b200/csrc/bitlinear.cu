@@ -415,7 +415,7 @@ TcTile tc_pick_tile(int64_t M, int64_t N, int sms) {
 bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,
                  const float* gamma, const float* gammaA, const int32_t* rowsum, void* Y,
                  int out, int relu2, int y_bf16, void* split_ws, size_t split_ws_bytes, int dev,
-                 int sms, cudaStream_t st) {
+                 int sms, cudaStream_t st, bool w_early = false) {
   if (M > 0x7FFFFFFF || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
   const int KBall = (int)((K + kTcBK - 1) / kTcBK);
   int sp = tc_splits(M, N, K, sms);
@@ -466,6 +466,7 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
   p.y_bf16 = y_bf16;
   p.kb_per_split = kbs;
   p.split_rows = sp > 1 ? tc_split_rows(M) : 0;
+  p.w_early = w_early ? 1 : 0;
   BL_TRY(outk == kTcDequant ? launch_tc_bn<kTcDequant>(tile, ta, tw, ty, p, sp, dev, st)
                             : launch_tc_bn<kTcRawI32>(tile, ta, tw, ty, p, sp, dev, st));
   if (sp == 1) return BL_OK;
@@ -620,7 +621,7 @@ bl_status run_contract(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K
     return run_skinny(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out == kTcRawI32 ? 1 : 0, relu2,
                       y_bf16, pdl, dev, sms, st);
   return run_tc(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out, relu2, y_bf16, split_ws,
-                split_ws_bytes, dev, sms, st);
+                split_ws_bytes, dev, sms, st, pdl);
 }
 
 // pdl: launch with programmatic dependent launch (the kernel waits for the

@@ -58,6 +58,8 @@ struct TcParams {
                      // (stored whole by the tensor stores) stay in z's own padding.
                      // Only split 0 subtracts the row sums.
   int64_t split_rows;  // Mp (0 when unsplit)
+  int w_early;         // 1: the kernel before this one does not write the packed weights, so
+                       //    the first weight stages are requested before the dependency wait
 };
 
 // DUAL: two CTAs per SM (BN 128 or 192). Each CTA then fits in half of the
@@ -316,15 +318,25 @@ tc_ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
   const uint32_t tmem = *s_tmem;
   // Launched with programmatic dependent launch: the set-up above overlaps
   // the previous kernel's tail; global memory is touched only after it has
-  // completed. The next kernel may start its own set-up from here on.
+  // completed, except the first weight stages when the caller says the
+  // weights are not written by that kernel (w_early). The next kernel may
+  // start its own set-up from here on.
   pdl_launch_dependents();
+  // Weight stages requested before the dependency wait (w_early; warp 0).
+  int w_pre = 0;
+  if (warp == 0 && p.w_early) {
+    w_pre = min((KB + 3) / 4, WS);
+    for (int ws = 0; ws < w_pre; ++ws)
+      tma_load_1x2d_warp(&wfull[ws], C::kWStage, s_w + ws * C::kWStage, &tm_w,
+                         (kb_lo + 4 * ws) * 32, (int32_t)n0);
+  }
   pdl_wait_prior_grid();
 
   if (warp == 0) {
     // ---------------- TMA producer (whole warp, one elected lane issues) ---
-    int kb = 0, wissued = 0;
+    int kb = 0, wissued = w_pre;
     for (; kb < KB; ++kb) {
-      if ((kb & 3) == 0) {  // a new weight stage covers K blocks kb .. kb+3
+      if ((kb & 3) == 0 && (kb >> 2) >= w_pre) {  // a new weight stage covers K blocks kb .. kb+3
         const int ws = kb >> 2, v = ws % WS;
         bool ok = ws < WS || wait_or_abort(&wempty[v], ((ws / WS) + 1) & 1, s_abort);
         if (!__all_sync(0xffffffffu, ok)) break;
