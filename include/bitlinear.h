@@ -169,6 +169,14 @@ bl_status bl_linear_q(const int8_t* A_q, const float* gamma_A,
                       const uint8_t* W_packed, const float* gamma, int64_t N,
                       int relu2, void* Y, bl_dtype y_dtype, void* workspace,
                       size_t ws_bytes, bl_stream_t stream);
+/* bl_linear_q with `flags`: BL_FLAG_PDL as for bl_linear_ex (the kernel
+ * before this call on `stream` does not write W_packed or gamma, so the
+ * contraction may stream its weights before waiting for that kernel). */
+bl_status bl_linear_q_ex(const int8_t* A_q, const float* gamma_A,
+                         const int32_t* rowsum, int64_t M, int64_t K,
+                         const uint8_t* W_packed, const float* gamma, int64_t N,
+                         int relu2, void* Y, bl_dtype y_dtype, void* workspace,
+                         size_t ws_bytes, unsigned flags, bl_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * bl_linear — BitLinear forward from float activations:

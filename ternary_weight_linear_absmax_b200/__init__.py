@@ -144,8 +144,9 @@ def bl_zero_gemm(A_q: torch.Tensor, W_packed: torch.Tensor, *, stream=None):
 
 
 def bl_linear_q(A_q, gamma_A, W_packed, gamma, *, rowsum=None, relu2=False,
-                out_dtype=torch.bfloat16, out=None, stream=None):
-    """Y = (A_q·W_qᵀ)·(γ_A·γ)/127 (ReLU² optional) from int8 tokens."""
+                out_dtype=torch.bfloat16, out=None, pdl=False, stream=None):
+    """Y = (A_q·W_qᵀ)·(γ_A·γ)/127 (ReLU² optional) from int8 tokens.
+    pdl: BL_FLAG_PDL (the kernel before this call does not write W_packed)."""
     for t, n in ((A_q, "A_q"), (gamma_A, "gamma_A"), (W_packed, "W_packed"), (gamma, "gamma")):
         _cuda(t, n)
     M, K = A_q.shape
@@ -164,10 +165,10 @@ def bl_linear_q(A_q, gamma_A, W_packed, gamma, *, rowsum=None, relu2=False,
     _shape(out, (M, N), "out")
     L = load()
     ws = None if rowsum is not None else _ws(int(L.bl_linear_q_workspace_bytes(M, K, N)), A_q.device)
-    check(L.bl_linear_q(A_q.data_ptr(), gamma_A.data_ptr(), _ptr(rowsum), M, K,
-                        W_packed.data_ptr(), gamma.data_ptr(), N, int(bool(relu2)),
-                        out.data_ptr(), _dt(out, "out"), _ptr(ws), _nbytes(ws),
-                        _stream(stream)), "bl_linear_q")
+    check(L.bl_linear_q_ex(A_q.data_ptr(), gamma_A.data_ptr(), _ptr(rowsum), M, K,
+                           W_packed.data_ptr(), gamma.data_ptr(), N, int(bool(relu2)),
+                           out.data_ptr(), _dt(out, "out"), _ptr(ws), _nbytes(ws),
+                           BL_FLAG_PDL if pdl else 0, _stream(stream)), "bl_linear_q")
     return out
 
 

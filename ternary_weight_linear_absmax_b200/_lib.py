@@ -45,6 +45,8 @@ SIGNATURES = {
     "bl_linear_q_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_linear_q": (_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _int, _vp, _int, _vp,
                            _sz, _vp]),
+    "bl_linear_q_ex": (_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _int, _vp, _int, _vp,
+                              _sz, _uint, _vp]),
     "bl_linear_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_linear": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _i64, _f32, _int, _vp, _int, _vp,
                          _sz, _vp]),

@@ -948,6 +948,16 @@ bl_status bl_linear_q(const int8_t* A_q, const float* gamma_A, const int32_t* ro
                       int64_t K, const uint8_t* W_packed, const float* gamma, int64_t N, int relu2,
                       void* Y, bl_dtype y_dtype, void* workspace, size_t ws_bytes,
                       bl_stream_t stream) {
+  return bl_linear_q_ex(A_q, gamma_A, rowsum, M, K, W_packed, gamma, N, relu2, Y, y_dtype,
+                        workspace, ws_bytes, 0u, stream);
+}
+
+bl_status bl_linear_q_ex(const int8_t* A_q, const float* gamma_A, const int32_t* rowsum,
+                         int64_t M, int64_t K, const uint8_t* W_packed, const float* gamma,
+                         int64_t N, int relu2, void* Y, bl_dtype y_dtype, void* workspace,
+                         size_t ws_bytes, unsigned flags, bl_stream_t stream) {
+  if ((flags & ~(unsigned)BL_FLAG_PDL) != 0) return BL_ERR_INVALID_ARG;
+  const bool pdl = (flags & BL_FLAG_PDL) != 0;
   BL_TRY(check_dtype(y_dtype));
   BL_TRY(check_k(K));
   BL_TRY(check_rows(M));
@@ -981,7 +991,7 @@ bl_status bl_linear_q(const int8_t* A_q, const float* gamma_A, const int32_t* ro
     p.eps = 1.0f;
     p.relu2 = relu2 ? 1 : 0;
     p.y_bf16 = y_dtype == BL_BF16;
-    return run_gemv(kSrcInt8, kOutDequant, BL_F32, p, false, dev, sms, st);
+    return run_gemv(kSrcInt8, kOutDequant, BL_F32, p, pdl, dev, sms, st);
   }
   const int32_t* rs = rowsum;
   if (rs == nullptr) {
@@ -991,12 +1001,12 @@ bl_status bl_linear_q(const int8_t* A_q, const float* gamma_A, const int32_t* ro
     rs = w;
   }
   // After this call's row-sum kernel the weights may stream early; without
-  // it the preceding kernel is the caller's, so no early start.
+  // it the preceding kernel is the caller's: early only with BL_FLAG_PDL.
   const size_t rs_part = align_up((size_t)M * 4);
   void* split_ws = (workspace != nullptr && ws_bytes > rs_part)
                        ? reinterpret_cast<uint8_t*>(workspace) + rs_part : nullptr;
   return run_contract(A_q, W_packed, M, K, N, gamma, gamma_A, rs, Y, kTcDequant, relu2 ? 1 : 0,
-                      y_dtype == BL_BF16, rowsum == nullptr, dev, sms, st, split_ws,
+                      y_dtype == BL_BF16, pdl || rowsum == nullptr, dev, sms, st, split_ws,
                       split_ws ? ws_bytes - rs_part : 0);
 }
 
