@@ -187,6 +187,29 @@ def test_zero_gemm_exact(bl, M, K, N):
     np.testing.assert_array_equal(acc, oracle.zero_gemm(Aq, codes))
 
 
+def _random_shapes(count, seed):
+    """Seeded shapes over every contraction path: GEMV (≤ 4 tokens), the
+    warp-level kernel (5-64), tensor-core tiles of 128/192/256 tokens, one or
+    two CTAs per SM, K splits, ragged N, K not a multiple of the 128-wide
+    block."""
+    u = si.uniform(seed, 3 * count).reshape(count, 3)
+    shapes = []
+    for a, b, c in u:
+        M = int(1 + a ** 2 * 700)            # biased towards small M
+        K = 64 * int(1 + b * 40)             # 64 .. 2560
+        N = int(1 + c ** 1.5 * 12000)
+        shapes.append((M, K, N))
+    return shapes
+
+
+@pytest.mark.parametrize("M,K,N", _random_shapes(24, seed=2024))
+def test_zero_gemm_random_shapes(bl, M, K, N):
+    Aq = random_int8(M, K, seed=M * 31 + K)
+    codes = random_codes(N, K, seed=N * 13 + K)
+    acc = bl.bl_zero_gemm(to_dev(Aq), to_dev(oracle.pack_ternary(codes))).cpu().numpy()
+    np.testing.assert_array_equal(acc, oracle.zero_gemm(Aq, codes))
+
+
 def test_zero_gemm_extremes(bl):
     """Worst-case magnitudes: all +127 / -127 activations against all-±1 rows."""
     for M in (1, 40):
