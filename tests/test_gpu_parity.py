@@ -366,6 +366,35 @@ def test_ffn_small(bl, M):
     _ffn_case(bl, M, 256, 640, seed=M)
 
 
+def _random_linear_cases(count, seed):
+    u = si.uniform(seed, 5 * count).reshape(count, 5)
+    cases = []
+    for a, b, c, d, e in u:
+        M = int(1 + a ** 3 * 500)
+        K = 64 * int(1 + b * 24)
+        N = int(8 + c ** 1.5 * 6000)
+        out = torch.float32 if d < 0.5 else torch.bfloat16
+        cases.append((M, K, N, out, bool(e < 0.3)))
+    return cases
+
+
+@pytest.mark.parametrize("M,K,N,out,relu2", _random_linear_cases(16, seed=77))
+def test_linear_random_shapes(bl, M, K, N, out, relu2):
+    """Seeded shapes through every dequantising epilogue (GEMV, warp-level,
+    tensor-core tiles, K splits), fp32 or bf16 out, ReLU² on some."""
+    _linear_case(bl, M, K, N, "bf16", "bf16", True, out, relu2=relu2, seed=M + N)
+
+
+def _random_ffn_cases(count, seed):
+    u = si.uniform(seed, 3 * count).reshape(count, 3)
+    return [(int(1 + a ** 2 * 400), 64 * int(2 + b * 14), 64 * int(2 + c * 30)) for a, b, c in u]
+
+
+@pytest.mark.parametrize("M,K,H", _random_ffn_cases(8, seed=91))
+def test_ffn_random_shapes(bl, M, K, H):
+    _ffn_case(bl, M, K, H, seed=M + H)
+
+
 @pytest.mark.parametrize("M", [1, 64, 512])
 def test_ffn_full_sampled(bl, M):
     """FFN block 4096 → 11008 → 4096 at M ∈ {1, 64, 512}; sampled tokens."""
