@@ -739,11 +739,11 @@ bl_status make_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint6
   return r == CUDA_SUCCESS ? BL_OK : BL_ERR_CUDA;
 }
 
-template <int BN, bool MASK>
+template <int BN, bool MASK, bool DUAL = false>
 bl_status launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const GmParams& p, int dev,
                         cudaStream_t st) {
-  auto* k = bf16_gemm_kernel<BN, MASK>;
-  constexpr size_t smem = GmConfig<BN>::kSmem;
+  auto* k = bf16_gemm_kernel<BN, MASK, DUAL>;
+  constexpr size_t smem = GmConfig<BN, DUAL>::kSmem;
   BL_TRY(ensure_smem(k, dev, smem));
   const dim3 grid((unsigned)((p.rows + kGmBM - 1) / kGmBM), (unsigned)((p.cols + BN - 1) / BN));
   k<<<grid, kGmThreads, smem, st>>>(ta, tb, p);
@@ -761,6 +761,15 @@ bl_status run_bf16_gemm(const void* A, int64_t lda, const void* B, int64_t ldb, 
   BL_TRY(make_map_bf16(&ta, A, (uint64_t)p.rows, (uint64_t)p.kdim, (uint64_t)lda, kGmBM));
   BL_TRY(make_map_bf16(&tb, B, (uint64_t)p.cols, (uint64_t)p.kdim, (uint64_t)ldb, wide ? 256 : 128));
   const bool mask = p.mask_w != nullptr;
+  // More tiles than SMs: two CTAs per SM (two stages each), so one CTA's
+  // epilogue overlaps the other's MMAs (2048 x 4096 x 4096: dA 69.4 -> 67.9 us,
+  // dW 98.6 -> 96.7 us; 128-wide tiles two per SM were slower).
+  int dev_sms = 0;
+  BL_CUDA(cudaDeviceGetAttribute(&dev_sms, cudaDevAttrMultiProcessorCount, dev));
+  const int64_t tiles = ((p.rows + kGmBM - 1) / kGmBM) * ((p.cols + 255) / 256);
+  if (wide && tiles > dev_sms)
+    return mask ? launch_gemm_t<256, true, true>(ta, tb, p, dev, st)
+                : launch_gemm_t<256, false, true>(ta, tb, p, dev, st);
   if (wide)
     return mask ? launch_gemm_t<256, true>(ta, tb, p, dev, st) : launch_gemm_t<256, false>(ta, tb, p, dev, st);
   return mask ? launch_gemm_t<128, true>(ta, tb, p, dev, st) : launch_gemm_t<128, false>(ta, tb, p, dev, st);

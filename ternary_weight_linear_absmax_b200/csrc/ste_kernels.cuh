@@ -28,11 +28,13 @@ constexpr int kGmThreads = 192;
 constexpr int kGmBM = 128;
 constexpr int kGmBK = 64;  // bf16 per stage row: one 128-byte swizzle row
 
-template <int BN>
+// DUAL: two CTAs per SM (each at most half of the shared memory, BN TMEM
+// columns), so one CTA's epilogue overlaps the other's MMAs.
+template <int BN, bool DUAL = false>
 struct GmConfig {
   static constexpr int kStageA = kGmBM * 128;
   static constexpr int kStageB = BN * 128;
-  static constexpr int kStages = BN >= 256 ? 4 : 6;
+  static constexpr int kStages = DUAL ? (BN >= 256 ? 2 : 3) : (BN >= 256 ? 4 : 6);
   static constexpr int kRing = kStages * (kStageA + kStageB);
   static constexpr int kSmem = 1024 + kRing + (2 * kStages + 2) * 8 + 16;
   static constexpr int kTmemCols = BN;
@@ -88,11 +90,11 @@ __device__ __forceinline__ void tma_load_2x2d_warp(uint64_t* bar, uint32_t tx, v
       : "memory");
 }
 
-template <int BN, bool MASK>
-__global__ void __launch_bounds__(kGmThreads, 1)
+template <int BN, bool MASK, bool DUAL = false>
+__global__ void __launch_bounds__(kGmThreads, DUAL ? 2 : 1)
 bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                  const GmParams p) {
-  using C = GmConfig<BN>;
+  using C = GmConfig<BN, DUAL>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(

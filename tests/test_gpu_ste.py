@@ -46,7 +46,9 @@ def _problem(M, N, K, seed, dy_dtype):
 
 
 CASES = [(4, 256, 512, "f32"), (130, 200, 320, "bf16"), (256, 1024, 768, "bf16"),
-         (37, 512, 4096, "f32"), (512, 2048, 1024, "bf16")]
+         (37, 512, 4096, "f32"), (512, 2048, 1024, "bf16"),
+         # more output tiles than SMs (two CTAs per SM): dW of (64, 4096, 1536), dA of (2560, 128, 2048)
+         (64, 4096, 1536, "bf16"), (2560, 128, 2048, "bf16")]
 
 
 @pytest.mark.parametrize("M,N,K,dt", CASES)
