@@ -880,7 +880,9 @@ def main(argv=None):
 
     dec = run_decode(bl, device, args.steps, args.warmup, peaks, ws)
     extra = {}
-    if not args.no_extra and rank == 0:
+    # The secondary workloads run in single-GPU runs only: in a multi-GPU run
+    # the other ranks would sit idle (holding their GPUs) while rank 0 works.
+    if not args.no_extra and rank == 0 and ws == 1:
         extra["decode_single_call_us"] = dec["single_call_us_median"]
         extra["decode_pool"] = dec["pool"]
         extra["small_batch"] = run_small_batch(bl, device, peaks)
