@@ -208,6 +208,23 @@ FfnWs ffn_ws(int64_t M, int64_t K, int64_t H) {
   return w;
 }
 
+// A kernel launched with programmatic dependent launch (it must wait for the
+// previous grid before it reads what that grid may write).
+template <typename... KArgs, typename... Args>
+bl_status launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  BL_CUDA(cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...));
+  return BL_OK;
+}
+
 // --------------------------------------------------------------------------
 // GEMV launches.
 template <int MT, typename TA, int SRC, int OUT>
@@ -471,12 +488,12 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
                             : launch_tc_bn<kTcRawI32>(tile, ta, tw, ty, p, sp, dev, st));
   if (sp == 1) return BL_OK;
   BL_TRY(ensure_smem(splitk_reduce_kernel, dev, 0));
-  const dim3 rgrid((unsigned)((N + 1023) / 1024), (unsigned)M);
-  splitk_reduce_kernel<<<rgrid, 256, 0, st>>>(
-      reinterpret_cast<const int32_t*>(Yk), sp, tc_split_rows(M) * N, M, N,
-      out == kTcRawI32 ? 1 : 0, gamma, gammaA, relu2, Y, y_bf16,
-      (N % 4 == 0 && (reinterpret_cast<uintptr_t>(Y) & 15) == 0) ? 1 : 0);
-  BL_CUDA(cudaGetLastError());
+  // With programmatic dependent launch: the reduce waits for the partials
+  // (the kernel's first step) and its launch overlaps the contraction's tail.
+  BL_TRY(launch_pdl(splitk_reduce_kernel, dim3((unsigned)((N + 1023) / 1024), (unsigned)M), dim3(256),
+                    st, reinterpret_cast<const int32_t*>(Yk), sp, tc_split_rows(M) * N, M, N,
+                    out == kTcRawI32 ? 1 : 0, gamma, gammaA, relu2, Y, y_bf16,
+                    (N % 4 == 0 && (reinterpret_cast<uintptr_t>(Y) & 15) == 0) ? 1 : 0));
   return BL_OK;
 }
 
@@ -1189,9 +1206,8 @@ static bl_status ffn_impl(const void* X, bl_dtype x_dtype, int64_t M, int64_t K,
   BL_TRY(run_contract(Xq, W_up, M, K, H, gamma_up, gX, rsX, acc_up, kTcRawI32, 0, 0, true, dev,
                       sms, st, split_ws, split_bytes));
   BL_TRY(ensure_smem(relu2_requant_kernel, dev, 0));
-  relu2_requant_kernel<<<(unsigned)M, kQuantThreads, 0, st>>>(acc_up, H, gX, gamma_up, eps, Rq, gR,
-                                                              rsR);
-  BL_CUDA(cudaGetLastError());
+  BL_TRY(launch_pdl(relu2_requant_kernel, dim3((unsigned)M), dim3(kQuantThreads), st, acc_up, H, gX,
+                    gamma_up, eps, Rq, gR, rsR));
   BL_TRY(run_contract(Rq, W_down, M, H, K, gamma_down, gR, rsR, Y, kTcDequant, 0,
                       y_dtype == BL_BF16, true, dev, sms, st, split_ws, split_bytes));
   if (taps) {

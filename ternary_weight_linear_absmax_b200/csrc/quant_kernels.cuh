@@ -300,6 +300,7 @@ relu2_requant_kernel(const int32_t* __restrict__ acc, int64_t H, const float* __
                      const float* __restrict__ g_up, float eps, int8_t* __restrict__ Rq,
                      float* __restrict__ gammaR, int32_t* __restrict__ rowsum) {
   pdl_launch_dependents();
+  pdl_wait_prior_grid();  // no-op unless launched with programmatic dependent launch
   const int64_t m = blockIdx.x;
   const int4* a4 = reinterpret_cast<const int4*>(acc + m * H);
   const int64_t nvec = H / 4;
@@ -434,6 +435,8 @@ splitk_reduce_kernel(const int32_t* __restrict__ part, int splits, int64_t strid
                      int64_t N, int raw, const float* __restrict__ gamma,
                      const float* __restrict__ gammaA, int relu2, void* Y, int y_bf16,
                      int vec) {
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();  // no-op unless launched with programmatic dependent launch
   const int64_t m = blockIdx.y;
   const float sc = raw ? 0.0f : __fdiv_rn(__fmul_rn(__ldg(gammaA + m), __ldg(gamma)), 127.0f);
   auto finish = [sc, relu2](int v) -> float { return dequant_value(v, sc, relu2); };
