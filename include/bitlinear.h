@@ -17,7 +17,7 @@
  *    pointers after the call returns. Scratch memory ("workspace") is passed
  *    in by the caller; its size comes from the matching *_workspace_bytes().
  *    For bl_zero_gemm, bl_linear_q, bl_linear and bl_ffn_relu2 part of that
- *    size is optional: with more than 64 tokens and too few output tiles to
+ *    size is optional: with more than 32 tokens and too few output tiles to
  *    fill half of the SMs, the tensor-core contraction splits K into up to 4
  *    ranges whose INT32 partials go there before one summing pass; a smaller
  *    workspace (down to the quantised tokens and row sums) gives the same
@@ -184,7 +184,7 @@ bl_status bl_linear_q_ex(const int8_t* A_q, const float* gamma_A,
  * call. For M ≤ bl_gemv_max_tokens() it is a single fused GEMV launch (the
  * activation quantiser runs in the kernel prologue; no workspace needed);
  * above that, an activation-quantiser launch and one contraction launch:
- * warp-level int8 MMAs over all SMs for M ≤ 64, tensor-core (tcgen05) tiles
+ * warp-level int8 MMAs over all SMs for M ≤ 32, tensor-core (tcgen05) tiles
  * above. The contraction launches with programmatic dependent launch; it
  * reads no memory written by the kernel before it until that kernel has
  * completed, except that after this call's own quantiser it streams W_packed

@@ -346,7 +346,7 @@ bl_status launch_tc_t(const CUtensorMap& ta, const CUtensorMap& tw, const CUtens
 }
 
 // Token tile of a launch: width 128, 192 or 256 (the tensor-core path only
-// sees M > 64; fewer tokens take the skinny kernel), one or two CTAs per SM.
+// sees M > 32), one or two CTAs per SM.
 struct TcTile {
   int bn;
   bool dual;
@@ -393,7 +393,7 @@ int64_t tc_split_rows(int64_t M) {
 }
 
 size_t tc_split_ws_bytes(int64_t M, int64_t N, int64_t K) {
-  if (M <= kSkMaxTokens) return 0;
+  if (M <= kSkPreferTokens) return 0;
   const int sp = tc_splits(M, N, K, kSplitWsSms);
   return sp > 1 ? align_up((size_t)sp * tc_split_rows(M) * N * 4) : 0;
 }
@@ -428,6 +428,17 @@ TcTile tc_pick_tile(int64_t M, int64_t N, int sms) {
   return TcTile{best, false};
 }
 
+// K ranges a launch gets: the split its tile count asks for, capped by the
+// one workspaces are sized for, and 1 without room for the partials.
+int tc_launch_splits(int64_t M, int64_t N, int64_t K, int sms, const void* split_ws,
+                     size_t split_ws_bytes) {
+  int sp = tc_splits(M, N, K, sms);
+  const int sp_ws = tc_splits(M, N, K, kSplitWsSms);
+  if (sp > sp_ws) sp = sp_ws;
+  if (sp > 1 && (split_ws == nullptr || split_ws_bytes < tc_split_ws_bytes(M, N, K))) sp = 1;
+  return sp;
+}
+
 // acc/Y[M,N] = epilogue(A_q[M,K] · W_q[N,K]ᵀ − rowsum).
 bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,
                  const float* gamma, const float* gammaA, const int32_t* rowsum, void* Y,
@@ -435,10 +446,7 @@ bl_status run_tc(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int6
                  int sms, cudaStream_t st, bool w_early = false) {
   if (M > 0x7FFFFFFF || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
   const int KBall = (int)((K + kTcBK - 1) / kTcBK);
-  int sp = tc_splits(M, N, K, sms);
-  const int sp_ws = tc_splits(M, N, K, kSplitWsSms);
-  if (sp > sp_ws) sp = sp_ws;
-  if (sp > 1 && (split_ws == nullptr || split_ws_bytes < tc_split_ws_bytes(M, N, K))) sp = 1;
+  int sp = tc_launch_splits(M, N, K, sms, split_ws, split_ws_bytes);
   const TcTile tile = sp > 1 ? TcTile{tc_split_bn(M), false} : tc_pick_tile(M, N, sms);
   const int bn = tile.bn;
   const int kbs = sp > 1 ? ((KBall + sp - 1) / sp + 3) / 4 * 4 : KBall;
@@ -626,17 +634,29 @@ bl_status run_skinny(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, 
   return launch_skinny_split<4>(split, tw, ta, p, grid, smem, pdl, dev, st);
 }
 
-// Contraction of pre-quantised tokens: the skinny kernel up to 64 tokens,
-// tensor-core tiles above. out: kTcDequant or kTcRawI32.
-// split_ws: optional scratch (tc2_ws_bytes) that lets under-filled tensor-core
-// launches split K.
+// Contraction of pre-quantised tokens: the skinny kernel up to 32 tokens,
+// tensor-core tiles above 64. From 33 to 64 tokens the skinny kernel needs
+// four 16-token m-tiles and costs what 64 tokens cost, while a 128-token tile
+// costs about the same for any M ≤ 128, so the tiles take the call when they
+// (times their K ranges) fill at least half of the SMs; otherwise the
+// skinny kernel's spread over every SM wins. Measured in chains at 48-64
+// tokens: 4096 -> 11008 (86 tiles) 15.2 us on tiles against 16.1 skinny;
+// 11008 -> 4096 (32 tiles × 4 K ranges) 16.3-17.3 against 17.8-17.9; a
+// 5504 -> 4096 shard without split workspace (32 tiles) ran slower on tiles.
+// split_ws: optional scratch (tc_split_ws_bytes) that lets under-filled
+// tensor-core launches split K.
 bl_status run_contract(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,
                        const float* gamma, const float* gammaA, const int32_t* rowsum, void* Y,
                        int out, int relu2, int y_bf16, bool pdl, int dev, int sms,
                        cudaStream_t st, void* split_ws = nullptr, size_t split_ws_bytes = 0) {
-  if (M <= kSkMaxTokens)
-    return run_skinny(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out == kTcRawI32 ? 1 : 0, relu2,
-                      y_bf16, pdl, dev, sms, st);
+  if (M <= kSkMaxTokens) {
+    const bool tiles =
+        M > kSkPreferTokens &&
+        2 * ((N + 127) / 128) * tc_launch_splits(M, N, K, sms, split_ws, split_ws_bytes) >= sms;
+    if (!tiles)
+      return run_skinny(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out == kTcRawI32 ? 1 : 0,
+                        relu2, y_bf16, pdl, dev, sms, st);
+  }
   return run_tc(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out, relu2, y_bf16, split_ws,
                 split_ws_bytes, dev, sms, st, pdl);
 }

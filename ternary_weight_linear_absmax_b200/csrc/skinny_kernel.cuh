@@ -51,6 +51,9 @@ constexpr int kSkThreads = 512;
 constexpr int kSkWarps = kSkThreads / 32;
 constexpr int kSkKC = 512;              // K values per stage (one weight box)
 constexpr int kSkMaxTokens = 64;
+// Above this many tokens the tensor-core tiles take a contraction when they
+// fill at least half of the SMs.
+constexpr int kSkPreferTokens = 32;
 constexpr int kSkMaxRowsPad = 128;      // rows computed per CTA ≤ 128: ≤ 16 n-tiles
 constexpr size_t kSkSmemCap = 226 * 1024;  // of the 227 KiB a CTA may opt into
 

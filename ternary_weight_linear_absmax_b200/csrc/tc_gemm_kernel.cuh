@@ -1,5 +1,5 @@
 // Ternary × INT8 contraction on the 5th-generation tensor cores (tcgen05,
-// kind::i8) for more than 64 tokens (prefill, the FFN at larger batches).
+// kind::i8) for more than 32 tokens (prefill, the FFN at larger batches).
 //
 // "BitNet b1.58 — quantização ternária, BitLinear, Zero-GEMM", section
 // "Como funciona a camada BitLinear ... (Zero-GEMM)?": acc = A_q·W_qᵀ in

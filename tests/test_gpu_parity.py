@@ -166,9 +166,13 @@ def test_quant_acts_special_rows(bl):
 
 ZG_CASES = [
     (1, 64, 128), (2, 128, 200), (3, 192, 256), (4, 512, 256),      # GEMV path
-    (5, 128, 128), (16, 4096, 384), (17, 192, 200), (33, 512, 130),  # skinny path (5..64 tokens)
-    (64, 1024, 256), (8, 64, 1), (48, 3200, 1500), (20, 640, 9000),
-    (7, 64, 20000), (64, 4096, 4096), (32, 4096, 11008),
+    (5, 128, 128), (16, 4096, 384), (17, 192, 200), (32, 512, 130),  # skinny path (5..32 tokens)
+    (31, 1024, 256), (8, 64, 1), (24, 3200, 1500), (20, 640, 9000),
+    (7, 64, 20000), (32, 4096, 4096), (32, 4096, 11008),
+    # 33..64 tokens: skinny (4 m-tiles) while tiles would fill under half the SMs ...
+    (33, 512, 130), (48, 3200, 1500), (64, 1024, 256),
+    # ... tensor-core tiles otherwise (unsplit, and with K split in 4)
+    (40, 256, 11008), (64, 4096, 4096),
     (65, 256, 200), (100, 320, 256), (128, 256, 128), (129, 640, 260),  # tensor-core path
     (256, 512, 384), (300, 384, 512), (520, 128, 136),
     (384, 128, 7680), (300, 256, 9000),  # 192-token tiles (one round instead of two of 128)

@@ -11,7 +11,7 @@ Checked element by element against the oracle: the int8 tokens, γ_A and
 Σ A_q that the fused decode-GEMV prologue makes (M ≤ 4; the first and the
 last CTA, since every CTA quantises for itself), and in the FFN block the
 quantised input X_q, the INT32 up-projection, the requantised R_q, γ_r and
-Σ R_q, at M ∈ {1, 2, 4} (fused GEMV prologues) and {5, 64, 512} (separate
+Σ R_q, at M ∈ {1, 2, 4} (fused GEMV prologues) and {5, 32, 64, 512} (separate
 kernels). Rounding-boundary exemptions are counted and printed in the
 terminal summary; integers must otherwise be identical.
 """
@@ -106,7 +106,7 @@ def ffn_weights():
     return cu, gu, cd, gd, dev
 
 
-FFN_CASES = [(1, 0), (1, -1), (2, 0), (4, -1), (5, 0), (64, 0), (512, 0)]
+FFN_CASES = [(1, 0), (1, -1), (2, 0), (4, -1), (5, 0), (32, 0), (64, 0), (512, 0)]
 
 
 @pytest.mark.parametrize("M,cta", FFN_CASES)

@@ -7,8 +7,8 @@ shard's step 3, then the INT32 SUM of the partial down-projections (what
 all-reduce(SUM) computes), then the dequantisation. No kernel waits on
 another. The result must equal the unsharded bl_ffn_relu2 output bit for bit
 and the oracle's INT32 down-projection exactly, for shards that take the
-fused GEMV (M = 1), the warp-level MMA (M = 5, 64) and the tensor-core
-(M = 130) paths.
+fused GEMV (M = 1), the warp-level MMA (M = 5, 32) and the tensor-core
+(M = 64, 130) paths.
 """
 import numpy as np
 import pytest
@@ -42,7 +42,7 @@ def block():
 
 
 @pytest.mark.parametrize("world", [2, 3, 4])
-@pytest.mark.parametrize("M", [1, 5, 64, 130])
+@pytest.mark.parametrize("M", [1, 5, 32, 64, 130])
 def test_tp_ffn_lockstep_equals_unsharded(bl, block, world, M):
     from ternary_weight_linear_absmax_b200.tp_ffn import shard_packed
     K, H, cu, gu, cd, gd = block
