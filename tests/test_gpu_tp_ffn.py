@@ -75,3 +75,39 @@ def test_dequant_i32_fp32_and_relu2(bl):
     Y2 = bl.bl_dequant_i32(to_dev(acc), to_dev(gA), to_dev(np.array([g], np.float32)), relu2=True,
                            out_dtype=torch.float32).cpu().numpy()
     assert_close(Y2, oracle.dequant(acc, gA, g, relu2=True), True)
+
+
+@pytest.fixture(scope="module")
+def block_wide():
+    K, H = 4096, 5504
+    cu, gu = oracle.quant_weights(si.weights(H, K, seed=3, dtype="bf16").f32, EPS)
+    cd, gd = oracle.quant_weights(si.weights(K, H, seed=4, dtype="bf16").f32, EPS)
+    return K, H, cu, gu, cd, gd
+
+
+@pytest.mark.parametrize("M", [64, 130])
+def test_tp_ffn_wide_shards(bl, block_wide, M):
+    """Wider shards (two ranks of 4096 -> 5504 -> 4096: 2752 hidden rows per
+    rank, 32 K blocks in the up-projection). The block output must equal
+    the unsharded block bit for bit; the oracle checks three tokens (every
+    step is per token)."""
+    from ternary_weight_linear_absmax_b200.tp_ffn import shard_packed
+    K, H, cu, gu, cd, gd = block_wide
+    pu, pd = to_dev(oracle.pack_ternary(cu)), to_dev(oracle.pack_ternary(cd))
+    gu_d, gd_d = to_dev(np.array([gu], np.float32)), to_dev(np.array([gd], np.float32))
+    X = si.activations(M, K, seed=90 + M, outliers=True, dtype="bf16")
+    Xd = X.torch(DEV)
+    shards = [shard_packed(pu, pd, H, 2, r) for r in range(2)]
+    ups = [bl.bl_ffn_tp_up(Xd, su, gu_d, EPS) for su, _ in shards]
+    gamma_r = torch.stack([u[2] for u in ups]).amax(dim=0)
+    parts = [bl.bl_ffn_tp_down(u[0], u[1], gu_d, gamma_r, sd, EPS) for u, (_, sd) in zip(ups, shards)]
+    acc_down = torch.stack(parts).sum(dim=0, dtype=torch.int32)
+    Y = bl.bl_dequant_i32(acc_down, gamma_r, gd_d)
+    Y_full = bl.bl_ffn_relu2(Xd, pu, gu_d, pd, gd_d, EPS)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y_full), "sharded block differs from the unsharded block"
+    rows = [0, M // 2, M - 1]
+    ref = oracle.ffn_relu2(X.f32[rows], cu, gu, cd, gd, EPS)
+    np.testing.assert_array_equal(acc_down.cpu().numpy()[rows], ref["acc_down"])
+    np.testing.assert_array_equal(gamma_r.cpu().numpy()[rows], ref["gammaR"])
+    assert_close(Y.float().cpu().numpy()[rows], ref["Y"], False)
