@@ -214,6 +214,31 @@ def test_zero_gemm_random_shapes(bl, M, K, N):
     np.testing.assert_array_equal(acc, oracle.zero_gemm(Aq, codes))
 
 
+def _band_shapes(count, seed):
+    """33..64 tokens: the tensor-core tiles take these when they (times their
+    K ranges) fill at least half of the SMs, the warp-level kernel otherwise."""
+    u = si.uniform(seed, 3 * count).reshape(count, 3)
+    return [(int(33 + a * 31.999), 64 * int(1 + b * 50), int(1 + c * 12000)) for a, b, c in u]
+
+
+@pytest.mark.parametrize("M,K,N", _band_shapes(12, seed=3364))
+def test_contraction_band_33_64(bl, M, K, N):
+    """Bit-exact INT32 with room for K-split partials (bl_zero_gemm), and the
+    same contraction through bl_linear_q with no workspace at all (row sums
+    given; γ_A = 127, γ = 1, so Y = acc exactly in fp32)."""
+    Aq = random_int8(M, K, seed=M * 17 + K)
+    codes = random_codes(N, K, seed=N * 29 + K)
+    packed = to_dev(oracle.pack_ternary(codes))
+    ref = oracle.zero_gemm(Aq, codes)
+    acc = bl.bl_zero_gemm(to_dev(Aq), packed).cpu().numpy()
+    np.testing.assert_array_equal(acc, ref)
+    rs = to_dev(Aq.astype(np.int32).sum(axis=1).astype(np.int32))
+    Y = bl.bl_linear_q(to_dev(Aq), to_dev(np.full(M, 127.0, np.float32)), packed,
+                       to_dev(np.array([1.0], np.float32)), rowsum=rs,
+                       out_dtype=torch.float32).cpu().numpy()
+    np.testing.assert_array_equal(Y, ref.astype(np.float32))
+
+
 def test_zero_gemm_extremes(bl):
     """Worst-case magnitudes: all +127 / -127 activations against all-±1 rows."""
     for M in (1, 40):
