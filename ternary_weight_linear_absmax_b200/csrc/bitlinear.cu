@@ -776,10 +776,10 @@ bl_status make_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint6
   return r == CUDA_SUCCESS ? BL_OK : BL_ERR_CUDA;
 }
 
-template <int BN, bool MASK, bool DUAL = false>
+template <int BN, bool MASK, bool DUAL, int MAJ>
 bl_status launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const GmParams& p, int dev,
                         cudaStream_t st) {
-  auto* k = bf16_gemm_kernel<BN, MASK, DUAL>;
+  auto* k = bf16_gemm_kernel<BN, MASK, DUAL, MAJ>;
   constexpr size_t smem = GmConfig<BN, DUAL>::kSmem;
   BL_TRY(ensure_smem(k, dev, smem));
   const dim3 grid((unsigned)((p.rows + kGmBM - 1) / kGmBM), (unsigned)((p.cols + BN - 1) / BN));
@@ -788,28 +788,39 @@ bl_status launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const GmPa
   return BL_OK;
 }
 
-// C[rows, cols] (fp32) = epilogue(A[rows, kdim] · B[cols, kdim]ᵀ); A, B bf16
-// with row strides lda, ldb elements.
+template <int MAJ, bool MASK>
+bl_status launch_gemm_form(const CUtensorMap& ta, const CUtensorMap& tb, const GmParams& p,
+                           bool wide, bool dual, int dev, cudaStream_t st) {
+  if (dual) return launch_gemm_t<256, MASK, true, MAJ>(ta, tb, p, dev, st);
+  if (wide) return launch_gemm_t<256, MASK, false, MAJ>(ta, tb, p, dev, st);
+  return launch_gemm_t<128, MASK, false, MAJ>(ta, tb, p, dev, st);
+}
+
+// C[rows, cols] (fp32) = epilogue(A · Bᵀ) over kdim, A and B bf16 with row
+// strides lda, ldb elements. The two forms the STE backward uses:
+//   maj = kMajBMN, no mask: A [rows, kdim], B stored [kdim, cols] (dA);
+//   maj = kMajAMN | kMajBMN, mask: A stored [kdim, rows], B [kdim, cols] (dW).
 bl_status run_bf16_gemm(const void* A, int64_t lda, const void* B, int64_t ldb, GmParams p,
-                        int dev, cudaStream_t st) {
+                        int maj, int dev, cudaStream_t st) {
   if (p.rows > (int64_t)65535 * kGmBM) return BL_ERR_SHAPE;
+  const bool mask = p.mask_w != nullptr;
+  if (maj != (mask ? (kMajAMN | kMajBMN) : kMajBMN)) return BL_ERR_UNSUPPORTED;
   const bool wide = p.cols >= 256;
   CUtensorMap ta, tb;
-  BL_TRY(make_map_bf16(&ta, A, (uint64_t)p.rows, (uint64_t)p.kdim, (uint64_t)lda, kGmBM));
-  BL_TRY(make_map_bf16(&tb, B, (uint64_t)p.cols, (uint64_t)p.kdim, (uint64_t)ldb, wide ? 256 : 128));
-  const bool mask = p.mask_w != nullptr;
+  if (maj & kMajAMN)
+    BL_TRY(make_map_bf16(&ta, A, (uint64_t)p.kdim, (uint64_t)p.rows, (uint64_t)lda, kGmBK));
+  else
+    BL_TRY(make_map_bf16(&ta, A, (uint64_t)p.rows, (uint64_t)p.kdim, (uint64_t)lda, kGmBM));
+  BL_TRY(make_map_bf16(&tb, B, (uint64_t)p.kdim, (uint64_t)p.cols, (uint64_t)ldb, kGmBK));
   // More tiles than SMs: two CTAs per SM (two stages each), so one CTA's
   // epilogue overlaps the other's MMAs (2048 x 4096 x 4096: dA 69.4 -> 67.9 us,
   // dW 98.6 -> 96.7 us; 128-wide tiles two per SM were slower).
   int dev_sms = 0;
   BL_CUDA(cudaDeviceGetAttribute(&dev_sms, cudaDevAttrMultiProcessorCount, dev));
   const int64_t tiles = ((p.rows + kGmBM - 1) / kGmBM) * ((p.cols + 255) / 256);
-  if (wide && tiles > dev_sms)
-    return mask ? launch_gemm_t<256, true, true>(ta, tb, p, dev, st)
-                : launch_gemm_t<256, false, true>(ta, tb, p, dev, st);
-  if (wide)
-    return mask ? launch_gemm_t<256, true>(ta, tb, p, dev, st) : launch_gemm_t<256, false>(ta, tb, p, dev, st);
-  return mask ? launch_gemm_t<128, true>(ta, tb, p, dev, st) : launch_gemm_t<128, false>(ta, tb, p, dev, st);
+  const bool dual = wide && tiles > dev_sms;
+  return mask ? launch_gemm_form<kMajAMN | kMajBMN, true>(ta, tb, p, wide, dual, dev, st)
+              : launch_gemm_form<kMajBMN, false>(ta, tb, p, wide, dual, dev, st);
 }
 
 inline int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
@@ -1531,7 +1542,7 @@ bl_status bl_linear_lut(const void* A, bl_dtype a_dtype, int64_t M, int64_t K, c
 // STE backward.
 
 size_t bl_ste_grad_input_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  // W_qᵀ [K, N8] bf16, plus a bf16 copy of dY [M, N] when it is fp32
+  // W_q [N, K] bf16 (room for K·N8), plus a bf16 copy of dY [M, N] when it is fp32
   return align_up((size_t)K * round8(N) * 2) + align_up((size_t)M * N * 2);
 }
 
@@ -1556,11 +1567,18 @@ bl_status bl_ste_grad_input(const void* dY, bl_dtype dy_dtype, int64_t M, int64_
   BL_TRY(current_device(&dev, &sms));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
-  __nv_bfloat16* wqt = reinterpret_cast<__nv_bfloat16*>(base);
+  // W_q in its own layout [N, K]: the GEMM reads it as an MN-major operand
+  // (the contraction index N is its row index).
+  __nv_bfloat16* wq = reinterpret_cast<__nv_bfloat16*>(base);
   const int64_t Np = round8(N);
-  expand_wqt_kernel<<<dim3((unsigned)((Np + 63) / 64), (unsigned)(K / 64)), 256, 0, st>>>(
-      W_packed, N, K, Np, wqt);
-  BL_CUDA(cudaGetLastError());
+  {
+    const int64_t words = N * (K / 16);
+    int64_t blocks = (words + 255) / 256;
+    if (blocks > 16 * (int64_t)sms) blocks = 16 * (int64_t)sms;
+    expand_wq_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(W_packed),
+                                                       words, wq);
+    BL_CUDA(cudaGetLastError());
+  }
   const void* a = dY;
   if (dy_dtype == BL_F32) {  // one bf16 rounding of dY
     __nv_bfloat16* dyb = reinterpret_cast<__nv_bfloat16*>(base + align_up((size_t)K * Np * 2));
@@ -1577,7 +1595,7 @@ bl_status bl_ste_grad_input(const void* dY, bl_dtype dy_dtype, int64_t M, int64_
   p.kdim = N;
   p.C = dA;
   p.scale = gamma;
-  return run_bf16_gemm(a, N, wqt, Np, p, dev, st);
+  return run_bf16_gemm(a, N, wq, K, p, kMajBMN, dev, st);
 }
 
 size_t bl_ste_grad_weight_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -1617,30 +1635,35 @@ bl_status bl_ste_grad_weight(const void* dY, bl_dtype dy_dtype, int64_t M, int64
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t Mp = round8(M);
   uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
-  __nv_bfloat16* dyt = reinterpret_cast<__nv_bfloat16*>(base);
-  __nv_bfloat16* aht = reinterpret_cast<__nv_bfloat16*>(base + align_up((size_t)N * Mp * 2));
-  // dYᵀ [N, Mp] and Âᵀ [K, Mp] (N, K multiples of 8; Mp of 8).
-  const dim3 gy((unsigned)((N + 63) / 64), (unsigned)((Mp + 63) / 64));
-  if (dy_dtype == BL_BF16)
-    transpose64_bf16_kernel<__nv_bfloat16><<<gy, 256, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16*>(dY), nullptr, M, N, Mp, dyt);
-  else
-    transpose64_bf16_kernel<float><<<gy, 256, 0, st>>>(reinterpret_cast<const float*>(dY), nullptr,
-                                                       M, N, Mp, dyt);
-  BL_CUDA(cudaGetLastError());
-  transpose64_bf16_kernel<int8_t><<<dim3((unsigned)((K + 63) / 64), (unsigned)((Mp + 63) / 64)), 256,
-                                    0, st>>>(A_q, gamma_A, M, K, Mp, aht);
+  // The GEMM reads dY [M, N] and Â [M, K] in their own layouts, as MN-major
+  // operands (the contraction index M is the row index of both): dY as given
+  // when bf16, else a bf16 copy; Â scaled into bf16. Rows past M read as
+  // zeros.
+  const __nv_bfloat16* dyb = reinterpret_cast<const __nv_bfloat16*>(dY);
+  if (dy_dtype != BL_BF16) {
+    __nv_bfloat16* dyc = reinterpret_cast<__nv_bfloat16*>(base);
+    int64_t blocks = (M * N / 4 + 255) / 256;
+    if (blocks > 16 * (int64_t)sms) blocks = 16 * (int64_t)sms;
+    convert_bf16_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const float*>(dY), M * N,
+                                                          dyc);
+    BL_CUDA(cudaGetLastError());
+    dyb = dyc;
+  }
+  __nv_bfloat16* ahb = reinterpret_cast<__nv_bfloat16*>(base + align_up((size_t)N * Mp * 2));
+  int64_t sblocks = (M * (K / 8) + 255) / 256;
+  if (sblocks > 16 * (int64_t)sms) sblocks = 16 * (int64_t)sms;
+  scale_rows_bf16_kernel<<<(unsigned)sblocks, 256, 0, st>>>(A_q, gamma_A, M, K, ahb);
   BL_CUDA(cudaGetLastError());
   GmParams p = {};
   p.rows = N;
   p.cols = K;
-  p.kdim = Mp;
+  p.kdim = M;
   p.C = dW;
   p.mask_w = W;
   p.mask_bf16 = w_dtype == BL_BF16;
   p.mask_gamma = gamma;
   p.eps = eps;
-  return run_bf16_gemm(dyt, Mp, aht, Mp, p, dev, st);
+  return run_bf16_gemm(dyb, N, ahb, K, p, kMajAMN | kMajBMN, dev, st);
 }
 
 bl_status bl_check_device_error(bl_stream_t stream) {

@@ -7,11 +7,13 @@
 //   dA = dY·Ŵ                         [M, K]   (contraction over N)
 //   dW = 1[|W ÷ (γ+ε)| ≤ 1] ⊙ dYᵀ·Â   [N, K]   (contraction over M)
 // Both are dense contractions, so both run as one tcgen05 kind::f16 GEMM
-// (bf16 operands, fp32 accumulation in tensor memory) after small layout
-// kernels that put the contraction dimension innermost:
-//   dA:  A = dY [M, N] (as given, bf16), B = W_qᵀ [K, N] bf16 {-1, 0, +1}
-//        expanded from the packed codes, scale γ in the epilogue;
-//   dW:  A = dYᵀ [N, M] bf16, B = Âᵀ [K, M] bf16, mask in the epilogue.
+// (bf16 operands, fp32 accumulation in tensor memory):
+//   dA:  A = dY [M, N] (as given, bf16; K-major), B = W_q [N, K] bf16
+//        {-1, 0, +1} expanded from the packed codes in its own layout and
+//        read as an MN-major operand; scale γ in the epilogue;
+//   dW:  A = dY and B = Â [M, K] bf16 in their natural row-major layouts,
+//        both read as MN-major operands (the contraction index M is the row
+//        index of both); mask in the epilogue.
 // W_q is exact in bf16; dY (when fp32) and Â are rounded to bf16 once.
 #pragma once
 
@@ -60,6 +62,23 @@ __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t m, uint32_t n) {
          | ((m >> 4) << 24);  // M / 16
 }
 
+// MN-major operand tile with the 128-byte swizzle, as a TMA box of 64
+// elements × 64 rows writes it: each 128-byte row holds 64 consecutive MN
+// elements of one K index, 8 K rows form a 1024-byte swizzle atom (stride
+// byte offset), and 64-element MN chunks sit `lbo` bytes apart (leading byte
+// offset). Same field encoding as smem_desc_sw128.
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+// Operand majors of the GEMM (instruction descriptor bits 15 and 16).
+constexpr int kMajAMN = 1, kMajBMN = 2;
+
 __device__ __forceinline__ void mma_bf16_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                                  uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -90,7 +109,11 @@ __device__ __forceinline__ void tma_load_2x2d_warp(uint64_t* bar, uint32_t tx, v
       : "memory");
 }
 
-template <int BN, bool MASK, bool DUAL = false>
+// MAJ: kMajAMN — A is stored [kdim, rows] instead of [rows, kdim]; kMajBMN —
+// B is stored [kdim, cols] instead of [cols, kdim] (row-major, the MN index
+// innermost). An MN-major operand takes one 64 × 64 box per 64 rows (cols)
+// of its tile and stage, a K-major one a single box of 64 K × its rows.
+template <int BN, bool MASK, bool DUAL = false, int MAJ = 0>
 __global__ void __launch_bounds__(kGmThreads, DUAL ? 2 : 1)
 bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                  const GmParams p) {
@@ -142,15 +165,43 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
         *s_abort = 1;
         break;
       }
-      tma_load_2x2d_warp(&full[s], C::kStageA + C::kStageB, s_a + s * C::kStageA, &tm_a,
-                         s_b + s * C::kStageB, &tm_b, kb * kGmBK, (int32_t)r0, (int32_t)c0);
+      if constexpr (MAJ != 0) {
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], C::kStageA + C::kStageB);
+          uint8_t* da = s_a + s * C::kStageA;
+          uint8_t* db = s_b + s * C::kStageB;
+          if constexpr ((MAJ & kMajAMN) != 0) {
+#pragma unroll
+            for (int j = 0; j < kGmBM / 64; ++j)
+              tma_load_2d(da + j * 8192, &tm_a, (int32_t)(r0 + 64 * j), kb * kGmBK, &full[s]);
+          } else {
+            tma_load_2d(da, &tm_a, kb * kGmBK, (int32_t)r0, &full[s]);
+          }
+          if constexpr ((MAJ & kMajBMN) != 0) {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(db + j * 8192, &tm_b, (int32_t)(c0 + 64 * j), kb * kGmBK, &full[s]);
+          } else {
+            tma_load_2d(db, &tm_b, kb * kGmBK, (int32_t)c0, &full[s]);
+          }
+        }
+        __syncwarp();
+      } else {
+        tma_load_2x2d_warp(&full[s], C::kStageA + C::kStageB, s_a + s * C::kStageA, &tm_a,
+                           s_b + s * C::kStageB, &tm_b, kb * kGmBK, (int32_t)r0, (int32_t)c0);
+      }
     }
     if (*s_abort && lane == 0) {  // drain copies in flight (bounded) before exit
       for (int d = max(0, kb - S); d < kb; ++d) mbar_wait_for(&full[d % S], (d / S) & 1, 100000000ull);
     }
   } else if (warp == 1) {
     // ---- MMA issuer ----
-    constexpr uint32_t idesc = idesc_bf16(kGmBM, BN);
+    constexpr uint32_t idesc = idesc_bf16(kGmBM, BN) | ((MAJ & kMajAMN) ? (1u << 15) : 0u) |
+                               ((MAJ & kMajBMN) ? (1u << 16) : 0u);
+    // Per 16-K MMA: a K-major tile advances 32 bytes inside its swizzle rows
+    // (+2 in the address field); an MN-major tile (64 K rows of 128 bytes per
+    // 64-element chunk) advances 16 K rows, two swizzle atoms (+128).
+    constexpr uint64_t a_step = (MAJ & kMajAMN) ? 128 : 2, b_step = (MAJ & kMajBMN) ? 128 : 2;
     const uint32_t a_base = __shfl_sync(0xffffffffu, smem_u32(s_a), 0);
     const uint32_t b_base = __shfl_sync(0xffffffffu, smem_u32(s_b), 0);
     for (int kb = 0; kb < KB; ++kb) {
@@ -161,11 +212,13 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
         break;
       }
       tc_fence_after();
-      const uint64_t ad = smem_desc_sw128(a_base + s * C::kStageA);
-      const uint64_t bd = smem_desc_sw128(b_base + s * C::kStageB);
+      const uint64_t ad = (MAJ & kMajAMN) ? smem_desc_sw128_mn(a_base + s * C::kStageA, 64 * 128)
+                                          : smem_desc_sw128(a_base + s * C::kStageA);
+      const uint64_t bd = (MAJ & kMajBMN) ? smem_desc_sw128_mn(b_base + s * C::kStageB, 64 * 128)
+                                          : smem_desc_sw128(b_base + s * C::kStageB);
 #pragma unroll
-      for (int kk = 0; kk < kGmBK / 16; ++kk)  // 16 bf16 = 32 bytes per MMA: +2 in the address field
-        mma_bf16_ss_warp(tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc,
+      for (int kk = 0; kk < kGmBK / 16; ++kk)
+        mma_bf16_ss_warp(tmem, ad + kk * a_step, bd + kk * b_step, idesc,
                          (kb > 0 || kk > 0) ? 1u : 0u);
       mma_commit_warp(&empty[s]);
     }
@@ -265,48 +318,37 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
 }
 
 // ---------------------------------------------------------------------------
-// Layout kernels (64 × 64 tiles through shared memory, 256 threads).
+// Layout kernels (256 threads).
 
-// W_qᵀ [K, Np] bf16 from the packed codes [N, K/4]: element (k, n) = c(n,k) - 1
-// (columns n ≥ N are zero; Np a multiple of 8). Block tile: 64 rows n × 64
-// weights k. Each thread loads one 32-bit word (16 codes; the 32 lanes of a
-// warp take 32 rows n at the same word) and expands it into the tile's
-// column n; then each thread writes 8 consecutive n of an output row k with
-// one 16-byte store.
+// W_q [N, K] bf16 from the packed codes [N, K/4]: element (n, k) = c(n, k) - 1.
+// Each thread expands one 32-bit word (16 codes; weight 16g + 4j + i of a row
+// sits at bits 8i + 2j of its word g) into 16 consecutive bf16 of the same
+// row: two 16-byte stores.
 __global__ void __launch_bounds__(256)
-expand_wqt_kernel(const uint8_t* __restrict__ W, int64_t N, int64_t K, int64_t Np,
-                  __nv_bfloat16* __restrict__ out) {
-  __shared__ __align__(16) __nv_bfloat16 tile[64][72];  // [k][n], rows 16-byte aligned
-  const int64_t n0 = (int64_t)blockIdx.x * 64, k0 = (int64_t)blockIdx.y * 64;
-  const int tid = threadIdx.x;
-  {
-    const int i = tid & 63, q = tid >> 6;  // row n0+i, word q of the 64 weights
-    const int64_t n = n0 + i;
-    uint32_t word = 0x55555555u;           // codes 1 (w = 0) past N
-    if (n < N) word = __ldg(reinterpret_cast<const uint32_t*>(W + n * (K / 4)) + (k0 >> 4) + q);
+expand_wq_kernel(const uint32_t* __restrict__ W, int64_t words, __nv_bfloat16* __restrict__ out) {
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < words;
+       t += (int64_t)gridDim.x * blockDim.x) {
+    const uint32_t word = __ldg(W + t);
+    uint32_t h[8];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {  // weight 16q + 4j + i2 at bits 8·i2 + 2·j
-      const int j = e >> 2, i2 = e & 3;
-      const int c = (int)((word >> (8 * i2 + 2 * j)) & 3u);
-      tile[16 * q + e][i] = __float2bfloat16_rn((float)(c - 1));
+    for (int e2 = 0; e2 < 8; ++e2) {  // weights 2·e2 and 2·e2 + 1 of the word
+      uint32_t pair = 0;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int e = 2 * e2 + u, i = e & 3, jj = e >> 2;
+        const int c = (int)((word >> (8 * i + 2 * jj)) & 3u);
+        pair |= (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn((float)(c - 1))) << (16 * u);
+      }
+      h[e2] = pair;
     }
-  }
-  __syncthreads();
-  for (int e = tid; e < 64 * 8; e += 256) {
-    const int r = e >> 3, g = e & 7;  // output row k0 + r, columns n0 + 8g .. + 7
-    const int64_t n = n0 + 8 * g;
-    if (n < Np)
-      *reinterpret_cast<uint4*>(out + (k0 + r) * Np + n) = *reinterpret_cast<const uint4*>(&tile[r][8 * g]);
+    uint4* o = reinterpret_cast<uint4*>(out + 16 * t);
+    o[0] = make_uint4(h[0], h[1], h[2], h[3]);
+    o[1] = make_uint4(h[4], h[5], h[6], h[7]);
   }
 }
 
-// Transpose-convert an [R, Cc] matrix (bf16, fp32 or int8; Cc a multiple of
-// 8) into [Cc, Rp] bf16 (Rp a multiple of 8; rows r ≥ R give zeros), row r
-// optionally scaled by fp32(rscale[r] ÷ 127): dYᵀ, and Âᵀ from int8 A_q with
-// Â[m, k] = fp32(γ_A[m] ÷ 127) · A_q[m, k]. 64 × 64 tiles: each thread reads
-// 8 consecutive elements of a row and writes 8 consecutive bf16 of an output
-// row; the tile's 16-byte chunks are swizzled by row ÷ 8 so that both passes
-// are free of shared-memory bank conflicts.
+// Conversion helpers: two floats to a bf16 pair (round to nearest even), and
+// eight consecutive elements of an int8 / bf16 / fp32 row to fp32.
 __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
   return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
@@ -332,51 +374,28 @@ __device__ __forceinline__ void load8_f32(const T* p, float (&v)[8]) {
   }
 }
 
-template <typename T>
+// Â = bf16(fp32(rscale[r] ÷ 127) · A_q[r, c]) for an int8 [R, Cc] matrix (Cc a
+// multiple of 8), in its own layout: one fp32 division per row, one fp32
+// product and one rounding to bf16 per element; eight elements per thread
+// and 16-byte stores.
 __global__ void __launch_bounds__(256)
-transpose64_bf16_kernel(const T* __restrict__ in, const float* __restrict__ rscale, int64_t R,
-                        int64_t Cc, int64_t Rp, __nv_bfloat16* __restrict__ out) {
-  __shared__ __align__(16) uint4 tile[64][8];  // 64 rows × 64 bf16
-  const int64_t c0 = (int64_t)blockIdx.x * 64, r0 = (int64_t)blockIdx.y * 64;
-  const int tid = threadIdx.x;
-  for (int e = tid; e < 64 * 8; e += 256) {
-    const int i = e >> 3, g = e & 7;
-    const int64_t r = r0 + i, c = c0 + 8 * g;
+scale_rows_bf16_kernel(const int8_t* __restrict__ in, const float* __restrict__ rscale, int64_t R,
+                       int64_t Cc, __nv_bfloat16* __restrict__ out) {
+  const int64_t per_row = Cc / 8;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < R * per_row;
+       t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = t / per_row, c = (t - r * per_row) * 8;
     float v[8];
-    if (r < R && c < Cc) {
-      load8_f32<T>(in + r * Cc + c, v);
-      if (rscale != nullptr) {
-        const float sc = __fdiv_rn(__ldg(rscale + r), 127.0f);
+    load8_f32<int8_t>(in + r * Cc + c, v);
+    const float sc = __fdiv_rn(__ldg(rscale + r), 127.0f);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(sc, v[j]);
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = 0.0f;
-    }
+    for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(sc, v[j]);
     uint4 w;
     w.x = bf16x2_bits(v[0], v[1]);
     w.y = bf16x2_bits(v[2], v[3]);
     w.z = bf16x2_bits(v[4], v[5]);
     w.w = bf16x2_bits(v[6], v[7]);
-    tile[i][g ^ ((i >> 3) & 7)] = w;
-  }
-  __syncthreads();
-  const uint16_t* tb = reinterpret_cast<const uint16_t*>(&tile[0][0]);
-  for (int e = tid; e < 64 * 8; e += 256) {
-    const int cc = e >> 3, l = e & 7;  // output row c0 + cc, columns r0 + 8l .. + 7
-    const int64_t c = c0 + cc, r = r0 + 8 * l;
-    if (c >= Cc || r >= Rp) continue;
-    uint32_t h[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)  // tile row 8l + j: its chunk cc/8 sits at slot (cc/8) ^ l
-      h[j] = tb[(8 * l + j) * 64 + ((((cc >> 3) ^ l)) << 3) + (cc & 7)];
-    uint4 w;
-    w.x = h[0] | (h[1] << 16);
-    w.y = h[2] | (h[3] << 16);
-    w.z = h[4] | (h[5] << 16);
-    w.w = h[6] | (h[7] << 16);
-    *reinterpret_cast<uint4*>(out + c * Rp + r) = w;
+    *reinterpret_cast<uint4*>(out + r * Cc + c) = w;
   }
 }
 
