@@ -118,7 +118,7 @@ __device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity,
 }
 
 // ---------------------------------------------------------------------------
-// Bulk copies (TMA). Non-multicast forms only.
+// Bulk copies (TMA), each into the issuing CTA's own shared memory.
 
 // 2-D tiled tensor copy global -> shared. x (innermost coordinate) must keep
 // x * element size a multiple of 16 bytes.
