@@ -169,27 +169,71 @@ def write_traffic_json(csv_path):
 
 
 # ---------------------------------------------------------------------------
-# clocks sampler (nvidia-smi during the timed region)
+# clocks sampler (during the timed region; reads only)
 
 class ClockSampler:
+    """SM clock and clock-event reasons while the timed region runs. NVML is
+    polled every 5 ms from a thread (the decode step is tens of ms long);
+    without NVML, `nvidia-smi -lms 100` is read instead. Entering waits for
+    the first sample, so the sampler is running when the timing starts."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASON_BITS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+                   ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.samples = []  # (sm_mhz, reason bits) from NVML
+        self.smax = None
+        self.source = None
         self.thread = None
+        self.stop = threading.Event()
+        self.first = threading.Event()
+
+    def _nvml_index(self):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        parts = [q.strip() for q in vis.split(",") if q.strip()]
+        if self.gpu < len(parts) and parts[self.gpu].isdigit():
+            return int(parts[self.gpu])
+        return self.gpu
 
     def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self._nvml_index())
+            self.smax = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.source = "nvml, 5 ms"
+
+            def poll():
+                while not self.stop.is_set():
+                    try:
+                        self.samples.append((float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)),
+                                             int(reasons(h))))
+                    except Exception:
+                        pass
+                    self.first.set()
+                    time.sleep(0.005)
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            self.first.wait(2.0)
+            return self
+        except Exception:
+            self.samples = []
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi, 100 ms"
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            self.first.wait(5.0)
         except Exception:
             self.proc = None
         return self
@@ -197,22 +241,29 @@ class ClockSampler:
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
+            self.first.set()
 
     def __exit__(self, *a):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
-            if self.thread is not None:
-                self.thread.join(timeout=2)
+        if self.thread is not None:
+            self.thread.join(timeout=2)
 
     def summary(self):
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, smax, reasons = [], self.smax, set()
+        for mhz, bits in self.samples:
+            sm.append(mhz)
+            for nm, bit in self.REASON_BITS:
+                if bits & bit:
+                    reasons.add(nm)
+        names = [nm for nm, _ in self.REASON_BITS]
         for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
+            parts = [q.strip() for q in ln.split(",")]
             if len(parts) < 9:
                 continue
             try:
@@ -224,9 +275,10 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(nm)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0,
+                    "source": self.source}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
 # ---------------------------------------------------------------------------
