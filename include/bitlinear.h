@@ -107,6 +107,19 @@ int bl_version(void);
 /* Number of decoded tokens up to which bl_linear uses the fused GEMV path. */
 int bl_gemv_max_tokens(void);
 
+/* Which kernel contracts M int8 tokens with an N × K packed matrix, on a
+ * device with `sms` SMs, when the call's workspace has split_ws_bytes of room
+ * for K-split partials (the optional part of the *_workspace_bytes() sizes):
+ *   0  the GEMV (M ≤ bl_gemv_max_tokens());
+ *   1  the warp-level int8 MMA kernel (5 ≤ M ≤ 32, and 33–64 tokens when the
+ *      tensor-core tiles, times their K ranges, would fill under half of the
+ *      SMs);
+ *   2  tensor-core tiles, K unsplit;
+ *   3  tensor-core tiles with K split into ranges.
+ * -1 for a non-positive size or K not a multiple of 64. Host only: reads no
+ * device state and launches nothing. */
+int bl_contraction_path(int64_t M, int64_t N, int64_t K, int sms, size_t split_ws_bytes);
+
 /* ---------------------------------------------------------------------------
  * bl_quant_weights — quantise_weights_ternary.
  * BLOG, section "Por que 1,58 bits por peso e qual a matemática da

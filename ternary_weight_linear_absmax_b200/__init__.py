@@ -26,7 +26,7 @@ __all__ = [
     "bl_ffn_tp_up", "bl_ffn_tp_down", "bl_dequant_i32", "bl_ste_grad_input", "bl_ste_grad_weight",
     "bl_pack_radix3", "bl_linear_radix3", "bl_pack_lut_index", "bl_linear_lut",
     "bl_probe_pdl_floor", "bl_check_device_error", "bl_selftest_wait_timeout",
-    "bl_gemv_max_tokens", "workspace_bytes", "BitLinearError", "load", "BL_FLAG_PDL",
+    "bl_gemv_max_tokens", "bl_contraction_path", "workspace_bytes", "BitLinearError", "load", "BL_FLAG_PDL",
 ]
 
 _DT = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}
@@ -80,6 +80,13 @@ def _nbytes(t):
 
 def bl_gemv_max_tokens() -> int:
     return int(load().bl_gemv_max_tokens())
+
+
+def bl_contraction_path(M: int, N: int, K: int, sms: int, split_ws_bytes: int = 0) -> int:
+    """Kernel that contracts M int8 tokens with an N × K packed matrix on a
+    device of `sms` SMs: 0 GEMV, 1 warp-level int8 MMA, 2 tensor-core tiles,
+    3 tensor-core tiles with K split (-1: invalid sizes). Host logic only."""
+    return int(load().bl_contraction_path(M, N, K, sms, split_ws_bytes))
 
 
 def workspace_bytes(op: str, M: int, K: int, N: int) -> int:

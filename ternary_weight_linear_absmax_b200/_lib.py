@@ -37,6 +37,7 @@ SIGNATURES = {
     "bl_status_string": (ctypes.c_char_p, [_int]),
     "bl_version": (_int, []),
     "bl_gemv_max_tokens": (_int, []),
+    "bl_contraction_path": (_int, [_i64, _i64, _i64, _int, _sz]),
     "bl_quant_weights_workspace_bytes": (_sz, [_i64, _i64]),
     "bl_quant_weights": (_int, [_vp, _int, _i64, _i64, _f32, _vp, _vp, _vp, _sz, _vp]),
     "bl_quant_acts": (_int, [_vp, _int, _i64, _i64, _f32, _vp, _vp, _vp, _vp]),

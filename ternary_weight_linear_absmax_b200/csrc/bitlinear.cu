@@ -645,18 +645,20 @@ bl_status run_skinny(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, 
 // 5504 -> 4096 shard without split workspace (32 tiles) ran slower on tiles.
 // split_ws: optional scratch (tc_split_ws_bytes) that lets under-filled
 // tensor-core launches split K.
+bool contract_on_tiles(int64_t M, int64_t N, int64_t K, int sms, const void* split_ws,
+                       size_t split_ws_bytes) {
+  if (M > kSkMaxTokens) return true;
+  return M > kSkPreferTokens &&
+         2 * ((N + 127) / 128) * tc_launch_splits(M, N, K, sms, split_ws, split_ws_bytes) >= sms;
+}
+
 bl_status run_contract(const int8_t* Aq, const uint8_t* Wp, int64_t M, int64_t K, int64_t N,
                        const float* gamma, const float* gammaA, const int32_t* rowsum, void* Y,
                        int out, int relu2, int y_bf16, bool pdl, int dev, int sms,
                        cudaStream_t st, void* split_ws = nullptr, size_t split_ws_bytes = 0) {
-  if (M <= kSkMaxTokens) {
-    const bool tiles =
-        M > kSkPreferTokens &&
-        2 * ((N + 127) / 128) * tc_launch_splits(M, N, K, sms, split_ws, split_ws_bytes) >= sms;
-    if (!tiles)
-      return run_skinny(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out == kTcRawI32 ? 1 : 0,
-                        relu2, y_bf16, pdl, dev, sms, st);
-  }
+  if (!contract_on_tiles(M, N, K, sms, split_ws, split_ws_bytes))
+    return run_skinny(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out == kTcRawI32 ? 1 : 0, relu2,
+                      y_bf16, pdl, dev, sms, st);
   return run_tc(Aq, Wp, M, K, N, gamma, gammaA, rowsum, Y, out, relu2, y_bf16, split_ws,
                 split_ws_bytes, dev, sms, st, pdl);
 }
@@ -881,6 +883,15 @@ const char* bl_status_string(bl_status s) {
 int bl_version(void) { return 100; }
 
 int bl_gemv_max_tokens(void) { return kGemvMaxTokens; }
+
+int bl_contraction_path(int64_t M, int64_t N, int64_t K, int sms, size_t split_ws_bytes) {
+  if (M <= 0 || N <= 0 || K <= 0 || K % 64 != 0 || sms <= 0) return -1;
+  if (M <= kGemvMaxTokens) return 0;
+  // Any non-null pointer stands for a workspace part of split_ws_bytes.
+  const void* ws = split_ws_bytes > 0 ? reinterpret_cast<const void*>(&split_ws_bytes) : nullptr;
+  if (!contract_on_tiles(M, N, K, sms, ws, split_ws_bytes)) return 1;
+  return tc_launch_splits(M, N, K, sms, ws, split_ws_bytes) > 1 ? 3 : 2;
+}
 
 size_t bl_quant_weights_workspace_bytes(int64_t N, int64_t K) {
   (void)N;

@@ -45,6 +45,29 @@ def test_status_strings(lib):
     assert lib.bl_gemv_max_tokens() == 4
 
 
+def test_contraction_path(lib):
+    """Routing of a contraction (host logic, no device): GEMV up to 4 tokens,
+    the warp-level kernel up to 32, tensor-core tiles above 64, and from 33 to
+    64 tokens the tiles only when they (times their K ranges) fill at least
+    half of the SMs."""
+    P = lib.bl_contraction_path
+    room = 1 << 40   # workspace with room for K-split partials
+    assert P(1, 6912, 2560, 148, 0) == 0
+    assert P(4, 6912, 2560, 148, room) == 0
+    assert P(16, 11008, 4096, 148, room) == 1
+    assert P(32, 11008, 4096, 148, room) == 1
+    assert P(40, 11008, 4096, 148, room) == 2      # 86 tiles: 2·86 ≥ 148, unsplit
+    assert P(64, 4096, 11008, 148, room) == 3      # 32 tiles × 4 K ranges
+    assert P(64, 4096, 11008, 148, 0) == 1         # no room to split: 32 tiles
+    assert P(48, 1500, 3200, 148, room) == 1       # 12 tiles × 3 ranges
+    assert P(65, 200, 256, 148, 0) == 2
+    assert P(2048, 4096, 4096, 148, room) == 2     # 256 tiles
+    assert P(512, 4096, 11008, 148, room) == 3     # the FFN down-projection
+    assert P(512, 4096, 11008, 148, 0) == 2
+    assert P(40, 11008, 4096, 132, room) == 2      # another SM count
+    assert P(0, 64, 64, 148, 0) == -1 and P(8, 64, 100, 148, 0) == -1
+
+
 def test_workspace_sizes(lib):
     assert lib.bl_quant_weights_workspace_bytes(4096, 4096) >= 1024 * 8
     assert lib.bl_linear_workspace_bytes(1, 2560, 6912) == 0
