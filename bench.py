@@ -863,7 +863,7 @@ def profile_case(name: str) -> int:
         torch.cuda.synchronize()
         for _ in range(3):
             bl.bl_linear_q(Aq, gA, pk, g, rowsum=rs, pdl=True, stream=st)
-    elif name in ("ffn1", "ffn512", "small_chain"):
+    elif name in ("ffn1", "ffn64", "ffn512", "small_chain"):
         K, H = 4096, 11008
         if name.startswith("ffn"):
             M = int(name[3:])
@@ -911,7 +911,7 @@ def main(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--profile-case", choices=["decode", "decode_radix3", "skinny", "prefill", "ste",
-                                               "ffn1", "ffn512", "small_chain"],
+                                               "ffn1", "ffn64", "ffn512", "small_chain"],
                     help="run one small case for an ncu capture and exit")
     ap.add_argument("--traffic-json", metavar="NCU_CSV",
                     help="write the decode GEMV traffic summary read by the bench line "
