@@ -543,3 +543,45 @@ def test_ffn_pdl_chain_shared_workspace(bl, M):
     for (X, cu, gu, cd, gd), y in zip(blocks, outs):
         assert_close(y.float().cpu().numpy(), oracle.ffn_relu2(X.f32, cu, gu, cd, gd, EPS)["Y"],
                      torch.bfloat16)
+
+
+def test_mixed_pdl_chain_shared_workspace(bl):
+    """Calls of every contraction path (GEMV, warp-level MMA, tensor-core tiles
+    with and without K split) and FFN blocks, chained with programmatic
+    dependent launch on one stream and one shared workspace. Each kernel may
+    start before its predecessor ends, so one that read its inputs or reused
+    the shared scratch too early would change a result: every output must
+    equal the same call made alone, bit for bit."""
+    K, N, H = 1024, 1536, 2048
+    W = si.weights(N, K, seed=41, dtype="bf16").torch(DEV)
+    Wu = si.weights(H, K, seed=42, dtype="bf16").torch(DEV)
+    Wd = si.weights(K, H, seed=43, dtype="bf16").torch(DEV)
+    pw, gw = bl.bl_quant_weights(W, EPS)
+    pu, gu = bl.bl_quant_weights(Wu, EPS)
+    pd, gd = bl.bl_quant_weights(Wd, EPS)
+    seq = [("linear", 1), ("linear", 16), ("ffn", 64), ("linear", 200), ("ffn", 1),
+           ("linear", 40), ("ffn", 300), ("linear", 3), ("linear", 600), ("ffn", 16),
+           ("linear", 64), ("ffn", 4)]
+    need = max(bl.workspace_bytes("linear" if op == "linear" else "ffn", M, K,
+                                  N if op == "linear" else H) for op, M in seq)
+    ws = torch.empty(max(1, need), dtype=torch.uint8, device=DEV)
+    xs = [si.activations(M, K, seed=1000 + i, dtype="bf16", outliers=True).torch(DEV)
+          for i, (_, M) in enumerate(seq)]
+
+    def call(i, pdl, workspace):
+        op, M = seq[i]
+        if op == "linear":
+            return bl.bl_linear(xs[i], pw, gw, EPS, workspace=workspace, pdl=pdl)
+        return bl.bl_ffn_relu2(xs[i], pu, gu, pd, gd, EPS, workspace=workspace, pdl=pdl)
+
+    torch.cuda.synchronize()
+    alone = []
+    for i in range(len(seq)):
+        alone.append(call(i, False, None))
+        torch.cuda.synchronize()
+    for _ in range(2):
+        chained = [call(i, True, ws) for i in range(len(seq))]
+        torch.cuda.synchronize()
+        for i, (y, r) in enumerate(zip(chained, alone)):
+            assert torch.equal(y, r), f"call {i} {seq[i]} differs when chained"
+    assert bl.bl_check_device_error() == 0
