@@ -89,3 +89,30 @@ def test_ste_mask_boundary(bl):
     ref = oracle.ste_grad_weight(dY.f32, Aq, gA, Wf, g, EPS)
     assert np.all(dW[0, 2:4] == 0.0) and np.all(ref[0, 2:4] == 0.0)
     assert np.all(dW[0, :2] != 0.0) and np.all(ref[0, :2] != 0.0)
+
+
+def test_ste_full_size_sampled(bl):
+    """The benchmark's shape, 2048 tokens × 4096 × 4096 (two CTAs per SM, 256
+    output tiles), in the launch form bench.py times. Every output row is
+    independent of the others, so the oracle computes three sampled rows of
+    each gradient from the same inputs: dA rows from the matching dY rows,
+    dW rows from the matching dY columns and latent weight rows."""
+    M, N, K = 2048, 4096, 4096
+    W, codes, g, Aq, gA, dY = _problem(M, N, K, seed=11, dy_dtype="bf16")
+    gd = to_dev(np.array([g], np.float32))
+    dA = bl.bl_ste_grad_input(dY.torch(DEV), to_dev(oracle.pack_ternary(codes)), gd).cpu().numpy()
+    dW = bl.bl_ste_grad_weight(dY.torch(DEV), to_dev(Aq), to_dev(gA), W.torch(DEV), gd,
+                               EPS).cpu().numpy()
+    rows_m = [0, 777, M - 1]
+    ref_a = oracle.ste_grad_input(np.ascontiguousarray(dY.f32[rows_m]), codes, g)
+    S_a = float(g) * (np.abs(dY.f32[rows_m].astype(np.float64)) @ np.abs(codes.astype(np.float64)))
+    assert np.all(np.abs(dA[rows_m] - ref_a) <= 2.0 ** -7 * S_a + 1e-30)
+    rows_n = [0, 1500, N - 1]
+    dY_n = np.ascontiguousarray(dY.f32[:, rows_n])
+    W_n = np.ascontiguousarray(W.f32[rows_n])
+    ref_w = oracle.ste_grad_weight(dY_n, Aq, gA, W_n, g, EPS)
+    mask = oracle.ste_weight_mask(W_n, g, EPS)
+    assert np.all(dW[rows_n][mask == 0] == 0.0)
+    A_hat = gA.astype(np.float64)[:, None] / 127.0 * Aq
+    S_w = mask * (np.abs(dY_n.astype(np.float64)).T @ np.abs(A_hat))
+    assert np.all(np.abs(dW[rows_n] - ref_w) <= 2.0 ** -7 * S_w + 1e-30)
