@@ -110,7 +110,9 @@ int bl_gemv_max_tokens(void);
 /* Which kernel contracts M int8 tokens with an N × K packed matrix, on a
  * device with `sms` SMs, when the call's workspace has split_ws_bytes of room
  * for K-split partials (the optional part of the *_workspace_bytes() sizes):
- *   0  the GEMV (M ≤ bl_gemv_max_tokens());
+ *   0  the fused GEMV: M ≤ bl_gemv_max_tokens() and one weight row plus the
+ *      M token rows fit a CTA's shared memory (K ≤ 37,376 at 1 token, 28,096
+ *      at 2, 22,464 at 3, 18,624 at 4); longer rows take path 1;
  *   1  the warp-level int8 MMA kernel (5 ≤ M ≤ 32, and 33–64 tokens when the
  *      tensor-core tiles, times their K ranges, would fill under half of the
  *      SMs);
@@ -195,10 +197,12 @@ bl_status bl_linear_q_ex(const int8_t* A_q, const float* gamma_A,
  * bl_linear — BitLinear forward from float activations:
  * bl_quant_acts, bl_zero_gemm and the dequantisation of bl_linear_q in one
  * call. For M ≤ bl_gemv_max_tokens() it is a single fused GEMV launch (the
- * activation quantiser runs in the kernel prologue; no workspace needed);
- * above that, an activation-quantiser launch and one contraction launch:
+ * activation quantiser runs in the kernel prologue; no workspace needed) as
+ * long as a weight row and the tokens fit one CTA's shared memory (K up to
+ * 37,376 at 1 token, 18,624 at 4; bl_contraction_path says which); above
+ * that, an activation-quantiser launch and one contraction launch:
  * warp-level int8 MMAs over all SMs for M ≤ 32, tensor-core (tcgen05) tiles
- * above. The contraction launches with programmatic dependent launch; it
+ * above. bl_linear_workspace_bytes follows the same rule. The contraction launches with programmatic dependent launch; it
  * reads no memory written by the kernel before it until that kernel has
  * completed, except that after this call's own quantiser it streams W_packed
  * early (the quantiser does not write it).
@@ -229,7 +233,7 @@ bl_status bl_linear_ex(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
  *   req_q      [M, H] int8  FFN only: requantised ReLU² of the up-projection
  *   req_gamma  [M]    fp32  FFN only: γ_r per token
  *   req_rowsum [M]    int32 FFN only: Σ_n R_q[m,n]
- *   cta        On the fused GEMV path (M ≤ bl_gemv_max_tokens()) every CTA
+ *   cta        On the fused GEMV path (bl_contraction_path() == 0) every CTA
  *              quantises the tokens for itself; the taps report the tokens
  *              of CTA `cta` (-1 or any value past the last CTA: the last one).
  * With more tokens the quantiser runs once in its own kernel and the taps are
@@ -264,7 +268,7 @@ bl_status bl_linear_taps(const void* A, bl_dtype a_dtype, int64_t M, int64_t K,
  * call cudaMalloc on its hot path (cudaMalloc may synchronise the device and
  * grows memory outside a fixed budget). This entry point takes the same
  * arguments as bl_linear minus the workspace and allocates nothing: the
- * scratch it needs for more than bl_gemv_max_tokens() tokens (the int8
+ * scratch it needs off the fused GEMV path (bl_contraction_path() != 0: the int8
  * tokens, their scales and row sums: M·K + 8·M bytes, 256-byte aligned
  * pieces) lives in one fixed 4 MiB array inside the library. Every GPU that
  * loads the library holds that array until the process exits.

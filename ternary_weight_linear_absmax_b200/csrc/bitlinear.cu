@@ -169,6 +169,20 @@ bl_status check_dtype(int d) {
 }
 
 // --------------------------------------------------------------------------
+// The fused GEMV (decode) path. Two CTAs per SM: 228 KiB of shared memory per
+// SM, 1 KiB reserved per CTA.
+constexpr size_t kGemvSmemCap = 112 * 1024;
+
+// Up to bl_gemv_max_tokens() tokens a call takes the fused GEMV when a CTA's
+// shared memory holds at least one weight row and the M int8 token rows
+// (K up to 37,376 at 1 token, 18,624 at 4). Longer rows go through the
+// activation quantiser and the warp-level kernel, whose stage ring streams any
+// K; the workspaces are sized accordingly.
+inline bool gemv_path(int64_t M, int64_t K) {
+  return M <= kGemvMaxTokens && gemv_smem_bytes(K, 1, (int)M) <= kGemvSmemCap;
+}
+
+// --------------------------------------------------------------------------
 // Workspace layouts (offsets are multiples of 256 bytes).
 struct ActWs {
   size_t aq, gamma, rowsum, total;
@@ -190,9 +204,14 @@ struct FfnWs {
   size_t rq;      // int8 [M, H]
   size_t gamma_r, rs_r, total;
 };
+// The FFN block takes its GEMV form when both projections fit the GEMV.
+inline bool ffn_gemv_path(int64_t M, int64_t K, int64_t H) {
+  return gemv_path(M, K) && gemv_path(M, H);
+}
+
 FfnWs ffn_ws(int64_t M, int64_t K, int64_t H) {
   FfnWs w{};
-  if (M <= kGemvMaxTokens) {
+  if (ffn_gemv_path(M, K, H)) {
     w.acc_up = 0;
     w.gamma_x = align_up((size_t)M * H * 4);
     w.rmax = w.gamma_x + align_up((size_t)M * 4);
@@ -255,9 +274,6 @@ bl_status launch_gemv_mt(const CUtensorMap& tw, const GemvParams& p, int grid, s
   if (p.M == 2) return launch_gemv_t<2, TA, SRC, OUT>(tw, p, grid, smem, pdl, dev, st);
   return launch_gemv_t<4, TA, SRC, OUT>(tw, p, grid, smem, pdl, dev, st);
 }
-
-// Two CTAs per SM (228 KiB shared memory per SM, 1 KiB reserved per CTA).
-constexpr size_t kGemvSmemCap = 112 * 1024;
 
 // Choose rows per CTA: one wave over the SMs when shared memory allows,
 // at most kGemvMaxRows rows.
@@ -886,7 +902,7 @@ int bl_gemv_max_tokens(void) { return kGemvMaxTokens; }
 
 int bl_contraction_path(int64_t M, int64_t N, int64_t K, int sms, size_t split_ws_bytes) {
   if (M <= 0 || N <= 0 || K <= 0 || K % 64 != 0 || sms <= 0) return -1;
-  if (M <= kGemvMaxTokens) return 0;
+  if (gemv_path(M, K)) return 0;
   // Any non-null pointer stands for a workspace part of split_ws_bytes.
   const void* ws = split_ws_bytes > 0 ? reinterpret_cast<const void*>(&split_ws_bytes) : nullptr;
   if (!contract_on_tiles(M, N, K, sms, ws, split_ws_bytes)) return 1;
@@ -964,7 +980,7 @@ bl_status bl_quant_acts(const void* A, bl_dtype a_dtype, int64_t M, int64_t K, f
 }
 
 size_t bl_zero_gemm_workspace_bytes(int64_t M, int64_t K, int64_t N) {
-  if (M <= kGemvMaxTokens) return 0;
+  if (gemv_path(M, K)) return 0;
   return align_up((size_t)M * 4) + tc_split_ws_bytes(M, N, K);
 }
 
@@ -980,7 +996,7 @@ bl_status bl_zero_gemm(const int8_t* A_q, int64_t M, int64_t K, const uint8_t* W
   BL_TRY(check_ptr(acc));
   // Required: the row sums; the rest of bl_zero_gemm_workspace_bytes (K
   // ranges of under-filled tensor-core launches) is used when present.
-  const size_t need = M <= kGemvMaxTokens ? 0 : align_up((size_t)M * 4);
+  const size_t need = gemv_path(M, K) ? 0 : align_up((size_t)M * 4);
   if (need > 0) {
     if (workspace == nullptr || ws_bytes < need) return BL_ERR_WORKSPACE;
     BL_TRY(check_ptr(workspace));
@@ -988,7 +1004,7 @@ bl_status bl_zero_gemm(const int8_t* A_q, int64_t M, int64_t K, const uint8_t* W
   int dev, sms;
   BL_TRY(current_device(&dev, &sms));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (M <= kGemvMaxTokens) {
+  if (gemv_path(M, K)) {
     GemvParams p = {};
     p.A = A_q;
     p.W = W_packed;
@@ -1008,7 +1024,7 @@ bl_status bl_zero_gemm(const int8_t* A_q, int64_t M, int64_t K, const uint8_t* W
 }
 
 size_t bl_linear_q_workspace_bytes(int64_t M, int64_t K, int64_t N) {
-  if (M <= kGemvMaxTokens) return 0;
+  if (gemv_path(M, K)) return 0;
   return align_up((size_t)M * 4) + tc_split_ws_bytes(M, N, K);
 }
 
@@ -1039,13 +1055,13 @@ bl_status bl_linear_q_ex(const int8_t* A_q, const float* gamma_A, const int32_t*
   BL_TRY(check_ptr(Y));
   // The row sums' part is needed only without rowsum; the rest (K ranges of
   // under-filled tensor-core launches) is used when present.
-  const size_t need = (rowsum || M <= kGemvMaxTokens) ? 0 : align_up((size_t)M * 4);
+  const size_t need = (rowsum || gemv_path(M, K)) ? 0 : align_up((size_t)M * 4);
   if (need > 0 && (workspace == nullptr || ws_bytes < need)) return BL_ERR_WORKSPACE;
   if (workspace != nullptr) BL_TRY(check_ptr(workspace));
   int dev, sms;
   BL_TRY(current_device(&dev, &sms));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (M <= kGemvMaxTokens) {
+  if (gemv_path(M, K)) {
     GemvParams p = {};
     p.A = A_q;
     p.a_scale = gamma_A;
@@ -1079,7 +1095,7 @@ bl_status bl_linear_q_ex(const int8_t* A_q, const float* gamma_A, const int32_t*
 }
 
 size_t bl_linear_workspace_bytes(int64_t M, int64_t K, int64_t N) {
-  if (M <= kGemvMaxTokens) return 0;
+  if (gemv_path(M, K)) return 0;
   return act_ws(M, K).total + tc_split_ws_bytes(M, N, K);
 }
 
@@ -1103,14 +1119,14 @@ static bl_status linear_impl(const void* A, bl_dtype a_dtype, int64_t M, int64_t
   BL_TRY(check_ptr(Y));
   // Required: the quantised tokens; the rest of bl_linear_workspace_bytes (K
   // ranges of under-filled tensor-core launches) is used when present.
-  const size_t need = M <= kGemvMaxTokens ? 0 : act_ws(M, K).total;
+  const size_t need = gemv_path(M, K) ? 0 : act_ws(M, K).total;
   if (need > 0) {
     if (workspace == nullptr || ws_bytes < need) return BL_ERR_WORKSPACE;
     BL_TRY(check_ptr(workspace));
   }
   int dev, sms;
   BL_TRY(current_device(&dev, &sms));
-  if (M <= kGemvMaxTokens) {
+  if (gemv_path(M, K)) {
     GemvParams p = {};
     p.A = A;
     p.W = W_packed;
@@ -1197,7 +1213,7 @@ static bl_status ffn_impl(const void* X, bl_dtype x_dtype, int64_t M, int64_t K,
   BL_TRY(current_device(&dev, &sms));
   uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
   int32_t* acc_up = reinterpret_cast<int32_t*>(base + w.acc_up);
-  if (M <= kGemvMaxTokens) {
+  if (ffn_gemv_path(M, K, H)) {
     float* gX = reinterpret_cast<float*>(base + w.gamma_x);
     GemvParams up = {};
     up.A = X;
@@ -1293,7 +1309,7 @@ bl_status bl_ffn_relu2_taps(const void* X, bl_dtype x_dtype, int64_t M, int64_t 
 // Tensor-parallel FFN steps (one rank's shard of the hidden dimension).
 
 size_t bl_ffn_tp_up_workspace_bytes(int64_t M, int64_t K) {
-  if (M <= kGemvMaxTokens) return 0;
+  if (gemv_path(M, K)) return 0;
   return align_up((size_t)M * K) + align_up((size_t)M * 4);
 }
 
@@ -1321,7 +1337,7 @@ bl_status bl_ffn_tp_up(const void* X, bl_dtype x_dtype, int64_t M, int64_t K, in
   int dev, sms;
   BL_TRY(current_device(&dev, &sms));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (M <= kGemvMaxTokens) {
+  if (gemv_path(M, K)) {
     GemvParams up = {};
     up.A = X;
     up.W = W_up_r;
@@ -1375,7 +1391,7 @@ bl_status bl_ffn_tp_down(const int32_t* acc_up, const float* gamma_x, const floa
   int dev, sms;
   BL_TRY(current_device(&dev, &sms));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (M <= kGemvMaxTokens) {
+  if (gemv_path(M, H_r)) {
     // One launch: the GEMV's prologue requantises the shard with γ_r.
     GemvParams p = {};
     p.A = acc_up;
@@ -1769,7 +1785,7 @@ extern "C" bl_status bl_linear_noalloc(const void* A, bl_dtype a_dtype, int64_t 
   if (gamma == nullptr) return BL_ERR_INVALID_ARG;
   BL_TRY(check_ptr(Y));
   // Scratch this call needs; refuse what the fixed array cannot hold.
-  const size_t need = M <= kGemvMaxTokens ? 0 : act_ws(M, K).total;
+  const size_t need = gemv_path(M, K) ? 0 : act_ws(M, K).total;
   if (need > kNoAllocScratchBytes) return BL_ERR_WORKSPACE;
   int dev, sms;
   BL_TRY(current_device(&dev, &sms));

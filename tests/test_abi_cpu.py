@@ -66,6 +66,12 @@ def test_contraction_path(lib):
     assert P(512, 4096, 11008, 148, 0) == 2
     assert P(40, 11008, 4096, 132, room) == 2      # another SM count
     assert P(0, 64, 64, 148, 0) == -1 and P(8, 64, 100, 148, 0) == -1
+    # a few tokens whose rows do not fit the fused GEMV's shared memory
+    assert P(1, 512, 37376, 148, 0) == 0 and P(1, 512, 37440, 148, 0) == 1
+    assert P(4, 200, 18624, 148, 0) == 0 and P(4, 200, 18688, 148, 0) == 1
+    assert lib.bl_linear_workspace_bytes(1, 37376, 512) == 0
+    assert lib.bl_linear_workspace_bytes(1, 37440, 512) >= 37440 + 8
+    assert lib.bl_zero_gemm_workspace_bytes(4, 18688, 200) >= 16
 
 
 def test_workspace_sizes(lib):

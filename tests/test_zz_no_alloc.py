@@ -93,3 +93,18 @@ def test_noalloc_refuses_scratch_beyond_4mib(lib):
     torch.cuda.synchronize()
     assert bool((Y == 7.0).all())  # nothing ran
     assert "workspace" in lib.bl_status_string(BL_ERR_WORKSPACE).decode()
+
+
+def test_noalloc_long_rows():
+    """Three tokens of 25,600 inputs: too long a row for the fused GEMV, so
+    the call takes the quantiser and the warp-level kernel on its fixed
+    scratch, against the oracle."""
+    import oracle
+    import ternary_weight_linear_absmax_b200 as bl
+    from parity_helpers import assert_close
+    M, K, N = 3, 25600, 256
+    codes, g = _oracle_codes(K, N, seed=71)
+    A = si.activations(M, K, seed=72, outliers=True, dtype="bf16")
+    Y = bl.bl_linear_noalloc(A.torch("cuda"), torch.from_numpy(oracle.pack_ternary(codes)).cuda(),
+                             torch.tensor([g], dtype=torch.float32, device="cuda"), EPS)
+    assert_close(Y.float().cpu().numpy(), oracle.bitlinear(A.f32, codes, g, EPS)["Y"], False)
