@@ -344,7 +344,10 @@ bl_status bl_ffn_relu2_taps(const void* X, bl_dtype x_dtype, int64_t M,
  *   bl_linear_radix3: bl_linear for M ≤ bl_gemv_max_tokens() tokens on
  *     radix-3 weights (one fused GEMV launch, same results as bl_linear);
  *     flags: BL_FLAG_PDL as for bl_linear_ex, BL_FLAG_RAW_I32 to write the
- *     INT32 accumulators instead (y_dtype ignored). M > 4: BL_ERR_SHAPE. */
+ *     INT32 accumulators instead (y_dtype ignored). M > 4, or K whose
+ *     weight row and decode tables do not fit in one CTA's shared memory
+ *     (K above 49,728 at 1 token, 30,080 at 2, 21,568 at 3, 16,768 at 4):
+ *     BL_ERR_SHAPE. */
 int64_t bl_radix3_row_bytes(int64_t K);
 bl_status bl_pack_radix3(const uint8_t* W_packed, int64_t N, int64_t K, uint8_t* W_r3,
                          bl_stream_t stream);
