@@ -585,3 +585,19 @@ def test_mixed_pdl_chain_shared_workspace(bl):
         for i, (y, r) in enumerate(zip(chained, alone)):
             assert torch.equal(y, r), f"call {i} {seq[i]} differs when chained"
     assert bl.bl_check_device_error() == 0
+
+
+@pytest.mark.parametrize("M", [1, 2, 16, 100])
+def test_wide_output_sampled(bl, M):
+    """An output as wide as a language-model head (128,256 rows × 2048
+    inputs): every path runs several waves of CTAs over the SMs (GEMV slabs,
+    128-row warp-level slabs, 128-row tensor-core tiles). The matrix repeats
+    one seeded 8192-row block; sampled rows from different repeats, the first
+    and the last are checked bit-exactly against the oracle."""
+    K, N = 2048, 128256
+    codes = np.tile(random_codes(8192, K, seed=99), (N // 8192 + 1, 1))[:N]
+    packed = to_dev(oracle.pack_ternary(codes))
+    Aq = random_int8(M, K, seed=500 + M)
+    acc = bl.bl_zero_gemm(to_dev(Aq), packed).cpu().numpy()
+    rows = [0, 1, 127, 128, 8191, 8192, 65535, 65536, 100000, 128127, N - 2, N - 1]
+    np.testing.assert_array_equal(acc[:, rows], oracle.zero_gemm(Aq, np.ascontiguousarray(codes[rows])))
