@@ -129,7 +129,7 @@ def profiled_traffic():
 TRAFFIC_COMMAND = ("python bench.py --profile-case decode  (then) ncu --metrics "
                    "gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum "
                    "--clock-control none -k regex:gemv_ternary -s 5 -c 5 --csv "
-                   "--log-file gpurun_out/ncu_decode.csv python bench.py --profile-case decode")
+                   "--log-file ncu_decode.csv python bench.py --profile-case decode")
 
 
 def write_traffic_json(csv_path):
